@@ -1,0 +1,459 @@
+"""Benchmark of the QLoRA NF4 linear hot path on B200 (one JSON line on rank 0).
+
+Step (the headline workload): one training-shaped 7B decoder layer's seven
+projections (q 4096x4096, k/v 1024x4096, o 4096x4096, gate/up 14336x4096,
+down 4096x14336) at 8192 tokens, LoRA r = 16, alpha = 32:
+  quantize + double-quantize all seven fp32 weights (one batched call),
+  forward of every projection, backward (dX, dA, dB) of every projection.
+Metric: algorithmic TFLOP/s of the forward + backward,
+  4 M sum(N K) + 6 M r sum(N + K) = 7.211 TFLOP per step per GPU
+(the quantize work is inside the timed step but not counted as FLOPs).
+
+Multi-GPU: one process per GPU (torchrun), each rank runs the same step on
+its own replica (the method has no exchange step on this path), so scaling is
+weak; time is the max over ranks of CUDA-event time.
+
+Also reported on rank 0 (not the headline): quantize and dequantize GB/s over
+the 168 OPT-1.3B-shaped tensors, dequant-GEMV GB/s on the 14336 x 4096 gate
+projection at M = 1, 4, 16 (L2 flushed before every call), the end-to-end
+number with pinned host buffers, and the CPU oracle baseline.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_nf4_quantized_blk_b200 import binding, workloads  # noqa: E402
+
+R = 16
+ALPHA = 32.0
+M_TOKENS = 8192
+METRIC = "QLoRA linear fwd+bwd TFLOP/s @8192 tok; dequant-GEMV & quantize GB/s vs HBM"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def step_flops(M=M_TOKENS, r=R):
+    snk = sum(p.n * p.k for p in workloads.LAYER7B)
+    snpk = sum(p.n + p.k for p in workloads.LAYER7B)
+    return 4 * M * snk + 6 * M * r * snpk
+
+
+def gemm_flops_per_step(M=M_TOKENS, r=R):
+    # forward GEMM: 2 M N (K + r); backward-input GEMM: 2 M K (N + r)
+    return sum(2 * M * p.n * (p.k + r) + 2 * M * p.k * (p.n + r) for p in workloads.LAYER7B)
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_PATH):
+        with open(PEAKS_PATH) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# The layer step
+# ---------------------------------------------------------------------------
+
+class LayerStep:
+    """Resident inputs, outputs and workspaces of one 7B layer step."""
+
+    def __init__(self, device, M=M_TOKENS):
+        self.M = M
+        self.cases = [workloads.layer7b_case(t, m=M, device=device) for t in range(7)]
+        self.outs = [binding.NF4Weight.empty(c.proj.n, c.proj.k, device=device) for c in self.cases]
+        self.qws = torch.empty(binding.qlora_nf4_quantize_batched_ws_bytes(self.outs), dtype=torch.uint8, device=device)
+        self.dstat = torch.zeros(1, dtype=torch.int32, device=device)
+        lws = max(binding.qlora_linear_ws_bytes(M, c.proj.n, c.proj.k, c.r) for c in self.cases)
+        self.lws = torch.empty(lws, dtype=torch.uint8, device=device)
+        binding.qlora_workspace_reset(self.lws)
+        self.Y = [torch.empty((M, c.proj.n), dtype=torch.bfloat16, device=device) for c in self.cases]
+        self.dX = [torch.empty((M, c.proj.k), dtype=torch.bfloat16, device=device) for c in self.cases]
+        self.dA = [torch.empty((c.r, c.proj.k), dtype=torch.float32, device=device) for c in self.cases]
+        self.dB = [torch.empty((c.proj.n, c.r), dtype=torch.float32, device=device) for c in self.cases]
+
+    def run(self):
+        binding.qlora_nf4_quantize_batched([c.W for c in self.cases], self.outs, self.qws, d_status=self.dstat)
+        for c, o, Y in zip(self.cases, self.outs, self.Y):
+            binding.qlora_linear_fwd(o, c.X, c.A, c.B, c.r, c.s, Y, None, self.lws)
+        for c, o, dX, dA, dB in reversed(list(zip(self.cases, self.outs, self.dX, self.dA, self.dB))):
+            binding.qlora_linear_bwd(o, c.X, c.dY, c.A, c.B, c.r, c.s, dX, 0, dA, dB, self.lws)
+
+    def check_status(self):
+        assert self.dstat.item() == 0, "quantize reported non-finite input"
+        st = binding.qlora_workspace_status(self.lws)
+        assert st == 0, f"device status {st}"
+
+    # end-to-end: host buffers in, host buffers out
+    def host_buffers(self):
+        pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+        self.h_in = [(pin(c.W), pin(c.X), pin(c.dY), pin(c.A), pin(c.B)) for c in self.cases]
+        self.h_out = [(torch.empty(y.shape, dtype=y.dtype).pin_memory(), torch.empty(dx.shape, dtype=dx.dtype).pin_memory(),
+                       torch.empty(da.shape, dtype=da.dtype).pin_memory(), torch.empty(db.shape, dtype=db.dtype).pin_memory())
+                      for y, dx, da, db in zip(self.Y, self.dX, self.dA, self.dB)]
+        h2d = sum(sum(t.numel() * t.element_size() for t in grp) for grp in self.h_in)
+        d2h = sum(sum(t.numel() * t.element_size() for t in grp) for grp in self.h_out)
+        return h2d, d2h
+
+    def run_e2e(self):
+        for c, (W, X, dY, A, B) in zip(self.cases, self.h_in):
+            c.W.copy_(W, non_blocking=True)
+            c.X.copy_(X, non_blocking=True)
+            c.dY.copy_(dY, non_blocking=True)
+            c.A.copy_(A, non_blocking=True)
+            c.B.copy_(B, non_blocking=True)
+        self.run()
+        for (y, dx, da, db), Y, dX, dA, dB in zip(self.h_out, self.Y, self.dX, self.dA, self.dB):
+            y.copy_(Y, non_blocking=True)
+            dx.copy_(dX, non_blocking=True)
+            da.copy_(dA, non_blocking=True)
+            db.copy_(dB, non_blocking=True)
+
+
+def timed(fn, steps, warmup, world):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        fn()
+    stop.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(stop) / steps
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    return ms
+
+
+# ---------------------------------------------------------------------------
+# Secondary measurements (rank 0): quantize / dequant / GEMV rows
+# ---------------------------------------------------------------------------
+
+def l2_flush_buffer():
+    size = 2 * torch.cuda.get_device_properties(0).L2_cache_size
+    return torch.empty(max(size, 256 << 20) // 4, dtype=torch.float32, device="cuda")
+
+
+def bench_quantize_dequant(reps=5):
+    items = workloads.opt13b_weight_shapes()
+    Ws = [workloads.opt13b_weight(layer, t, device="cuda") for layer, t, _ in items]
+    outs = [binding.NF4Weight.empty(p.n, p.k) for _, _, p in items]
+    ws = torch.empty(binding.qlora_nf4_quantize_batched_ws_bytes(outs), dtype=torch.uint8, device="cuda")
+    dstat = torch.zeros(1, dtype=torch.int32, device="cuda")
+    n = sum(p.n * p.k for _, _, p in items)
+    q_ms = timed(lambda: binding.qlora_nf4_quantize_batched(Ws, outs, ws, d_status=dstat), reps, 2, 1)
+    assert dstat.item() == 0
+    ys = [torch.empty((p.n, p.k), dtype=torch.bfloat16, device="cuda") for _, _, p in items]
+    d_ms = timed(lambda: binding.qlora_nf4_dequantize_batched(outs, ys, 0), reps, 2, 1)
+    q_bytes = n * (4 + 0.5 + 1 / 64) + 4 * sum(o.c2.numel() + 1 for o in outs)
+    d_bytes = n * (0.5 + 1 / 64 + 2) + 4 * sum(o.c2.numel() + 1 for o in outs)
+    del Ws, ys
+    return {
+        "quantize": {"weights": n, "ms": q_ms, "GB/s": q_bytes / q_ms / 1e6, "bytes_per_weight": 4.5159},
+        "dequant_bf16": {"weights": n, "ms": d_ms, "GB/s": d_bytes / d_ms / 1e6, "bytes_per_weight": 2.5159},
+    }
+
+
+def bench_gemv(reps=50):
+    case = workloads.gemv_case(16, device="cuda")
+    out = binding.NF4Weight.empty(14336, 4096)
+    qws = torch.empty(binding.qlora_nf4_sizes(14336, 4096)["ws_bytes"], dtype=torch.uint8, device="cuda")
+    binding.qlora_nf4_quantize(case.W, out, qws)
+    flush = l2_flush_buffer()
+    res = {}
+    for M in (1, 4, 16):
+        X = workloads.normal_bf16((M, 4096), 1.0, 3000 + M, device="cuda")
+        Y = torch.empty((M, 14336), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(binding.qlora_linear_ws_bytes(M, 14336, 4096, 16), dtype=torch.uint8, device="cuda")
+        binding.qlora_workspace_reset(ws)
+        fwd = lambda: binding.qlora_linear_fwd(out, X, case.A, case.B, 16, case.s, Y, None, ws)  # noqa: E731
+        for _ in range(3):
+            fwd()
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fwd()
+            b.record()
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        nbytes = (out.packed.numel() + out.qscale.numel() + 4 * out.c2.numel() + 4 + 2 * (case.A.numel() + case.B.numel())
+                  + 2 * M * (4096 + 14336))
+        res[f"M={M}"] = {"us": ms * 1e3, "GB/s": nbytes / ms / 1e6, "bytes": nbytes}
+        assert binding.qlora_workspace_status(ws) == 0
+    return res
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(cases_cpu, row_div: int, tokens: int):
+    """Run the oracle on a bounded sample of the layer step and extrapolate.
+
+    Sample: for each projection, quantize + double-quantize + dequantize the
+    first N/row_div rows of the weight, and run the fp64 LoRA forward and
+    backward of `tokens` tokens against that slice.  Each part's time is
+    scaled by the fraction of the full step's work it represents.
+    """
+    from oracle import lora, nf4
+
+    t_quant = 0.0
+    t_lora = 0.0
+    lora_flops = 0.0
+    for c in cases_cpu:
+        n_rows = max(8, c.proj.n // row_div)
+        W = c["W"][:n_rows]
+        t0 = time.perf_counter()
+        st = nf4.quantize_weight(W)
+        Wh = nf4.bf16_bits_to_f32(nf4.dequantize_weight(st, "bf16")).astype(np.float64)
+        t_quant += (time.perf_counter() - t0) * (c.proj.n / n_rows)
+        X, dY, A, B = c["X"][:tokens], c["dY"][:tokens, :n_rows], c["A"], c["B"][:n_rows]
+        t0 = time.perf_counter()
+        lora.lora_forward(X, Wh, A, B, c.s)
+        lora.lora_backward(X, dY, Wh, A, B, c.s)
+        dt = time.perf_counter() - t0
+        f_sample = 4 * tokens * n_rows * c.proj.k + 6 * tokens * R * (n_rows + c.proj.k)
+        f_full = 4 * M_TOKENS * c.proj.n * c.proj.k + 6 * M_TOKENS * R * (c.proj.n + c.proj.k)
+        t_lora += dt * f_full / f_sample
+        lora_flops += f_sample
+    total = t_quant + t_lora
+    return step_flops() / total / 1e12, total
+
+
+class CpuCase(dict):
+    """Host copies of one projection's inputs (first `tokens` token rows only)."""
+
+    def __init__(self, case, tokens):
+        f64 = lambda t: t.float().cpu().numpy().astype(np.float64)  # noqa: E731
+        super().__init__(W=case.W.cpu().numpy(), X=f64(case.X[:tokens]), dY=f64(case.dY[:tokens]),
+                         A=f64(case.A), B=f64(case.B))
+        self.proj = case.proj
+        self.s = case.s
+
+
+def cpu_cases(device, tokens):
+    return [CpuCase(workloads.layer7b_case(t, m=M_TOKENS, device=device), tokens) for t in range(7)]
+
+
+def cores_used():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ---------------------------------------------------------------------------
+# Arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    row_div, tokens = 256, 32
+    cases = cpu_cases("cuda" if torch.cuda.is_available() else "cpu", tokens)
+    for _ in range(args.warmup):
+        oracle_sample_step(cases, row_div, tokens)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, _ = oracle_sample_step(cases, row_div, tokens)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    sample = (f"oracle (numpy, fp64 LoRA) on 1/{row_div} of each weight's rows and {tokens} of {M_TOKENS} tokens "
+              f"per projection, times scaled to the full step")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_flops() / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "7B decoder layer, 7 NF4+DQ projections, 8192 tokens, r=16 alpha=32, quantize+fwd+bwd"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }))
+
+
+def run_ours(args, rank, world, local_rank):
+    from bit_nf4_quantized_blk_b200 import build
+
+    build.build()
+    device = "cuda"
+    peaks, peak_src = load_peaks()
+    step = LayerStep(device)
+    step.run()
+    torch.cuda.synchronize()
+    step.check_status()
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clock = ClockSampler(int(vis.split(",")[local_rank]) if vis and vis.split(",")[0].isdigit() else local_rank)
+    binding.qlora_timing_enable(True)
+    clock.start()
+    ms = timed(step.run, args.steps, args.warmup, world)
+    clocks = clock.stop()
+    fam = {f: binding.qlora_timing_read(f) for f in ("quantize", "dequant", "gemv", "side", "gemm")}
+    binding.qlora_timing_enable(False)
+    step.check_status()
+    launches_total = sum(n for _, n in fam.values())
+    steps_recorded = args.steps + args.warmup
+    gemm_ms, gemm_n = fam["gemm"]
+    gemm_ms_per_step = gemm_ms / steps_recorded
+    gemm_tflops = gemm_flops_per_step() / (gemm_ms_per_step / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+
+    flops = step_flops()
+    value = flops * world / (ms / 1e3) / 1e12
+
+    # end-to-end through host buffers
+    h2d, d2h = step.host_buffers()
+    e2e_ms = timed(step.run_e2e, max(2, args.steps // 4), 1, world)
+    e2e_value = flops * world / (e2e_ms / 1e3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "7B decoder layer, 7 NF4+DQ projections (q 4096x4096, k/v 1024x4096, o 4096x4096, "
+                               "gate/up 14336x4096, down 4096x14336), 8192 tokens, r=16 alpha=32: "
+                               "quantize+DQ, forward, backward (dX, dA, dB)",
+                   "flops_per_step_per_gpu": flops, "l2": "inputs larger than L2 (GBs per step)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_tn_kernel (tcgen05 128x256 tile)",
+                     "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tflops / peak,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": None,
+                     "share_of_step": gemm_ms_per_step / ms},
+        "gpu_launches": int(round(launches_total / steps_recorded * args.steps)),
+        "kernel_ms_per_step": {f: v[0] / steps_recorded for f, v in fam.items()},
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+    }
+    if rank == 0 and not args.no_extras:
+        del step
+        torch.cuda.empty_cache()
+        extras = bench_quantize_dequant()
+        extras["gemv_gate_14336x4096"] = bench_gemv()
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        for k in ("quantize", "dequant_bf16"):
+            extras[k]["frac_hbm"] = extras[k]["GB/s"] / hbm
+        for k, v in extras["gemv_gate_14336x4096"].items():
+            v["frac_hbm"] = v["GB/s"] / hbm
+        extras["hbm_peak_gbs"] = hbm
+        line["secondary"] = extras
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cases = cpu_cases(device, 256)
+        v, t = oracle_sample_step(cases, 32, 256)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+                                "sample": "oracle (numpy; fp64 LoRA) on 1/32 of each weight's rows and 256 of 8192 "
+                                          "tokens per projection, times scaled to the full step",
+                                "extrapolated_step_s": t}
+    if rank == 0:
+        print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

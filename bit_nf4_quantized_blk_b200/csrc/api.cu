@@ -1,0 +1,677 @@
+// C ABI of the QLoRA NF4 library: argument checks, workspace layout and the
+// launch sequences of quantize / dequantize / linear forward / backward.
+//
+// The host never computes any part of the method's results: it checks
+// arguments, carves the caller's workspace and enqueues kernels.  The one
+// table it builds, the decision cells of the nearest-level search, is derived
+// here from the codebook of "QLoRA: NF4 storage, gradients and local
+// integration" (section "Exact CPU teaching quantizer and adapter gradient
+// path") with the same fp32 rule the definition uses.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace qnf4;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Decision table
+// ---------------------------------------------------------------------------
+
+// Nearest level of x by the definition: fp32 distances |x - L_j|, the lowest
+// index wins a tie.  Host fp32 arithmetic (SSE, no contraction) is IEEE.
+int host_nearest(float x) {
+  int best = 0;
+  volatile float bd = std::fabs(x - nf4_level(0));
+  for (int j = 1; j < 16; ++j) {
+    volatile float d = std::fabs(x - nf4_level(j));
+    if (d < bd) {
+      bd = d;
+      best = j;
+    }
+  }
+  return best;
+}
+
+int64_t ordered_key(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return (u >> 31) ? -static_cast<int64_t>(u & 0x7FFFFFFFu) : static_cast<int64_t>(u);
+}
+
+float from_key(int64_t k) {
+  const uint32_t u = k >= 0 ? static_cast<uint32_t>(k) : (0x80000000u | static_cast<uint32_t>(-k));
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+// The 15 decision thresholds: T_j is the smallest fp32 x whose nearest level
+// is j (the choice between neighbouring levels flips once between them).
+void derive_thresholds(float (&T)[16]) {
+  T[0] = -INFINITY;
+  for (int j = 1; j < 16; ++j) {
+    int64_t lo = ordered_key(nf4_level(j - 1)), hi = ordered_key(nf4_level(j));
+    while (hi - lo > 1) {
+      const int64_t mid = lo + (hi - lo) / 2;
+      if (host_nearest(from_key(mid)) >= j) hi = mid; else lo = mid;
+    }
+    T[j] = from_key(hi);
+  }
+}
+
+// Cells of x in [-1, 1] by c = trunc(64 x) + 64; each cell is an interval of
+// fp32 values [xlo, xhi] that holds at most one threshold, so
+// code(x) = base[c] + (x >= thr[c]).  Verified against host_nearest at every
+// cell edge and around every threshold.
+bool build_decision_table(Nf4DecisionTable* tab) {
+  float T[16];
+  derive_thresholds(T);
+  for (int c = 0; c <= 128; ++c) {
+    const int t = c - 64;
+    float xlo, xhi;
+    if (t >= 1) {
+      xlo = static_cast<float>(t) / 64.0f;
+      xhi = t == 64 ? 1.0f : std::nextafter(static_cast<float>(t + 1) / 64.0f, -INFINITY);
+    } else if (t == 0) {
+      xlo = std::nextafter(-1.0f / 64.0f, INFINITY);
+      xhi = std::nextafter(1.0f / 64.0f, -INFINITY);
+    } else {
+      xlo = t == -64 ? -1.0f : std::nextafter(static_cast<float>(t - 1) / 64.0f, INFINITY);
+      xhi = static_cast<float>(t) / 64.0f;
+    }
+    int base = 0, inside = 0;
+    float thr = INFINITY;
+    for (int j = 1; j < 16; ++j) {
+      if (T[j] <= xlo) ++base;
+      else if (T[j] <= xhi) {
+        thr = T[j];
+        ++inside;
+      }
+    }
+    if (inside > 1) return false;
+    tab->thr[c] = thr;
+    tab->base[c] = base;
+    auto code_of = [&](float x) { return base + (x >= thr ? 1 : 0); };
+    if (code_of(xlo) != host_nearest(xlo) || code_of(xhi) != host_nearest(xhi)) return false;
+    if (inside) {
+      if (code_of(thr) != host_nearest(thr)) return false;
+      const float below = std::nextafter(thr, -INFINITY);
+      if (code_of(below) != host_nearest(below)) return false;
+    }
+  }
+  return true;
+}
+
+const Nf4DecisionTable* decision_table() {
+  static Nf4DecisionTable tab;
+  static bool ok = false;
+  static std::once_flag once;
+  std::call_once(once, [] { ok = build_decision_table(&tab); });
+  return ok ? &tab : nullptr;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel timing (instrumentation): CUDA events around each launch family.
+// ---------------------------------------------------------------------------
+
+enum Family { kFamQuant, kFamDequant, kFamGemv, kFamSide, kFamGemm, kFamCount };
+const char* const kFamNames[kFamCount] = {"quantize", "dequant", "gemv", "side", "gemm"};
+
+struct TimingState {
+  bool enabled = false;
+  std::vector<cudaEvent_t> pool;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending[kFamCount];
+  double ms[kFamCount] = {};
+  int64_t launches[kFamCount] = {};
+};
+
+TimingState& timing() {
+  static TimingState t;
+  return t;
+}
+
+cudaEvent_t take_event() {
+  TimingState& T = timing();
+  if (!T.pool.empty()) {
+    cudaEvent_t e = T.pool.back();
+    T.pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets the kernels enqueued during its lifetime with two events.
+class Timed {
+ public:
+  Timed(Family fam, cudaStream_t s, int kernels = 1) : fam_(fam), s_(s), kernels_(kernels) {
+    if (timing().enabled) {
+      start_ = take_event();
+      if (start_ != nullptr) cudaEventRecord(start_, s_);
+    }
+  }
+  ~Timed() {
+    if (start_ == nullptr) return;
+    cudaEvent_t stop = take_event();
+    if (stop == nullptr) return;
+    cudaEventRecord(stop, s_);
+    timing().pending[fam_].push_back({start_, stop});
+    timing().launches[fam_] += kernels_;
+  }
+  Timed(const Timed&) = delete;
+  Timed& operator=(const Timed&) = delete;
+
+ private:
+  Family fam_;
+  cudaStream_t s_;
+  int kernels_;
+  cudaEvent_t start_ = nullptr;
+};
+
+// ---------------------------------------------------------------------------
+// Helpers
+// ---------------------------------------------------------------------------
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+qlora_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+qlora_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  return (major == 10 && minor == 0) ? QLORA_OK : QLORA_ERR_UNSUPPORTED;
+}
+
+qlora_status check_weight(const qlora_nf4_weight* w) {
+  if (w == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (w->rows < 1 || w->cols < kBlock || w->cols % kBlock != 0) return QLORA_ERR_INVALID_ARG;
+  if (w->rows > (int64_t{1} << 40) / w->cols) return QLORA_ERR_UNSUPPORTED;
+  if (!w->packed || !w->qscale || !w->c2 || !w->mu) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(w->packed, 16) || !aligned(w->qscale, 16) || !aligned(w->c2, 4) || !aligned(w->mu, 4))
+    return QLORA_ERR_ALIGNMENT;
+  return QLORA_OK;
+}
+
+int64_t n_chunks_of(int64_t rows, int64_t cols) {
+  const int64_t nb = rows * cols / kBlock;
+  return (nb + kDqBlock - 1) / kDqBlock;
+}
+
+// Quantize workspace: [status 256 B][counters][absmax][chunk sums][chunk exponents]
+struct QuantWs {
+  size_t counters, absmax, sums, exps, total;
+};
+
+QuantWs quant_ws_layout(int count, int64_t chunks) {
+  QuantWs l;
+  size_t off = kWsHeader;
+  l.counters = off;
+  off = align_up(off + sizeof(unsigned) * kMaxQuantBatch, 256);
+  l.absmax = off;
+  off = align_up(off + sizeof(float) * kDqBlock * static_cast<size_t>(chunks), 256);
+  l.sums = off;
+  off = align_up(off + sizeof(double) * static_cast<size_t>(chunks), 256);
+  l.exps = off;
+  off = align_up(off + 2 * sizeof(int) * static_cast<size_t>(chunks), 256);
+  l.total = off;
+  (void)count;
+  return l;
+}
+
+// Largest number of chunks any launch group of a batch holds.
+int64_t max_group_chunks(const qlora_nf4_weight* outs, int32_t count) {
+  int64_t best = 0;
+  for (int32_t g0 = 0; g0 < count; g0 += kMaxQuantBatch) {
+    int64_t c = 0;
+    for (int32_t i = g0; i < count && i < g0 + kMaxQuantBatch; ++i) c += n_chunks_of(outs[i].rows, outs[i].cols);
+    if (c > best) best = c;
+  }
+  return best;
+}
+
+// Linear workspace layout.
+struct LinearWs {
+  size_t wbf, u32, us, uhi, ulo, vs, vhi, vlo, bpad, atpad, part, total;
+};
+
+LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
+  LinearWs l;
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t mr = static_cast<size_t>(M) * kRankPad;
+  l.wbf = take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
+  l.u32 = take(mr * 4);
+  l.us = take(mr * 2);
+  l.uhi = take(mr * 2);
+  l.ulo = take(mr * 2);
+  l.vs = take(mr * 2);
+  l.vhi = take(mr * 2);
+  l.vlo = take(mr * 2);
+  l.bpad = take(static_cast<size_t>(N) * kRankPad * 2);
+  l.atpad = take(static_cast<size_t>(K) * kRankPad * 2);
+  const size_t p1 = colsum_partial_bytes(M, N), p2 = colsum_partial_bytes(M, K);
+  l.part = take(p1 > p2 ? p1 : p2);
+  l.total = off;
+  return l;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+WeightView view_of(const qlora_nf4_weight* w) {
+  return WeightView{w->packed, w->qscale, w->c2, w->mu, w->rows, w->cols};
+}
+
+qlora_status check_linear_args(const qlora_nf4_weight* w, int64_t M, int32_t r, size_t ws_bytes, const void* ws) {
+  qlora_status st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  if (M < 1 || r < 1 || r > kMaxRank) return QLORA_ERR_INVALID_ARG;
+  if (w->rows % 8 != 0) return QLORA_ERR_INVALID_ARG;
+  if (M > (int64_t{1} << 31) / kRankPad) return QLORA_ERR_UNSUPPORTED;
+  if (ws == nullptr || !aligned(ws, 256)) return ws == nullptr ? QLORA_ERR_WORKSPACE : QLORA_ERR_ALIGNMENT;
+  if (ws_bytes < linear_ws_layout(M, w->rows, w->cols).total) return QLORA_ERR_WORKSPACE;
+  return QLORA_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// Exported entry points
+// ===========================================================================
+
+extern "C" const char* qlora_status_string(qlora_status status) {
+  switch (status) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_ALIGNMENT: return "misaligned pointer";
+    case QLORA_ERR_NONFINITE: return "non-finite value in the weight";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_TIMEOUT: return "device-side wait timed out";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported device or size";
+  }
+  return "unknown status";
+}
+
+extern "C" qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, size_t* packed_bytes, size_t* n_blocks,
+                                        size_t* n_chunks, size_t* ws_bytes) {
+  if (rows < 1 || cols < kBlock || cols % kBlock != 0) return QLORA_ERR_INVALID_ARG;
+  if (rows > (int64_t{1} << 40) / cols) return QLORA_ERR_UNSUPPORTED;
+  const int64_t n = rows * cols;
+  if (packed_bytes) *packed_bytes = static_cast<size_t>(n / 2);
+  if (n_blocks) *n_blocks = static_cast<size_t>(n / kBlock);
+  if (n_chunks) *n_chunks = static_cast<size_t>(n_chunks_of(rows, cols));
+  if (ws_bytes) *ws_bytes = quant_ws_layout(1, n_chunks_of(rows, cols)).total;
+  return QLORA_OK;
+}
+
+extern "C" size_t qlora_nf4_quantize_batched_ws_bytes(const qlora_nf4_weight* outs, int32_t count) {
+  if (outs == nullptr || count < 1) return 0;
+  for (int32_t i = 0; i < count; ++i)
+    if (outs[i].rows < 1 || outs[i].cols < kBlock || outs[i].cols % kBlock != 0) return 0;
+  return quant_ws_layout(count, max_group_chunks(outs, count)).total;
+}
+
+extern "C" qlora_status qlora_nf4_quantize_batched(const float* const* W, const qlora_nf4_weight* outs, int32_t count,
+                                                   void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (W == nullptr || outs == nullptr || count < 1) return QLORA_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < count; ++i) {
+    const qlora_status st = check_weight(&outs[i]);
+    if (st != QLORA_OK) return st;
+    if (W[i] == nullptr) return QLORA_ERR_INVALID_ARG;
+    if (!aligned(W[i], 32)) return QLORA_ERR_ALIGNMENT;
+  }
+  if (ws == nullptr) return QLORA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
+  const QuantWs lay = quant_ws_layout(count, max_group_chunks(outs, count));
+  if (ws_bytes < lay.total) return QLORA_ERR_WORKSPACE;
+  if (d_status != nullptr && !aligned(d_status, 4)) return QLORA_ERR_ALIGNMENT;
+  qlora_status st = check_device();
+  if (st != QLORA_OK) return st;
+  const Nf4DecisionTable* tab = decision_table();
+  if (tab == nullptr) return QLORA_ERR_UNSUPPORTED;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = d_status != nullptr ? d_status : at<int>(ws, 0);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e != cudaSuccess) return from_cuda(e);
+
+  QuantBatchParams p;
+  for (int32_t g0 = 0; g0 < count; g0 += kMaxQuantBatch) {
+    std::memset(&p, 0, sizeof(p));
+    const int n = (count - g0 < kMaxQuantBatch) ? count - g0 : kMaxQuantBatch;
+    p.count = n;
+    int64_t c = 0;
+    for (int i = 0; i < n; ++i) {
+      const qlora_nf4_weight& o = outs[g0 + i];
+      p.chunk_begin[i] = c;
+      p.n_blocks[i] = o.rows * o.cols / kBlock;
+      p.W[i] = W[g0 + i];
+      p.packed[i] = o.packed;
+      p.qscale[i] = o.qscale;
+      p.c2[i] = o.c2;
+      p.mu[i] = o.mu;
+      c += n_chunks_of(o.rows, o.cols);
+    }
+    p.chunk_begin[n] = c;
+    p.total_chunks = c;
+    p.absmax = at<float>(ws, lay.absmax);
+    p.chunk_sum = at<double>(ws, lay.sums);
+    p.chunk_exp = at<int>(ws, lay.exps);
+    p.counters = at<unsigned>(ws, lay.counters);
+    p.status = status;
+    p.table = *tab;
+    e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * kMaxQuantBatch, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    {
+      Timed tm(kFamQuant, s, 2);
+      e = launch_quantize_batch(p, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  if (d_status != nullptr) return QLORA_OK;
+  int32_t h = 0;
+  e = cudaMemcpyAsync(&h, status, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return from_cuda(e);
+  return static_cast<qlora_status>(h);
+}
+
+extern "C" qlora_status qlora_nf4_quantize(const float* W, const qlora_nf4_weight* out, void* ws, size_t ws_bytes,
+                                           int32_t* d_status, void* stream) {
+  if (out == nullptr) return QLORA_ERR_INVALID_ARG;
+  const float* const ws_list[1] = {W};
+  return qlora_nf4_quantize_batched(ws_list, out, 1, ws, ws_bytes, d_status, stream);
+}
+
+extern "C" qlora_status qlora_nf4_dequantize_batched(const qlora_nf4_weight* weights, void* const* outs, int32_t count,
+                                                     int32_t out_dtype, void* stream) {
+  if (weights == nullptr || outs == nullptr || count < 1) return QLORA_ERR_INVALID_ARG;
+  if (out_dtype != 0 && out_dtype != 1) return QLORA_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < count; ++i) {
+    const qlora_status st = check_weight(&weights[i]);
+    if (st != QLORA_OK) return st;
+    if (outs[i] == nullptr) return QLORA_ERR_INVALID_ARG;
+    if (!aligned(outs[i], 16)) return QLORA_ERR_ALIGNMENT;
+  }
+  qlora_status st = check_device();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DequantBatchParams p;
+  for (int32_t g0 = 0; g0 < count; g0 += kMaxDequantBatch) {
+    std::memset(&p, 0, sizeof(p));
+    const int n = (count - g0 < kMaxDequantBatch) ? count - g0 : kMaxDequantBatch;
+    p.count = n;
+    int64_t c = 0;
+    for (int i = 0; i < n; ++i) {
+      const qlora_nf4_weight& w = weights[g0 + i];
+      p.begin16[i] = c;
+      p.packed[i] = w.packed;
+      p.qscale[i] = w.qscale;
+      p.c2[i] = w.c2;
+      p.mu[i] = w.mu;
+      p.out[i] = outs[g0 + i];
+      c += w.rows * w.cols / 32;
+    }
+    p.begin16[n] = c;
+    p.total16 = c;
+    cudaError_t e;
+    {
+      Timed tm(kFamDequant, s);
+      e = launch_dequant_batch(p, out_dtype, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return QLORA_OK;
+}
+
+extern "C" qlora_status qlora_nf4_dequantize(const qlora_nf4_weight* w, void* out, int32_t out_dtype,
+                                             int32_t transpose, void* stream) {
+  if (transpose != 0 && transpose != 1) return QLORA_ERR_INVALID_ARG;
+  if (!transpose) {
+    void* const outs[1] = {out};
+    return qlora_nf4_dequantize_batched(w, outs, 1, out_dtype, stream);
+  }
+  qlora_status st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  if (out == nullptr || out_dtype != 0) return QLORA_ERR_INVALID_ARG;
+  if (w->rows % 8 != 0) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return QLORA_ERR_ALIGNMENT;
+  st = check_device();
+  if (st != QLORA_OK) return st;
+  Timed tm(kFamDequant, static_cast<cudaStream_t>(stream));
+  return from_cuda(launch_dequant_transposed(view_of(w), static_cast<uint16_t*>(out), static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (M < 1 || N < 1 || K < kBlock || K % kBlock != 0 || r < 1 || r > kMaxRank) return 0;
+  return linear_ws_layout(M, N, K).total;
+}
+
+extern "C" qlora_status qlora_workspace_reset(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < kWsHeader) return QLORA_ERR_WORKSPACE;
+  return from_cuda(cudaMemsetAsync(ws, 0, kWsHeader, static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" qlora_status qlora_workspace_status(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < kWsHeader) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return from_cuda(e);
+  return static_cast<qlora_status>(h);
+}
+
+extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
+                                         const uint16_t* B, int32_t r, float scale, uint16_t* Y, uint16_t* U_out,
+                                         void* ws, size_t ws_bytes, void* stream) {
+  qlora_status st = check_linear_args(w, M, r, ws_bytes, ws);
+  if (st != QLORA_OK) return st;
+  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) || (U_out && !aligned(U_out, 2)))
+    return QLORA_ERR_ALIGNMENT;
+  if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
+  st = check_device();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t N = w->rows, K = w->cols;
+  const LinearWs lay = linear_ws_layout(M, N, K);
+  int* status = at<int>(ws, 0);
+  cudaError_t e;
+  if (M <= kGemvMaxM) {
+    {
+      Timed tm(kFamSide, s);
+      e = launch_small_xa(X, A, static_cast<int>(M), static_cast<int>(K), r, at<float>(ws, lay.u32), U_out, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+    Timed tm(kFamGemv, s);
+    return from_cuda(launch_gemv(view_of(w), X, static_cast<int>(M), B, r, scale, at<float>(ws, lay.u32), Y, s));
+  }
+  // Tensor-core path: dense bf16 weight, U = X A^T, padded B, GEMM with the rank-r step.
+  DequantBatchParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.count = 1;
+  p.begin16[1] = p.total16 = N * K / 32;
+  p.packed[0] = w->packed;
+  p.qscale[0] = w->qscale;
+  p.c2[0] = w->c2;
+  p.mu[0] = w->mu;
+  p.out[0] = at<uint16_t>(ws, lay.wbf);
+  {
+    Timed tm(kFamDequant, s);
+    e = launch_dequant_batch(p, 0, s);
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  SkinnyOut so{};
+  so.os = at<uint16_t>(ws, lay.us);
+  so.obf = U_out;
+  so.scale = scale;
+  {
+    Timed tm(kFamSide, s, 2);
+    e = launch_skinny(X, M, K, A, true, r, so, s);
+    if (e == cudaSuccess) e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  GemmArgs g{};
+  g.A = X;
+  g.B = at<uint16_t>(ws, lay.wbf);
+  g.A2 = at<uint16_t>(ws, lay.us);
+  g.B2 = at<uint16_t>(ws, lay.bpad);
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.r = r;
+  g.D = Y;
+  g.accumulate = 0;
+  g.status = status;
+  Timed tm(kFamGemm, s);
+  return from_cuda(launch_gemm_tn(g, s));
+}
+
+extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,
+                                         const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* dX,
+                                         int32_t accumulate, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  qlora_status st = check_linear_args(w, M, r, ws_bytes, ws);
+  if (st != QLORA_OK) return st;
+  if (!X || !dY || !A || !B) return QLORA_ERR_INVALID_ARG;
+  if (accumulate != 0 && accumulate != 1) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(dY, 16) || !aligned(A, 16) || !aligned(B, 2) || (dX && !aligned(dX, 16)) ||
+      (dA && !aligned(dA, 4)) || (dB && !aligned(dB, 4)))
+    return QLORA_ERR_ALIGNMENT;
+  if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
+  st = check_device();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t N = w->rows, K = w->cols;
+  const LinearWs lay = linear_ws_layout(M, N, K);
+  int* status = at<int>(ws, 0);
+  cudaError_t e;
+
+  // V = dY B (bf16 s*V for the dX rank step; hi/lo split for dA).
+  SkinnyOut vo{};
+  vo.os = at<uint16_t>(ws, lay.vs);
+  vo.ohi = at<uint16_t>(ws, lay.vhi);
+  vo.olo = at<uint16_t>(ws, lay.vlo);
+  vo.scale = scale;
+  {
+    Timed tm(kFamSide, s, 2);
+    e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
+    if (e == cudaSuccess) e = launch_skinny(dY, M, N, at<uint16_t>(ws, lay.bpad), false, r, vo, s);
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+
+  if (dB != nullptr) {  // dB = s dY^T U with U = X A^T
+    SkinnyOut uo{};
+    uo.ohi = at<uint16_t>(ws, lay.uhi);
+    uo.olo = at<uint16_t>(ws, lay.ulo);
+    uo.scale = 1.0f;
+    {
+      Timed tm(kFamSide, s, 3);
+      e = launch_skinny(X, M, K, A, true, r, uo, s);
+      if (e == cudaSuccess)
+        e = launch_colsum(dY, M, N, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), r, scale,
+                          at<float>(ws, lay.part), dB, false, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  if (dX != nullptr) {  // dX = dY W_hat + s V A
+    {
+      Timed tm(kFamDequant, s);
+      e = launch_dequant_transposed(view_of(w), at<uint16_t>(ws, lay.wbf), s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+    {
+      Timed tm(kFamSide, s);
+      e = launch_pad_rank(A, true, K, r, at<uint16_t>(ws, lay.atpad), s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+    GemmArgs g{};
+    g.A = dY;
+    g.B = at<uint16_t>(ws, lay.wbf);
+    g.A2 = at<uint16_t>(ws, lay.vs);
+    g.B2 = at<uint16_t>(ws, lay.atpad);
+    g.M = M;
+    g.N = K;
+    g.K = N;
+    g.r = r;
+    g.D = dX;
+    g.accumulate = accumulate;
+    g.status = status;
+    {
+      Timed tm(kFamGemm, s);
+      e = launch_gemm_tn(g, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  if (dA != nullptr) {  // dA = s V^T X
+    {
+      Timed tm(kFamSide, s, 2);
+      e = launch_colsum(X, M, K, at<uint16_t>(ws, lay.vhi), at<uint16_t>(ws, lay.vlo), r, scale,
+                        at<float>(ws, lay.part), dA, true, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return QLORA_OK;
+}
+
+extern "C" qlora_status qlora_timing_enable(int32_t enable) {
+  TimingState& T = timing();
+  if (enable) {
+    for (int f = 0; f < kFamCount; ++f) {
+      for (auto& pr : T.pending[f]) {
+        T.pool.push_back(pr.first);
+        T.pool.push_back(pr.second);
+      }
+      T.pending[f].clear();
+      T.ms[f] = 0.0;
+      T.launches[f] = 0;
+    }
+  }
+  T.enabled = enable != 0;
+  return QLORA_OK;
+}
+
+extern "C" qlora_status qlora_timing_read(const char* family, double* total_ms, int64_t* launches) {
+  if (family == nullptr) return QLORA_ERR_INVALID_ARG;
+  int f = -1;
+  for (int i = 0; i < kFamCount; ++i)
+    if (std::strcmp(family, kFamNames[i]) == 0) f = i;
+  if (f < 0) return QLORA_ERR_INVALID_ARG;
+  TimingState& T = timing();
+  for (auto& pr : T.pending[f]) {
+    float ms = 0.0f;
+    cudaError_t e = cudaEventSynchronize(pr.second);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pr.first, pr.second);
+    if (e != cudaSuccess) return from_cuda(e);
+    T.ms[f] += ms;
+    T.pool.push_back(pr.first);
+    T.pool.push_back(pr.second);
+  }
+  T.pending[f].clear();
+  if (total_ms) *total_ms = T.ms[f];
+  if (launches) *launches = T.launches[f];
+  return QLORA_OK;
+}

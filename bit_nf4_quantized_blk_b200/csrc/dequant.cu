@@ -1,0 +1,141 @@
+// NF4 + double-quant dequantization to dense bf16 / fp32 (sm_100a).
+//
+// Method: "QLoRA Deep Dive: 4-bit NormalFloat & Double Quantization
+// Internals", section "The Quantization Process in QLoRA" (load the 4-bit
+// codes and the block constant, multiply, cast to bf16); "QLoRA: NF4 storage,
+// gradients and local integration", ``dequantize_nf4`` of the teaching
+// program.  Block scale decode a = fp32(fp32(fp32(q/127) * c2) + mu); weight
+// fp32(L[code] * a); bf16 output rounds that value to nearest even.
+//
+// HBM-bound: 0.5 B of codes + 1/64 B of scale codes read and 2 B (bf16) or
+// 4 B (fp32) written per weight.  Each thread owns 16 packed bytes (half a
+// block, one 128-bit load) and writes 64 / 128 contiguous output bytes.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace qnf4 {
+
+namespace {
+
+__device__ __forceinline__ void fill_pair_table(float2* tab) {
+  for (int b = threadIdx.x; b < 256; b += blockDim.x) tab[b] = make_float2(nf4_level(b & 15), nf4_level(b >> 4));
+}
+
+}  // namespace
+
+__device__ __forceinline__ int find_tensor16(const DequantBatchParams& p, int64_t chunk) {
+  int lo = 0, hi = p.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.begin16[mid] <= chunk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <bool kFp32>
+__global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ DequantBatchParams p) {
+  __shared__ float2 s_pair[256];
+  fill_pair_table(s_pair);
+  __syncthreads();
+  const int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // 16-byte chunk index
+  if (gi >= p.total16) return;
+  const int t = find_tensor16(p, gi);
+  const int64_t i = gi - p.begin16[t];
+  const int64_t blk = i >> 1;  // two chunks per 64-weight block
+  const float a = decode_scale(p.qscale[t][blk], p.c2[t][blk / kDqBlock], *p.mu[t]);
+  const uint4 pk = ld_stream_u4(p.packed[t] + i * 16);
+  const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+  if constexpr (kFp32) {
+    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out[t]) + i * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float vals[8];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float2 lv = s_pair[(words[q] >> (8 * b)) & 0xFF];
+        vals[2 * b] = __fmul_rn(lv.x, a);
+        vals[2 * b + 1] = __fmul_rn(lv.y, a);
+      }
+      st_stream_u4(o + 2 * q, make_uint4(__float_as_uint(vals[0]), __float_as_uint(vals[1]), __float_as_uint(vals[2]),
+                                         __float_as_uint(vals[3])));
+      st_stream_u4(o + 2 * q + 1, make_uint4(__float_as_uint(vals[4]), __float_as_uint(vals[5]),
+                                             __float_as_uint(vals[6]), __float_as_uint(vals[7])));
+    }
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[t]) + i * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t pr[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float2 lv = s_pair[(words[q] >> (8 * b)) & 0xFF];
+        pr[b] = pack_bf16x2(__fmul_rn(lv.x, a), __fmul_rn(lv.y, a));
+      }
+      st_stream_u4(o + q, make_uint4(pr[0], pr[1], pr[2], pr[3]));
+    }
+  }
+}
+
+// Transposed bf16 output out[k][n] = W_hat[n][k]: one CTA per 64 x 64 tile
+// (exactly one block per row of the tile), staged through shared memory.
+__global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, uint16_t* __restrict__ out) {
+  __shared__ float2 s_pair[256];
+  __shared__ __align__(16) uint16_t s_t[64][64];  // [k][n]
+  fill_pair_table(s_pair);
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 64;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * 64;
+  const int tid = threadIdx.x;
+  const int nn = tid & 63;         // row of the weight tile
+  const int kq = (tid >> 6) * 16;  // 16 weights of that row
+  const int64_t n = n0 + nn;
+  __syncthreads();
+  uint32_t lo = 0, hi = 0;
+  float a = 0.0f;
+  if (n < w.rows) {
+    const int64_t blk = (n * w.cols + k0) / kBlock;
+    a = decode_scale(w.qscale[blk], w.c2[blk / kDqBlock], *w.mu);
+    const uint2 pk = *reinterpret_cast<const uint2*>(w.packed + (n * w.cols + k0 + kq) / 2);
+    lo = pk.x;
+    hi = pk.y;
+  }
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    const uint32_t byte = ((b < 4 ? lo : hi) >> (8 * (b & 3))) & 0xFF;
+    const float2 lv = s_pair[byte];
+    const uint32_t pr = pack_bf16x2(__fmul_rn(lv.x, a), __fmul_rn(lv.y, a));
+    s_t[kq + 2 * b][nn] = static_cast<uint16_t>(pr & 0xFFFF);
+    s_t[kq + 2 * b + 1][nn] = static_cast<uint16_t>(pr >> 16);
+  }
+  __syncthreads();
+  const int kk = tid >> 2;        // output row within the tile
+  const int nc = (tid & 3) * 16;  // 16 outputs of that row
+  const int64_t k = k0 + kk;
+  if (k >= w.cols) return;
+  uint16_t* dst = out + k * w.rows + n0 + nc;
+  if (n0 + nc + 16 <= w.rows) {
+    const uint4* src = reinterpret_cast<const uint4*>(&s_t[kk][nc]);
+    reinterpret_cast<uint4*>(dst)[0] = src[0];
+    reinterpret_cast<uint4*>(dst)[1] = src[1];
+  } else {
+    for (int j = 0; j < 16; ++j)
+      if (n0 + nc + j < w.rows) dst[j] = s_t[kk][nc + j];
+  }
+}
+
+cudaError_t launch_dequant_batch(const DequantBatchParams& p, int out_fp32, cudaStream_t stream) {
+  if (p.total16 <= 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((p.total16 + 255) / 256);
+  if (out_fp32)
+    dequant_kernel<true><<<grid, 256, 0, stream>>>(p);
+  else
+    dequant_kernel<false><<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_transposed(const WeightView& w, uint16_t* out, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>(w.cols / 64), static_cast<unsigned>((w.rows + 63) / 64));
+  dequant_transposed_kernel<<<grid, 256, 0, stream>>>(w, out);
+  return cudaGetLastError();
+}
+
+}  // namespace qnf4

@@ -1,0 +1,132 @@
+// Kernel parameter blocks and host-side launchers shared by the library's
+// translation units.
+#pragma once
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+// ---------------------------------------------------------------------------
+// Quantize + double quantize (quantize.cu)
+// ---------------------------------------------------------------------------
+
+constexpr int kMaxQuantBatch = 128;  // tensors per launch (kernel parameter block)
+
+struct QuantBatchParams {
+  int count;
+  int64_t total_chunks;
+  int64_t chunk_begin[kMaxQuantBatch + 1];  // prefix sums of chunks per tensor
+  int64_t n_blocks[kMaxQuantBatch];
+  const float* W[kMaxQuantBatch];
+  uint8_t* packed[kMaxQuantBatch];
+  int8_t* qscale[kMaxQuantBatch];
+  float* c2[kMaxQuantBatch];
+  float* mu[kMaxQuantBatch];
+  // workspace
+  float* absmax;        // [total_chunks * 256] first-level scales, slot per chunk
+  double* chunk_sum;    // [total_chunks]
+  int* chunk_exp;       // [2 * total_chunks] min / max exponent field per chunk
+  unsigned* counters;   // [count], zero on entry
+  int* status;          // device status word, zero on entry
+  Nf4DecisionTable table;
+};
+
+cudaError_t launch_quantize_batch(const QuantBatchParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// Dequantize (dequant.cu)
+// ---------------------------------------------------------------------------
+
+struct WeightView {
+  const uint8_t* packed;
+  const int8_t* qscale;
+  const float* c2;
+  const float* mu;
+  int64_t rows, cols;
+};
+
+constexpr int kMaxDequantBatch = 128;
+
+struct DequantBatchParams {
+  int count;
+  int64_t total16;                          // 16-byte packed chunks in the batch
+  int64_t begin16[kMaxDequantBatch + 1];    // prefix sums of chunks per tensor
+  const uint8_t* packed[kMaxDequantBatch];
+  const int8_t* qscale[kMaxDequantBatch];
+  const float* c2[kMaxDequantBatch];
+  const float* mu[kMaxDequantBatch];
+  void* out[kMaxDequantBatch];
+};
+
+cudaError_t launch_dequant_batch(const DequantBatchParams& p, int out_fp32, cudaStream_t stream);
+cudaError_t launch_dequant_transposed(const WeightView& w, uint16_t* out, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// Decode-shaped dequant-GEMV (gemv.cu), M <= 16
+// ---------------------------------------------------------------------------
+
+constexpr int kGemvMaxM = 16;
+
+// U[m][j] = sum_k X[m][k] * A[j][k] in fp32 for m < M <= 16 (written to
+// U32 [M][kRankPad]); optionally the bf16 copy U_out [M][r].
+cudaError_t launch_small_xa(const uint16_t* X, const uint16_t* A, int M, int K, int r, float* U32,
+                            uint16_t* U_out, cudaStream_t stream);
+// Y[m][n] = sum_k X[m][k] W[n][k] + s * sum_j U32[m][j] B[n][j].
+cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, int M, const uint16_t* B, int r, float scale,
+                        const float* U32, uint16_t* Y, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// Skinny LoRA side products (lora_side.cu)
+// ---------------------------------------------------------------------------
+
+// out[m][j] = sum_c In[m][c] * Wt(j, c) for j < r, with Wt(j, c) = Wr[j][c]
+// (row layout [r, C]) or Wc[c][j] (column layout [C, r]).  Writes
+//   o32   [M][64] fp32 (columns >= r zero)          (may be null)
+//   os    [M][64] bf16 of scale * out, zero padded   (may be null)
+//   ohi / olo [M][64] bf16 split of out (hi + lo ~ fp32) (may be null)
+//   obf   [M][r] bf16 of out                         (may be null)
+struct SkinnyOut {
+  float* o32;
+  uint16_t* os;
+  uint16_t* ohi;
+  uint16_t* olo;
+  uint16_t* obf;
+  float scale;
+};
+cudaError_t launch_skinny(const uint16_t* In, int64_t M, int64_t C, const uint16_t* Wt, bool wt_is_rc, int r,
+                          const SkinnyOut& out, cudaStream_t stream);
+
+// Column sums over tokens: out(c, j) = scale * sum_m In[m][c] * (hi[m][j] + lo[m][j]).
+// part: [ms][C][64] fp32 partials; then written to dst as [C][r] (dst_rc = false)
+// or [r][C] (dst_rc = true).
+int colsum_splits(int64_t M, int64_t C);
+size_t colsum_partial_bytes(int64_t M, int64_t C);
+cudaError_t launch_colsum(const uint16_t* In, int64_t M, int64_t C, const uint16_t* hi, const uint16_t* lo, int r,
+                          float scale, float* part, float* dst, bool dst_rc, cudaStream_t stream);
+
+// Copy a bf16 [rows][r] matrix into [rows][64] zero padded, optionally from
+// the transposed source [r][rows].
+cudaError_t launch_pad_rank(const uint16_t* src, bool src_transposed, int64_t rows, int r, uint16_t* dst,
+                            cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// tcgen05 GEMM (gemm_tc.cu):  D[M][N] (+)= A[M][K] B[N][K]^T + A2[M][64] B2[N][64]^T
+// ---------------------------------------------------------------------------
+struct GemmArgs {
+  const uint16_t* A;
+  const uint16_t* B;
+  const uint16_t* A2;  // may be null (no extra rank product)
+  const uint16_t* B2;
+  int64_t M, N, K;
+  int r;               // rank of the extra product (<= 64)
+  uint16_t* D;
+  int accumulate;      // D += ... instead of D = ...
+  int* status;
+};
+cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream);
+
+// Driver entry point used to encode TMA descriptors (resolved once).
+bool encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                          uint32_t box_cols);
+
+}  // namespace qnf4

@@ -1,0 +1,212 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) QLoRA NF4 linear library.
+ *
+ * The library implements the hot path of a QLoRA linear layer:
+ *
+ *   1. NF4 blockwise quantization of a frozen fp32 weight W0 [rows, cols]
+ *      (absolute maximum per block of 64 consecutive weights of the row-major
+ *      flattening, nearest of the 16 NF4 levels, two 4-bit codes per byte with
+ *      the even element in the low nibble).
+ *      Source: "QLoRA: NF4 storage, gradients and local integration",
+ *      sections "NF4: nonuniform reconstruction levels" and "Exact CPU
+ *      teaching quantizer and adapter gradient path".
+ *   2. Double quantization of the fp32 block scales: a per-tensor fp32 mean
+ *      offset, int8 codes in chunks of 256 scales, one fp32 second-level
+ *      absmax per chunk (about 4.127 bits per weight in total).
+ *      Source: same page, section "Double quantization: correct the scale
+ *      arithmetic"; "QLoRA Deep Dive: 4-bit NormalFloat & Double Quantization
+ *      Internals", section "2. Squeezing More Memory: Double Quantization (DQ)".
+ *   3. Dequantization to bf16 or fp32, and the LoRA linear forward and backward
+ *         Y  = X W^T + s (X A^T) B^T
+ *         dX = dY W + s (dY B) A,  dA = s (dY B)^T X,  dB = s dY^T (X A^T)
+ *      with W the dequantized weight.
+ *      Source: "QLoRA: NF4 storage, gradients and local integration", the
+ *      gradient paragraph after the teaching program; "FT-02: QLoRA --
+ *      Fine-Tuning with Quantization", section "4. The LoRA mechanics the API
+ *      wraps" (LoRALinear, scaling = alpha / r).
+ *
+ * Conventions for every entry point:
+ *   - Every pointer argument except host descriptor structs points to DEVICE
+ *     memory owned by the caller.  The library allocates and frees nothing;
+ *     scratch space is a caller-provided workspace whose size the matching
+ *     *_ws_bytes function returns.
+ *   - bf16 tensors are passed as uint16_t bit patterns, row-major.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued on it and the call returns without waiting, except where a
+ *     status must be read back (see qlora_nf4_quantize).
+ *   - Alignment: fp32 weights to quantize 32 bytes; packed codes, scale codes,
+ *     bf16 activations and outputs 16 bytes; fp32 scalars and gradients 4.
+ *     A misaligned pointer returns QLORA_ERR_ALIGNMENT.
+ *   - Argument checks run on the host before anything is enqueued; a failed
+ *     check returns an error status and enqueues nothing.
+ *   - A CUDA launch or runtime error is returned as QLORA_ERR_CUDA.
+ *   - Calls that share a workspace must not run concurrently on the GPU.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qlora_status {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, bad rank, bad dtype  */
+  QLORA_ERR_ALIGNMENT = 2,    /* a device pointer is not 16-byte aligned      */
+  QLORA_ERR_NONFINITE = 3,    /* the weight to quantize holds NaN or Inf      */
+  QLORA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required   */
+  QLORA_ERR_CUDA = 5,         /* a CUDA runtime/launch error                  */
+  QLORA_ERR_TIMEOUT = 6,      /* a device-side wait ran past its time limit   */
+  QLORA_ERR_UNSUPPORTED = 7   /* no sm_100 device, or a size beyond limits    */
+} qlora_status;
+
+/*
+ * One quantized tensor.  The struct itself lives in host memory; its pointers
+ * are device memory owned by the caller.
+ *   rows, cols : W0 is [rows, cols] row-major (rows = d_out, cols = d_in);
+ *                cols must be a multiple of 64 so every block lies in one row.
+ *   packed     : rows*cols/2 bytes; byte i holds code 2i (low nibble) and
+ *                code 2i+1 (high nibble).
+ *   qscale     : rows*cols/64 int8 scale codes in [-127, 127], one per block.
+ *   c2         : ceil(rows*cols/16384) fp32 second-level scales, one per chunk
+ *                of 256 consecutive blocks.
+ *   mu         : one fp32, the per-tensor mean of the block absmax values.
+ * The block scale is decoded as a = fp32(fp32(fp32(q/127)*c2) + mu) and the
+ * weight as fp32(L[code] * a) (bf16 outputs round that to nearest even).
+ */
+typedef struct qlora_nf4_weight {
+  int64_t rows;
+  int64_t cols;
+  uint8_t *packed;
+  int8_t *qscale;
+  float *c2;
+  float *mu;
+} qlora_nf4_weight;
+
+/* Human-readable name of a status code (static string). */
+const char *qlora_status_string(qlora_status status);
+
+/*
+ * Sizes of the quantized state of a [rows, cols] tensor and the workspace
+ * qlora_nf4_quantize needs for it.  Any output pointer may be NULL.
+ * Errors: INVALID_ARG if rows < 1, cols < 64 or cols % 64 != 0.
+ */
+qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, size_t *packed_bytes, size_t *n_blocks,
+                             size_t *n_chunks, size_t *ws_bytes);
+
+/*
+ * Quantize + double-quantize one fp32 tensor W [out->rows, out->cols]
+ * (steps: block absmax, normalisation, nearest NF4 level, packing, mean
+ * offset, second-level absmax per 256-block chunk, int8 scale codes).
+ * Results are bit-identical to the definition: fp32 IEEE division and
+ * comparisons, fp64 strictly sequential mean (per chunk, then over chunks).
+ *   W        : device fp32 input, not modified.
+ *   out      : host struct describing the caller's output buffers.
+ *   ws       : device workspace of at least qlora_nf4_sizes(...).ws_bytes.
+ *   d_status : device int32 or NULL.  If non-NULL the call does not wait: the
+ *              device writes 0 or QLORA_ERR_NONFINITE there when the work
+ *              completes.  If NULL the call synchronizes `stream` and returns
+ *              QLORA_ERR_NONFINITE itself when W holds NaN/Inf (the outputs are
+ *              then unspecified).
+ */
+qlora_status qlora_nf4_quantize(const float *W, const qlora_nf4_weight *out, void *ws, size_t ws_bytes,
+                                int32_t *d_status, void *stream);
+
+/*
+ * Quantize `count` independent tensors in one pass (same per-tensor results
+ * as qlora_nf4_quantize on each; every tensor has its own mean offset).
+ *   W    : host array of `count` device pointers.
+ *   outs : host array of `count` descriptors.
+ *   ws   : at least qlora_nf4_quantize_batched_ws_bytes(...) bytes.
+ *   d_status, stream : as qlora_nf4_quantize (one status for the batch).
+ */
+size_t qlora_nf4_quantize_batched_ws_bytes(const qlora_nf4_weight *outs, int32_t count);
+qlora_status qlora_nf4_quantize_batched(const float *const *W, const qlora_nf4_weight *outs, int32_t count,
+                                        void *ws, size_t ws_bytes, int32_t *d_status, void *stream);
+
+/*
+ * Dequantize to a dense [rows, cols] tensor.
+ *   out_dtype : 0 = bf16 (uint16_t bit patterns), 1 = fp32.
+ *   transpose : 0 = out is [rows, cols]; 1 = out is [cols, rows] (the
+ *               transposed weight, bf16 only).
+ * Bit-identical to the decode formula above.  No workspace.
+ */
+qlora_status qlora_nf4_dequantize(const qlora_nf4_weight *w, void *out, int32_t out_dtype, int32_t transpose,
+                                  void *stream);
+qlora_status qlora_nf4_dequantize_batched(const qlora_nf4_weight *weights, void *const *outs, int32_t count,
+                                          int32_t out_dtype, void *stream);
+
+/*
+ * Device-side status of a linear-layer workspace.  Kernels record the first
+ * device-detected error (QLORA_ERR_TIMEOUT: a barrier wait ran past its one
+ * second limit, the kernel gave up and returned) in the first word of the
+ * workspace; it stays set until read.
+ *   qlora_workspace_reset  : zero the status word (enqueued on `stream`); call
+ *                            once after allocating a workspace.
+ *   qlora_workspace_status : synchronize `stream`, return the recorded status
+ *                            (QLORA_OK if none) and clear it.
+ */
+qlora_status qlora_workspace_reset(void *ws, size_t ws_bytes, void *stream);
+qlora_status qlora_workspace_status(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Workspace bytes for qlora_linear_fwd / qlora_linear_bwd at tokens M,
+ * weight [N, K] and rank r (the larger of the two needs; one workspace may
+ * serve both).  Returns 0 for invalid sizes.
+ */
+size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
+
+/*
+ * LoRA linear forward:  Y = X W^T + scale * (X A^T) B^T.
+ *   w     : quantized weight, rows = N (d_out), cols = K (d_in).
+ *   X     : bf16 [M, K].   A : bf16 [r, K].   B : bf16 [N, r].
+ *   r     : 1..64.  scale : s = alpha / r (finite).
+ *   ws    : 256-byte aligned workspace of qlora_linear_ws_bytes(M, N, K, r).
+ *   Y     : bf16 [M, N] output (overwritten).
+ *   U_out : bf16 [M, r] output X A^T (for the backward), or NULL.
+ * M <= 16 runs the decode-shaped dequant-GEMV; larger M the tensor-core path.
+ * Accumulation is fp32.  N must be a multiple of 8.
+ */
+qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t M, const uint16_t *A,
+                              const uint16_t *B, int32_t r, float scale, uint16_t *Y, uint16_t *U_out, void *ws,
+                              size_t ws_bytes, void *stream);
+
+/*
+ * LoRA linear backward for upstream gradient dY of Y.
+ *   X, dY      : bf16 [M, K] and [M, N].
+ *   dX         : bf16 [M, K] output, or NULL to skip.  dX = dY W + s (dY B) A.
+ *   accumulate : 0 overwrites dX, 1 adds into it (dX += ...; the sum is
+ *                formed in fp32 and rounded once).
+ *   dA         : fp32 [r, K] output, or NULL.   dA = s (dY B)^T X.
+ *   dB         : fp32 [N, r] output, or NULL.   dB = s dY^T (X A^T).
+ * dA and dB are overwritten, never accumulated.  No gradient is produced for
+ * the frozen weight.
+ */
+qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t M,
+                              const uint16_t *A, const uint16_t *B, int32_t r, float scale, uint16_t *dX,
+                              int32_t accumulate, float *dA, float *dB, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Kernel timing (instrumentation for benchmarks; off by default).
+ * While enabled, every kernel the library enqueues is bracketed by CUDA
+ * events recorded on the launching stream, grouped by family:
+ *   "quantize" (quantize + double quant), "dequant", "gemv", "side" (rank-r
+ *   products, gradient column sums, padding), "gemm" (tensor-core GEMM).
+ *   qlora_timing_enable : 1 starts recording (clearing earlier records), 0 stops.
+ *   qlora_timing_read   : waits for the recorded events of `family` and returns
+ *                         the summed device time in milliseconds and the number
+ *                         of launches since enabling; INVALID_ARG for an unknown
+ *                         family name.
+ * Not thread-safe with concurrent enqueueing from several host threads.
+ */
+qlora_status qlora_timing_enable(int32_t enable);
+qlora_status qlora_timing_read(const char *family, double *total_ms, int64_t *launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,104 @@
+"""The C ABI library loads and exports every entry point its header declares.
+
+CPU-only: no call here reaches a GPU.  Host-side size arithmetic and argument
+checks return before anything is enqueued, so they run without a device.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_nf4_quantized_blk_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fname in sorted(os.listdir(inc)):
+        if not fname.endswith(".h"):
+            continue
+        text = open(os.path.join(inc, fname)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(qlora_[a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_nf4_quantized_blk_b200 import build
+
+    build.build()
+    return binding.lib()
+
+
+def test_header_declares_the_four_method_calls():
+    names = _declared_functions()
+    for n in ("qlora_nf4_quantize", "qlora_nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(names) == sorted(binding.EXPORTED)
+
+
+def test_status_strings(lib):
+    assert binding.qlora_status_string(0) == "ok"
+    assert "workspace" in binding.qlora_status_string(4)
+    assert binding.qlora_status_string(99) == "unknown status"
+
+
+def test_sizes(lib):
+    s = binding.qlora_nf4_sizes(1024, 1024)
+    assert s["packed_bytes"] == 1024 * 1024 // 2
+    assert s["n_blocks"] == 1024 * 1024 // 64
+    assert s["n_chunks"] == 64
+    assert s["ws_bytes"] >= 256 + 64 * 256 * 4
+    s = binding.qlora_nf4_sizes(3, 192)  # 9 blocks: one partial chunk
+    assert s["n_blocks"] == 9 and s["n_chunks"] == 1
+    for rows, cols in ((0, 64), (4, 0), (4, 96), (-1, 64)):
+        with pytest.raises(binding.QloraError) as e:
+            binding.qlora_nf4_sizes(rows, cols)
+        assert e.value.status == 1
+
+
+def test_linear_ws_bytes(lib):
+    assert binding.qlora_linear_ws_bytes(16, 1024, 1024, 8) > 1024 * 1024 * 2
+    assert binding.qlora_linear_ws_bytes(8192, 14336, 4096, 16) > 14336 * 4096 * 2
+    assert binding.qlora_linear_ws_bytes(0, 1024, 1024, 8) == 0
+    assert binding.qlora_linear_ws_bytes(16, 1024, 1000, 8) == 0
+    assert binding.qlora_linear_ws_bytes(16, 1024, 1024, 65) == 0
+
+
+def test_argument_checks_run_before_any_launch(lib):
+    W = binding.QloraNf4WeightC(64, 64, 0, 0, 0, 0)  # null device pointers
+    st = lib.qlora_nf4_quantize(None, ctypes.byref(W), None, 0, None, None)
+    assert st == 1  # INVALID_ARG: nothing enqueued
+    W2 = binding.QloraNf4WeightC(64, 64, 16, 16, 16, 16)
+    st = lib.qlora_nf4_quantize(32, ctypes.byref(W2), None, 0, None, None)
+    assert st == 4  # WORKSPACE
+    st = lib.qlora_nf4_quantize(32, ctypes.byref(W2), 256, 1 << 20, None, None)
+    assert st in (5, 7)  # no device here: CUDA error / unsupported, never a launch
+    W3 = binding.QloraNf4WeightC(64, 64, 17, 16, 16, 16)
+    assert lib.qlora_nf4_quantize(32, ctypes.byref(W3), 256, 1 << 20, None, None) == 2  # ALIGNMENT
+    W4 = binding.QloraNf4WeightC(64, 100, 16, 16, 16, 16)
+    assert lib.qlora_nf4_dequantize(ctypes.byref(W4), 16, 0, 0, None) == 1
+    assert lib.qlora_nf4_dequantize(ctypes.byref(W2), 16, 2, 0, None) == 1  # bad dtype
+    assert lib.qlora_linear_fwd(ctypes.byref(W2), 16, 4, 16, 16, 0, 1.0, 16, None, 256, 1 << 30, None) == 1  # r = 0
+    assert lib.qlora_linear_fwd(ctypes.byref(W2), 16, 4, 16, 16, 8, 1.0, 16, None, 256, 16, None) == 4  # small ws
+    assert lib.qlora_linear_bwd(ctypes.byref(W2), 16, 16, 4, 16, 16, 8, 1.0, None, 2, None, None, 256, 1 << 30,
+                                None) == 1  # accumulate must be 0 or 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        binding.lib()
