@@ -245,16 +245,19 @@ def bench_gemv(reps=50):
         fwd = lambda: binding.qlora_linear_fwd(out, X, case.A, case.B, 16, case.s, Y, None, ws)  # noqa: E731
         for _ in range(3):
             fwd()
-        times = []
+        # Enqueue every repetition before waiting: the L2 flush between calls
+        # keeps the GPU busy while the host enqueues the next call, so no
+        # host launch latency lands inside the timed interval.
+        evs = []
         for _ in range(reps):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fwd()
             b.record()
-            b.synchronize()
-            times.append(a.elapsed_time(b))
-        ms = statistics.median(times)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
         nbytes = (out.packed.numel() + out.qscale.numel() + 4 * out.c2.numel() + 4 + 2 * (case.A.numel() + case.B.numel())
                   + 2 * M * (4096 + 14336))
         res[f"M={M}"] = {"us": ms * 1e3, "GB/s": nbytes / ms / 1e6, "bytes": nbytes}
