@@ -36,6 +36,7 @@ EXPORTED = [
     "qlora_nf4_quantize",
     "qlora_nf4_quantize_batched_ws_bytes",
     "qlora_nf4_quantize_batched",
+    "qlora_nf4_quantize_noalloc",
     "qlora_nf4_dequantize",
     "qlora_nf4_dequantize_batched",
     "qlora_workspace_reset",
@@ -88,6 +89,7 @@ def lib() -> ctypes.CDLL:
         "qlora_nf4_quantize": (i32, [P, W, P, sz, P, P]),
         "qlora_nf4_quantize_batched_ws_bytes": (sz, [W, i32]),
         "qlora_nf4_quantize_batched": (i32, [ctypes.POINTER(P), W, i32, P, sz, P, P]),
+        "qlora_nf4_quantize_noalloc": (i32, [P, W, P, P]),
         "qlora_nf4_dequantize": (i32, [W, P, i32, i32, P]),
         "qlora_nf4_dequantize_batched": (i32, [W, ctypes.POINTER(P), i32, i32, P]),
         "qlora_workspace_reset": (i32, [P, sz, P]),
@@ -185,6 +187,13 @@ def qlora_nf4_quantize_batched(Ws, outs, ws: torch.Tensor, d_status=None, stream
     _check("qlora_nf4_quantize_batched",
            lib().qlora_nf4_quantize_batched(ptrs, arr, len(outs), ws.data_ptr(), ws.numel() * ws.element_size(),
                                             _ptr(d_status), _stream(stream)))
+
+
+def qlora_nf4_quantize_noalloc(W: torch.Tensor, out: NF4Weight, d_status=None, stream=None) -> None:
+    """Quantize without a workspace (library-internal scratch; tensors up to 2^26 weights)."""
+    st = out.c_struct()
+    _check("qlora_nf4_quantize_noalloc",
+           lib().qlora_nf4_quantize_noalloc(W.data_ptr(), ctypes.byref(st), _ptr(d_status), _stream(stream)))
 
 
 def qlora_nf4_dequantize(w: NF4Weight, out: torch.Tensor, out_dtype: int = 0, transpose: int = 0, stream=None) -> None:

@@ -182,7 +182,7 @@ class Timed {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 qlora_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
@@ -215,8 +215,8 @@ struct QuantWs {
   size_t counters, absmax, sums, exps, total;
 };
 
-QuantWs quant_ws_layout(int count, int64_t chunks) {
-  QuantWs l;
+constexpr QuantWs quant_ws_layout(int count, int64_t chunks) {
+  QuantWs l{};
   size_t off = kWsHeader;
   l.counters = off;
   off = align_up(off + sizeof(unsigned) * kMaxQuantBatch, 256);
@@ -674,4 +674,101 @@ extern "C" qlora_status qlora_timing_read(const char* family, double* total_ms, 
   if (total_ms) *total_ms = T.ms[f];
   if (launches) *launches = T.launches[f];
   return QLORA_OK;
+}
+
+// ===========================================================================
+// Quantize without a caller-provided workspace
+// ===========================================================================
+//
+// qlora_nf4_quantize needs ~1 KB of device scratch per 16384 weights (block
+// scales, chunk sums, a counter and a status word) which the caller normally
+// provides as a workspace.  qlora_nf4_quantize_noalloc takes that scratch from
+// the static device array below instead, so a caller that cannot allocate
+// device memory can still quantize.  The array is sized for tensors of up to
+// kNoAllocMaxWeights weights; every GPU that loads this library holds it
+// until the process exits.
+namespace {
+
+constexpr int64_t kNoAllocMaxWeights = int64_t{1} << 26;  // 67,108,864 weights per call
+constexpr int64_t kNoAllocMaxChunks = kNoAllocMaxWeights / kChunkWeights;
+constexpr QuantWs kNoAllocLayout = quant_ws_layout(1, kNoAllocMaxChunks);
+
+// Device scratch shared by every qlora_nf4_quantize_noalloc call on a device.
+static __device__ __align__(256) unsigned char g_quant_scratch[kNoAllocLayout.total];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_scratch[kNoAllocMaxDevices] = {};
+
+// Device address of g_quant_scratch on the current device, resolved once per
+// device.  In host code the array's name only stands for the symbol; the
+// address the kernels need comes from cudaGetSymbolAddress.
+qlora_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return QLORA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_scratch[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_quant_scratch);
+    if (e != cudaSuccess || p == nullptr) return QLORA_ERR_CUDA;
+    g_noalloc_scratch[dev] = p;
+  }
+  *out = g_noalloc_scratch[dev];
+  return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" qlora_status qlora_nf4_quantize_noalloc(const float* W, const qlora_nf4_weight* out, int32_t* d_status,
+                                                   void* stream) {
+  qlora_status st = check_weight(out);
+  if (st != QLORA_OK) return st;
+  if (W == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (out->rows > kNoAllocMaxWeights / out->cols) return QLORA_ERR_UNSUPPORTED;  // beyond the static scratch
+  if (!aligned(W, 32)) return QLORA_ERR_ALIGNMENT;
+  if (d_status != nullptr && !aligned(d_status, 4)) return QLORA_ERR_ALIGNMENT;
+  st = check_device();
+  if (st != QLORA_OK) return st;
+  const Nf4DecisionTable* tab = decision_table();
+  if (tab == nullptr) return QLORA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != QLORA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = d_status != nullptr ? d_status : at<int>(scratch, 0);
+  // The scratch keeps the previous call's contents: clear what must start at zero.
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(at<unsigned>(scratch, kNoAllocLayout.counters), 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return from_cuda(e);
+
+  QuantBatchParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.count = 1;
+  p.chunk_begin[0] = 0;
+  p.chunk_begin[1] = p.total_chunks = n_chunks_of(out->rows, out->cols);
+  p.n_blocks[0] = out->rows * out->cols / kBlock;
+  p.W[0] = W;
+  p.packed[0] = out->packed;
+  p.qscale[0] = out->qscale;
+  p.c2[0] = out->c2;
+  p.mu[0] = out->mu;
+  p.absmax = at<float>(scratch, kNoAllocLayout.absmax);
+  p.chunk_sum = at<double>(scratch, kNoAllocLayout.sums);
+  p.chunk_exp = at<int>(scratch, kNoAllocLayout.exps);
+  p.counters = at<unsigned>(scratch, kNoAllocLayout.counters);
+  p.status = status;
+  p.table = *tab;
+  {
+    Timed tm(kFamQuant, s, 2);
+    e = launch_quantize_batch(p, s);
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  if (d_status != nullptr) return QLORA_OK;
+  int32_t h = 0;
+  e = cudaMemcpyAsync(&h, status, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return from_cuda(e);
+  return static_cast<qlora_status>(h);
 }

@@ -128,6 +128,31 @@ qlora_status qlora_nf4_quantize_batched(const float *const *W, const qlora_nf4_w
                                         void *ws, size_t ws_bytes, int32_t *d_status, void *stream);
 
 /*
+ * Quantize + double-quantize one tensor exactly as qlora_nf4_quantize does,
+ * without a workspace.  (The pages have no counterpart: this is an interface
+ * for callers, not a step of the method.)
+ *
+ * Some callers cannot allocate device memory or hand over a workspace: a
+ * serving engine or framework plugin whose host reserves all device memory in
+ * its own pool up front and forbids allocation while it runs, or a plain C
+ * caller that owns no device allocator.  This entry point takes its scratch
+ * from a fixed array inside the library instead: about 4.1 MB of device
+ * memory that every GPU which loads the library holds until the process
+ * exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   W, out, d_status, stream : as qlora_nf4_quantize.
+ *   Limit: rows * cols <= 67,108,864 (2^26) weights; larger tensors return
+ *   QLORA_ERR_UNSUPPORTED before anything is enqueued.
+ * The first call on each device resolves the array's device address
+ * (cudaGetSymbolAddress) for that device; make that first call before any
+ * stream capture.  All calls on a device share the one array and it keeps
+ * the previous call's contents (each call clears the parts that must start
+ * at zero), so calls that overlap on the GPU -- on different streams or from
+ * several host threads -- race and give wrong results: serialize them.
+ */
+qlora_status qlora_nf4_quantize_noalloc(const float *W, const qlora_nf4_weight *out, int32_t *d_status,
+                                        void *stream);
+
+/*
  * Dequantize to a dense [rows, cols] tensor.
  *   out_dtype : 0 = bf16 (uint16_t bit patterns), 1 = fp32.
  *   transpose : 0 = out is [rows, cols]; 1 = out is [cols, rows] (the
