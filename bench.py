@@ -139,13 +139,14 @@ class LayerStep:
         self.dX = [torch.empty((M, c.proj.k), dtype=torch.bfloat16, device=device) for c in self.cases]
         self.dA = [torch.empty((c.r, c.proj.k), dtype=torch.float32, device=device) for c in self.cases]
         self.dB = [torch.empty((c.proj.n, c.r), dtype=torch.float32, device=device) for c in self.cases]
+        self.U = [torch.empty((M, c.r), dtype=torch.float32, device=device) for c in self.cases]
 
     def run(self):
         binding.qlora_nf4_quantize_batched([c.W for c in self.cases], self.outs, self.qws, d_status=self.dstat)
-        for c, o, Y in zip(self.cases, self.outs, self.Y):
-            binding.qlora_linear_fwd(o, c.X, c.A, c.B, c.r, c.s, Y, None, self.lws)
-        for c, o, dX, dA, dB in reversed(list(zip(self.cases, self.outs, self.dX, self.dA, self.dB))):
-            binding.qlora_linear_bwd(o, c.X, c.dY, c.A, c.B, c.r, c.s, dX, 0, dA, dB, self.lws)
+        for c, o, Y, U in zip(self.cases, self.outs, self.Y, self.U):
+            binding.qlora_linear_fwd(o, c.X, c.A, c.B, c.r, c.s, Y, U, self.lws)
+        for c, o, dX, dA, dB, U in reversed(list(zip(self.cases, self.outs, self.dX, self.dA, self.dB, self.U))):
+            binding.qlora_linear_bwd(o, c.X, c.dY, c.A, c.B, c.r, c.s, dX, 0, dA, dB, self.lws, U=U)
 
     def check_status(self):
         assert self.dstat.item() == 0, "quantize reported non-finite input"

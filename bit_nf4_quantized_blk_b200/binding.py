@@ -96,7 +96,7 @@ def lib() -> ctypes.CDLL:
         "qlora_workspace_status": (i32, [P, sz, P]),
         "qlora_linear_ws_bytes": (sz, [i64, i64, i64, i32]),
         "qlora_linear_fwd": (i32, [W, P, i64, P, P, i32, f32, P, P, P, sz, P]),
-        "qlora_linear_bwd": (i32, [W, P, P, i64, P, P, i32, f32, P, i32, P, P, P, sz, P]),
+        "qlora_linear_bwd": (i32, [W, P, P, i64, P, P, i32, f32, P, P, i32, P, P, P, sz, P]),
         "qlora_timing_enable": (i32, [i32]),
         "qlora_timing_read": (i32, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]),
     }
@@ -230,12 +230,12 @@ def qlora_linear_fwd(w: NF4Weight, X, A, B, r: int, scale: float, Y, U_out, ws, 
 
 
 def qlora_linear_bwd(w: NF4Weight, X, dY, A, B, r: int, scale: float, dX, accumulate: int, dA, dB, ws,
-                     stream=None) -> None:
+                     U=None, stream=None) -> None:
     st = w.c_struct()
     _check("qlora_linear_bwd",
            lib().qlora_linear_bwd(ctypes.byref(st), X.data_ptr(), dY.data_ptr(), X.shape[0], A.data_ptr(),
-                                  B.data_ptr(), r, float(scale), _ptr(dX), int(accumulate), _ptr(dA), _ptr(dB),
-                                  ws.data_ptr(), ws.numel(), _stream(stream)))
+                                  B.data_ptr(), r, float(scale), _ptr(U), _ptr(dX), int(accumulate), _ptr(dA),
+                                  _ptr(dB), ws.data_ptr(), ws.numel(), _stream(stream)))
 
 
 def qlora_timing_enable(enable: bool) -> None:

@@ -87,7 +87,7 @@ bool build_decision_table(Nf4DecisionTable* tab) {
       xhi = static_cast<float>(t) / 64.0f;
     }
     int base = 0, inside = 0;
-    float thr = INFINITY;
+    float thr = 4.0f;  // no threshold in this cell: a value no x in [-1, 1] reaches
     for (int j = 1; j < 16; ++j) {
       if (T[j] <= xlo) ++base;
       else if (T[j] <= xhi) {
@@ -96,6 +96,9 @@ bool build_decision_table(Nf4DecisionTable* tab) {
       }
     }
     if (inside > 1) return false;
+    // The quantize kernel's reciprocal fast path needs every threshold well
+    // inside its cell (relative gap > 2^-14 to both cell edges).
+    if (inside && (thr - xlo < std::fabs(thr) * 0x1p-14f || xhi - thr < std::fabs(thr) * 0x1p-14f)) return false;
     tab->thr[c] = thr;
     tab->base[c] = base;
     auto code_of = [&](float x) { return base + (x >= thr ? 1 : 0); };
@@ -244,7 +247,7 @@ int64_t max_group_chunks(const qlora_nf4_weight* outs, int32_t count) {
 
 // Linear workspace layout.
 struct LinearWs {
-  size_t wbf, u32, us, uhi, ulo, vs, vhi, vlo, bpad, atpad, part, total;
+  size_t wbf, u32, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, total;
 };
 
 LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
@@ -265,9 +268,10 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
   l.vhi = take(mr * 2);
   l.vlo = take(mr * 2);
   l.bpad = take(static_cast<size_t>(N) * kRankPad * 2);
-  l.atpad = take(static_cast<size_t>(K) * kRankPad * 2);
   const size_t p1 = colsum_partial_bytes(M, N), p2 = colsum_partial_bytes(M, K);
   l.part = take(p1 > p2 ? p1 : p2);
+  const size_t s1 = skinny_partial_bytes(M, N), s2 = skinny_partial_bytes(M, K);
+  l.skpart = take(s1 > s2 ? s1 : s2);
   l.total = off;
   return l;
 }
@@ -424,16 +428,17 @@ extern "C" qlora_status qlora_nf4_dequantize_batched(const qlora_nf4_weight* wei
     int64_t c = 0;
     for (int i = 0; i < n; ++i) {
       const qlora_nf4_weight& w = weights[g0 + i];
-      p.begin16[i] = c;
+      p.begin_seg[i] = c;
+      p.n_words[i] = w.rows * w.cols / 8;
       p.packed[i] = w.packed;
       p.qscale[i] = w.qscale;
       p.c2[i] = w.c2;
       p.mu[i] = w.mu;
       p.out[i] = outs[g0 + i];
-      c += w.rows * w.cols / 32;
+      c += (p.n_words[i] + 127) / 128;
     }
-    p.begin16[n] = c;
-    p.total16 = c;
+    p.begin_seg[n] = c;
+    p.total_seg = c;
     cudaError_t e;
     {
       Timed tm(kFamDequant, s);
@@ -485,12 +490,12 @@ extern "C" qlora_status qlora_workspace_status(void* ws, size_t ws_bytes, void* 
 }
 
 extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
-                                         const uint16_t* B, int32_t r, float scale, uint16_t* Y, uint16_t* U_out,
+                                         const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* U_out,
                                          void* ws, size_t ws_bytes, void* stream) {
   qlora_status st = check_linear_args(w, M, r, ws_bytes, ws);
   if (st != QLORA_OK) return st;
   if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) || (U_out && !aligned(U_out, 2)))
+  if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) || (U_out && !aligned(U_out, 4)))
     return QLORA_ERR_ALIGNMENT;
   if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
   st = check_device();
@@ -513,7 +518,8 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
   DequantBatchParams p;
   std::memset(&p, 0, sizeof(p));
   p.count = 1;
-  p.begin16[1] = p.total16 = N * K / 32;
+  p.n_words[0] = N * K / 8;
+  p.begin_seg[1] = p.total_seg = (p.n_words[0] + 127) / 128;
   p.packed[0] = w->packed;
   p.qscale[0] = w->qscale;
   p.c2[0] = w->c2;
@@ -525,20 +531,25 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
   }
   if (e != cudaSuccess) return from_cuda(e);
   SkinnyOut so{};
+  so.o32 = U_out;
+  so.o32_ld = r;
   so.os = at<uint16_t>(ws, lay.us);
-  so.obf = U_out;
   so.scale = scale;
+  // The caller's B [N, r] feeds the rank step directly when its rows are
+  // 16-byte multiples; otherwise a zero-padded copy [N, 64] does.
+  const bool b_direct = (r % 8) == 0 && aligned(B, 16);
   {
-    Timed tm(kFamSide, s, 2);
-    e = launch_skinny(X, M, K, A, true, r, so, s);
-    if (e == cudaSuccess) e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
+    Timed tm(kFamSide, s, b_direct ? 2 : 3);
+    e = launch_skinny(X, M, K, A, true, r, 0, at<float>(ws, lay.skpart), so, status, s);
+    if (e == cudaSuccess && !b_direct) e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
   }
   if (e != cudaSuccess) return from_cuda(e);
   GemmArgs g{};
   g.A = X;
   g.B = at<uint16_t>(ws, lay.wbf);
   g.A2 = at<uint16_t>(ws, lay.us);
-  g.B2 = at<uint16_t>(ws, lay.bpad);
+  g.B2 = b_direct ? B : at<uint16_t>(ws, lay.bpad);
+  g.ldb2 = b_direct ? r : kRankPad;
   g.M = M;
   g.N = N;
   g.K = K;
@@ -551,15 +562,15 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
 }
 
 extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,
-                                         const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* dX,
-                                         int32_t accumulate, float* dA, float* dB, void* ws, size_t ws_bytes,
-                                         void* stream) {
+                                         const uint16_t* A, const uint16_t* B, int32_t r, float scale, const float* U,
+                                         uint16_t* dX, int32_t accumulate, float* dA, float* dB, void* ws,
+                                         size_t ws_bytes, void* stream) {
   qlora_status st = check_linear_args(w, M, r, ws_bytes, ws);
   if (st != QLORA_OK) return st;
   if (!X || !dY || !A || !B) return QLORA_ERR_INVALID_ARG;
   if (accumulate != 0 && accumulate != 1) return QLORA_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(dY, 16) || !aligned(A, 16) || !aligned(B, 2) || (dX && !aligned(dX, 16)) ||
-      (dA && !aligned(dA, 4)) || (dB && !aligned(dB, 4)))
+      (dA && !aligned(dA, 4)) || (dB && !aligned(dB, 4)) || (U && !aligned(U, 4)))
     return QLORA_ERR_ALIGNMENT;
   if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
   st = check_device();
@@ -576,43 +587,58 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
   vo.ohi = at<uint16_t>(ws, lay.vhi);
   vo.olo = at<uint16_t>(ws, lay.vlo);
   vo.scale = scale;
+  const bool b_direct = (r % 8) == 0 && aligned(B, 16);
   {
-    Timed tm(kFamSide, s, 2);
-    e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
-    if (e == cudaSuccess) e = launch_skinny(dY, M, N, at<uint16_t>(ws, lay.bpad), false, r, vo, s);
+    Timed tm(kFamSide, s, b_direct ? 2 : 3);
+    if (!b_direct) e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
+    if (b_direct)
+      e = launch_skinny(dY, M, N, B, false, r, r, at<float>(ws, lay.skpart), vo, status, s);
+    else if (e == cudaSuccess)
+      e = launch_skinny(dY, M, N, at<uint16_t>(ws, lay.bpad), false, r, kRankPad, at<float>(ws, lay.skpart), vo,
+                        status, s);
   }
   if (e != cudaSuccess) return from_cuda(e);
 
-  if (dB != nullptr) {  // dB = s dY^T U with U = X A^T
-    SkinnyOut uo{};
-    uo.ohi = at<uint16_t>(ws, lay.uhi);
-    uo.olo = at<uint16_t>(ws, lay.ulo);
-    uo.scale = 1.0f;
+  if (dB != nullptr) {  // dB = s dY^T U with U = X A^T (saved by the forward, or recomputed)
     {
-      Timed tm(kFamSide, s, 3);
-      e = launch_skinny(X, M, K, A, true, r, uo, s);
+      Timed tm(kFamSide, s, U != nullptr ? 3 : 4);
+      if (U != nullptr) {
+        e = launch_split_hilo(U, M, r, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), s);
+      } else {
+        SkinnyOut uo{};
+        uo.ohi = at<uint16_t>(ws, lay.uhi);
+        uo.olo = at<uint16_t>(ws, lay.ulo);
+        uo.scale = 1.0f;
+        e = launch_skinny(X, M, K, A, true, r, 0, at<float>(ws, lay.skpart), uo, status, s);
+      }
       if (e == cudaSuccess)
         e = launch_colsum(dY, M, N, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), r, scale,
-                          at<float>(ws, lay.part), dB, false, s);
+                          at<float>(ws, lay.part), dB, false, status, s);
     }
     if (e != cudaSuccess) return from_cuda(e);
   }
-  if (dX != nullptr) {  // dX = dY W_hat + s V A
+  if (dX != nullptr) {  // dX = dY W_hat + s V A, reading W_hat [N, K] and A [r, K] as MN-major operands
+    DequantBatchParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.count = 1;
+    p.n_words[0] = N * K / 8;
+    p.begin_seg[1] = p.total_seg = (p.n_words[0] + 127) / 128;
+    p.packed[0] = w->packed;
+    p.qscale[0] = w->qscale;
+    p.c2[0] = w->c2;
+    p.mu[0] = w->mu;
+    p.out[0] = at<uint16_t>(ws, lay.wbf);
     {
       Timed tm(kFamDequant, s);
-      e = launch_dequant_transposed(view_of(w), at<uint16_t>(ws, lay.wbf), s);
-    }
-    if (e != cudaSuccess) return from_cuda(e);
-    {
-      Timed tm(kFamSide, s);
-      e = launch_pad_rank(A, true, K, r, at<uint16_t>(ws, lay.atpad), s);
+      e = launch_dequant_batch(p, 0, s);
     }
     if (e != cudaSuccess) return from_cuda(e);
     GemmArgs g{};
     g.A = dY;
     g.B = at<uint16_t>(ws, lay.wbf);
     g.A2 = at<uint16_t>(ws, lay.vs);
-    g.B2 = at<uint16_t>(ws, lay.atpad);
+    g.B2 = A;
+    g.b_mn_major = 1;
     g.M = M;
     g.N = K;
     g.K = N;
@@ -630,7 +656,7 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
     {
       Timed tm(kFamSide, s, 2);
       e = launch_colsum(X, M, K, at<uint16_t>(ws, lay.vhi), at<uint16_t>(ws, lay.vlo), r, scale,
-                        at<float>(ws, lay.part), dA, true, s);
+                        at<float>(ws, lay.part), dA, true, status, s);
     }
     if (e != cudaSuccess) return from_cuda(e);
   }

@@ -26,9 +26,8 @@ constexpr int kChunkWeights = kBlock * kDqBlock;  // 16384 weights per chunk
 constexpr int kMaxRank = 64;       // largest LoRA rank the kernels take
 constexpr int kRankPad = 64;       // padded row length of rank-r side buffers
 
-// Workspace header: the first 256 bytes of every linear-layer workspace hold
-// the device status word (sticky error code) and the GEMV tile counters area
-// offset is carved after it by the host code.
+// Workspace header: the first 256 bytes of every workspace hold the device
+// status word (sticky error code); the host carves the rest after it.
 constexpr size_t kWsHeader = 256;
 
 // Time limit of every device-side wait, in nanoseconds of %globaltimer.
@@ -243,12 +242,27 @@ __device__ __forceinline__ uint64_t smem_desc_k128(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major operand tile in the 128-byte
+// swizzle layout: atoms of 8 rows along K x 128 bytes (64 bf16) along MN;
+// `lbo` = byte stride between 64-element MN groups, `sbo` = byte stride
+// between 8-row K groups.
+__device__ __forceinline__ uint64_t smem_desc_mn128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulator,
-// both operands K-major, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+// A K-major, B K-major (b_mn = false) or MN-major (b_mn = true), shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn = false) {
   return (1u << 4)                                  // D format: fp32
          | (1u << 7)                                // A format: bf16
          | (1u << 10)                               // B format: bf16
+         | (b_mn ? (1u << 16) : 0u)                 // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
@@ -335,7 +349,8 @@ __host__ __device__ constexpr float nf4_level(int j) {
 
 // Decision table of the nearest-level search on x in [-1, 1] (built once on
 // the host, see api.cu): cell c = trunc(64 x) + 64 covers a fixed interval of
-// x holding at most one decision threshold; code(x) = base[c] + (x >= thr[c]).
+// x holding at most one decision threshold; code(x) = base[c] + (x >= thr[c])
+// (thr[c] = 4 where the cell holds none).
 struct Nf4DecisionTable {
   float thr[129];
   int base[129];

@@ -8,8 +8,7 @@
 // fp32(L[code] * a); bf16 output rounds that value to nearest even.
 //
 // HBM-bound: 0.5 B of codes + 1/64 B of scale codes read and 2 B (bf16) or
-// 4 B (fp32) written per weight.  Each thread owns 16 packed bytes (half a
-// block, one 128-bit load) and writes 64 / 128 contiguous output bytes.
+// 4 B (fp32) written per weight.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -23,55 +22,69 @@ __device__ __forceinline__ void fill_pair_table(float2* tab) {
 
 }  // namespace
 
-__device__ __forceinline__ int find_tensor16(const DequantBatchParams& p, int64_t chunk) {
+__device__ __forceinline__ int find_tensor_seg(const DequantBatchParams& p, int64_t seg) {
   int lo = 0, hi = p.count - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (p.begin16[mid] <= chunk) lo = mid; else hi = mid - 1;
+    if (p.begin_seg[mid] <= seg) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
+// One warp per 512-byte segment of packed codes (1024 weights, 16 blocks):
+// lane t reads the 32-bit words t, t+32, t+64, t+96 of the segment, so every
+// load and every store instruction of the warp covers one contiguous span.
 template <bool kFp32>
 __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ DequantBatchParams p) {
   __shared__ float2 s_pair[256];
   fill_pair_table(s_pair);
   __syncthreads();
-  const int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // 16-byte chunk index
-  if (gi >= p.total16) return;
-  const int t = find_tensor16(p, gi);
-  const int64_t i = gi - p.begin16[t];
-  const int64_t blk = i >> 1;  // two chunks per 64-weight block
-  const float a = decode_scale(p.qscale[t][blk], p.c2[t][blk / kDqBlock], *p.mu[t]);
-  const uint4 pk = ld_stream_u4(p.packed[t] + i * 16);
-  const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
-  if constexpr (kFp32) {
-    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out[t]) + i * 32);
+  const int lane = threadIdx.x & 31;
+  const int64_t gseg = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (gseg >= p.total_seg) return;
+  const int t = find_tensor_seg(p, gseg);
+  const int64_t seg = gseg - p.begin_seg[t];
+  const int64_t n_words = p.n_words[t];
+  const uint32_t* __restrict__ packed = reinterpret_cast<const uint32_t*>(p.packed[t]);
+  const float mu = *p.mu[t];
+  uint32_t words[4];
+  float a[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < 4; ++q) {
+    const int64_t w = seg * 128 + lane + 32 * q;
+    words[q] = 0;
+    a[q] = 0.0f;
+    if (w < n_words) {
+      words[q] = __ldcs(packed + w);
+      const int64_t blk = w >> 3;  // 8 words per 64-weight block
+      a[q] = decode_scale(p.qscale[t][blk], p.c2[t][blk / kDqBlock], mu);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int64_t w = seg * 128 + lane + 32 * q;
+    if (w >= n_words) continue;
+    if constexpr (kFp32) {
       float vals[8];
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         const float2 lv = s_pair[(words[q] >> (8 * b)) & 0xFF];
-        vals[2 * b] = __fmul_rn(lv.x, a);
-        vals[2 * b + 1] = __fmul_rn(lv.y, a);
+        vals[2 * b] = __fmul_rn(lv.x, a[q]);
+        vals[2 * b + 1] = __fmul_rn(lv.y, a[q]);
       }
-      st_stream_u4(o + 2 * q, make_uint4(__float_as_uint(vals[0]), __float_as_uint(vals[1]), __float_as_uint(vals[2]),
-                                         __float_as_uint(vals[3])));
-      st_stream_u4(o + 2 * q + 1, make_uint4(__float_as_uint(vals[4]), __float_as_uint(vals[5]),
-                                             __float_as_uint(vals[6]), __float_as_uint(vals[7])));
-    }
-  } else {
-    uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[t]) + i * 32);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out[t]) + w * 8);
+      st_stream_u4(o, make_uint4(__float_as_uint(vals[0]), __float_as_uint(vals[1]), __float_as_uint(vals[2]),
+                                 __float_as_uint(vals[3])));
+      st_stream_u4(o + 1, make_uint4(__float_as_uint(vals[4]), __float_as_uint(vals[5]), __float_as_uint(vals[6]),
+                                     __float_as_uint(vals[7])));
+    } else {
       uint32_t pr[4];
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         const float2 lv = s_pair[(words[q] >> (8 * b)) & 0xFF];
-        pr[b] = pack_bf16x2(__fmul_rn(lv.x, a), __fmul_rn(lv.y, a));
+        pr[b] = pack_bf16x2(__fmul_rn(lv.x, a[q]), __fmul_rn(lv.y, a[q]));
       }
-      st_stream_u4(o + q, make_uint4(pr[0], pr[1], pr[2], pr[3]));
+      st_stream_u4(static_cast<uint16_t*>(p.out[t]) + w * 8, make_uint4(pr[0], pr[1], pr[2], pr[3]));
     }
   }
 }
@@ -123,8 +136,8 @@ __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, u
 }
 
 cudaError_t launch_dequant_batch(const DequantBatchParams& p, int out_fp32, cudaStream_t stream) {
-  if (p.total16 <= 0) return cudaSuccess;
-  const unsigned grid = static_cast<unsigned>((p.total16 + 255) / 256);
+  if (p.total_seg <= 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((p.total_seg + 7) / 8);  // 8 warps per CTA
   if (out_fp32)
     dequant_kernel<true><<<grid, 256, 0, stream>>>(p);
   else

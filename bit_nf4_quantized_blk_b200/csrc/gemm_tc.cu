@@ -9,10 +9,11 @@
 // The rank-r product is one more pipeline step that issues ceil(r/16)
 // K=16 MMAs into the same accumulator.
 //
-// One CTA computes a 128 x 256 tile with a 4-stage TMA ring:
+// Persistent CTAs (one per SM) compute 128 x 256 tiles with a 4-stage TMA ring:
 //   warp 0      TMA producer (one elected thread), 128B-swizzled tiles
 //   warp 1      TMEM allocation + MMA issue (one thread): tcgen05.mma
-//               kind::f16, M=128 N=256 K=16, fp32 accumulator in TMEM
+//               kind::f16, M=128 N=256 K=16, fp32 accumulators in TMEM,
+//               double-buffered so the epilogue overlaps the next tile
 //   warps 2-5   epilogue: tcgen05.ld 32 columns at a time -> bf16 -> global
 // Every barrier wait is bounded (see common.cuh); a timeout aborts the CTA,
 // which then waits (bounded) for its copies and MMAs in flight and frees its
@@ -27,7 +28,8 @@ namespace {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_TILE = BM * BK * 2;  // 16 KB
 constexpr int B_TILE = BN * BK * 2;  // 32 KB
-constexpr int TMEM_COLS = 256;
+constexpr int TMEM_COLS = 512;       // two 128 x 256 fp32 accumulators
+constexpr int kGroupM = 16;          // M tiles per raster group
 constexpr int SMEM_BYTES = 1024 + STAGES * (A_TILE + B_TILE) + 256;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -48,21 +50,44 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-// bf16 row-major [rows][cols] (cols contiguous), box box_rows x box_cols,
-// 128-byte swizzle, zero fill outside the tensor.
+// bf16 row-major [rows][cols] (cols contiguous, row pitch ld elements), box
+// box_rows x box_cols, 128-byte swizzle (or none), zero fill outside the tensor.
 bool encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
-                          uint32_t box_cols) {
+                          uint32_t box_cols, bool swizzle128, uint64_t ld) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t gdim[2] = {cols, rows};
-  const cuuint64_t gstride[1] = {cols * 2};
+  const cuuint64_t gstride[1] = {(ld ? ld : cols) * 2};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estride[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tile order: groups of kGroupM consecutive M tiles sweep the N tiles, so the
+// CTAs resident at one time share a few A row panels and a few B row panels
+// (both stay in L2 instead of being re-read from HBM every wave).
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int& mb, int& nb) {
+  const int per_group = kGroupM * n_tiles;
+  const int group = t / per_group;
+  const int first_m = group * kGroupM;
+  const int gsize = min(kGroupM, m_tiles - first_m);
+  const int local = t - group * per_group;
+  mb = first_m + local % gsize;
+  nb = local / gsize;
+}
+
+// Persistent: one CTA per SM loops over output tiles.  The TMA ring runs
+// across tile boundaries; the accumulator is double-buffered in TMEM (2 x 256
+// columns) so the epilogue of one tile overlaps the main loop of the next.
+//
+// kBMN selects the B operand's major-ness.  K-major: B tiles are 256 rows (N)
+// of 64 K elements, one TMA box.  MN-major: B is stored [K][N] (N
+// contiguous, e.g. the weight [d_out, d_in] read as W^T); a stage holds four
+// 64 (K) x 64 (N) boxes 8 KB apart, described with LBO = 8 KB between N
+// groups and SBO = 1 KB between 8-row K groups.
+template <bool kBMN>
 __global__ void __launch_bounds__(192, 1)
     gemm_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, int M, int N,
@@ -73,20 +98,27 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sB = smem + STAGES * A_TILE;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_TILE);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* acc_full = empty + STAGES;     // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-  const int total = num_k + (r_steps > 0 ? 1 : 0);
+  const int m_tiles = (M + BM - 1) / BM, n_tiles = (N + BN - 1) / BN;
+  const int total_tiles = m_tiles * n_tiles;
+  const int k_iters = num_k + (r_steps > 0 ? 1 : 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -107,57 +139,100 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmA2);
         tma_prefetch_desc(&tmB2);
       }
-      int issued = 0;
-      for (int i = 0; i < total; ++i) {
-        const int s = i % STAGES, u = i / STAGES;
-        if (i >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag, status)) break;
-        mbar_arrive_expect_tx(&full[s], A_TILE + B_TILE);
-        if (i < num_k) {
-          tma_load_2d(sA + s * A_TILE, &tmA, &full[s], i * BK, m0);
-          tma_load_2d(sB + s * B_TILE, &tmB, &full[s], i * BK, n0);
-        } else {
-          tma_load_2d(sA + s * A_TILE, &tmA2, &full[s], 0, m0);
-          tma_load_2d(sB + s * B_TILE, &tmB2, &full[s], 0, n0);
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, m_tiles, n_tiles, mb, nb);
+        const int m0 = mb * BM, n0 = nb * BN;
+        for (int i = 0; i < k_iters; ++i, ++it) {
+          const int s = it % STAGES, u = it / STAGES;
+          if (it >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          if constexpr (!kBMN) {
+            mbar_arrive_expect_tx(&full[s], A_TILE + B_TILE);
+            if (i < num_k) {
+              tma_load_2d(sA + s * A_TILE, &tmA, &full[s], i * BK, m0);
+              tma_load_2d(sB + s * B_TILE, &tmB, &full[s], i * BK, n0);
+            } else {
+              tma_load_2d(sA + s * A_TILE, &tmA2, &full[s], 0, m0);
+              tma_load_2d(sB + s * B_TILE, &tmB2, &full[s], 0, n0);
+            }
+          } else {
+            if (i < num_k) {
+              mbar_arrive_expect_tx(&full[s], A_TILE + B_TILE);
+              tma_load_2d(sA + s * A_TILE, &tmA, &full[s], i * BK, m0);
+              for (int j = 0; j < BN / 64; ++j)
+                tma_load_2d(sB + s * B_TILE + j * 8192, &tmB, &full[s], n0 + 64 * j, i * BK);
+            } else {
+              // rank step: B2 is [r][N]; boxes of r16 rows at the same 8 KB spacing
+              mbar_arrive_expect_tx(&full[s], A_TILE + (BN / 64) * r_steps * 16 * 128);
+              tma_load_2d(sA + s * A_TILE, &tmA2, &full[s], 0, m0);
+              for (int j = 0; j < BN / 64; ++j)
+                tma_load_2d(sB + s * B_TILE + j * 8192, &tmB2, &full[s], n0 + 64 * j, 0);
+            }
+          }
         }
-        issued = i + 1;
       }
       // Teardown: every issued copy must have landed before shared memory is released.
-      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+      for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
         mbar_wait_teardown(&full[i % STAGES], (i / STAGES) & 1, status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, BN);
-      for (int i = 0; i < total; ++i) {
-        const int s = i % STAGES, u = i / STAGES;
-        if (!mbar_wait(&full[s], u & 1, abort_flag, status)) break;
+      const uint32_t idesc = idesc_bf16_f32(BM, BN, kBMN);
+      int it = 0, tl = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tl) {
+        const int buf = tl & 1, use = tl >> 1;
+        if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1, abort_flag, status)) break;
         tc_fence_after();
-        const int nsteps = i < num_k ? BK / 16 : r_steps;
-        const uint64_t adesc = smem_desc_k128(smem_u32(sA + s * A_TILE));
-        const uint64_t bdesc = smem_desc_k128(smem_u32(sB + s * B_TILE));
-        for (int kk = 0; kk < nsteps; ++kk) {
-          // +32 bytes (16 bf16 of K) inside the 128-byte swizzle atom
-          tc_mma_bf16_ss(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN);
+        for (int i = 0; i < k_iters; ++i, ++it) {
+          const int s = it % STAGES, u = it / STAGES;
+          if (!mbar_wait(&full[s], u & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nsteps = i < num_k ? BK / 16 : r_steps;
+          const uint64_t adesc = smem_desc_k128(smem_u32(sA + s * A_TILE));
+          const uint64_t bdesc = kBMN ? smem_desc_mn128(smem_u32(sB + s * B_TILE), 8192, 1024)
+                                      : smem_desc_k128(smem_u32(sB + s * B_TILE));
+          // One K=16 step: A (K-major) +32 bytes inside the swizzle atom;
+          // B +32 bytes (K-major) or +2 atoms of 8 rows = 2048 bytes (MN-major).
+          const uint32_t bstep = kBMN ? (2048 >> 4) : 2;
+          for (int kk = 0; kk < nsteps; ++kk)
+            tc_mma_bf16_ss(acc, adesc + 2 * kk, bdesc + bstep * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
         }
-        tc_commit(&empty[s]);
+        if (ok) tc_commit(&acc_full[buf]);
       }
-      tc_commit(acc_full);
-      // The accumulator must be complete before the tensor memory is released.
-      mbar_wait_teardown(acc_full, 0, status);
+      // Every MMA must be complete before the tensor memory is released.
+      tc_commit(drain);
+      mbar_wait_teardown(drain, 0, status);
     }
   } else {
     // Epilogue warps 2..5 own TMEM lane quadrants (warp % 4).
-    // The tcgen05.ld below is warp-collective: take the decision warp-uniformly.
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, status) ? 1 : 0) != 0;
-    tc_fence_after();
-    if (ok) {
-      const int q = warp & 3;
-      const int row = m0 + q * 32 + lane;
+    const int q = warp & 3;
+    int tl = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tl) {
+      const int buf = tl & 1, use = tl >> 1;
+      // The tcgen05.ld below is warp-collective: take the decision warp-uniformly.
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], use & 1, abort_flag, status) ? 1 : 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      int mb, nb;
+      tile_coords(t, m_tiles, n_tiles, mb, nb);
+      const int row = mb * BM + q * 32 + lane;
+      const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(q * 32) << 16);
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+        tmem_ld_32x32b_x32(acc + c * 32, v);
         tmem_wait_ld();
-        const int col = n0 + c * 32;
+        const int col = nb * BN + c * 32;
         if (row >= M || col >= N) continue;
         uint16_t* dst = D + static_cast<int64_t>(row) * N + col;
         if (col + 32 <= N) {
@@ -193,6 +268,10 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
+      // Hand the accumulator buffer back to the MMA warp.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
   tc_fence_before();
@@ -206,26 +285,53 @@ __global__ void __launch_bounds__(192, 1)
 cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_tn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   CUtensorMap tA, tB, tA2, tB2;
   if (!encode_tensor_map_2d(&tA, a.A, a.M, a.K, BM, BK)) return cudaErrorInvalidValue;
-  if (!encode_tensor_map_2d(&tB, a.B, a.N, a.K, BN, BK)) return cudaErrorInvalidValue;
+  if (a.b_mn_major) {
+    if (!encode_tensor_map_2d(&tB, a.B, a.K, a.N, BK, 64)) return cudaErrorInvalidValue;  // B stored [K][N]
+  } else {
+    if (!encode_tensor_map_2d(&tB, a.B, a.N, a.K, BN, BK, true, a.ldb)) return cudaErrorInvalidValue;
+  }
   int r_steps = 0;
   if (a.A2 != nullptr && a.r > 0) {
-    if (!encode_tensor_map_2d(&tA2, a.A2, a.M, kRankPad, BM, BK)) return cudaErrorInvalidValue;
-    if (!encode_tensor_map_2d(&tB2, a.B2, a.N, kRankPad, BN, BK)) return cudaErrorInvalidValue;
     r_steps = (a.r + 15) / 16;
+    if (!encode_tensor_map_2d(&tA2, a.A2, a.M, kRankPad, BM, BK)) return cudaErrorInvalidValue;
+    if (a.b_mn_major) {
+      // B2 stored [r][N]
+      if (!encode_tensor_map_2d(&tB2, a.B2, a.r, a.N, static_cast<uint32_t>(16 * r_steps), 64))
+        return cudaErrorInvalidValue;
+    } else {
+      // B2 stored [N][ldb2] with r valid columns (zero filled up to 64)
+      if (!encode_tensor_map_2d(&tB2, a.B2, a.N, a.r, BN, BK, true, a.ldb2)) return cudaErrorInvalidValue;
+    }
   } else {
     tA2 = tA;
     tB2 = tB;
   }
   const int num_k = static_cast<int>((a.K + BK - 1) / BK);
-  dim3 grid(static_cast<unsigned>((a.N + BN - 1) / BN), static_cast<unsigned>((a.M + BM - 1) / BM));
-  gemm_tn_kernel<<<grid, 192, SMEM_BYTES, stream>>>(tA, tB, tA2, tB2, static_cast<int>(a.M), static_cast<int>(a.N),
-                                                     num_k, r_steps, a.D, a.accumulate, a.status);
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  const int64_t tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  if (a.b_mn_major)
+    gemm_tn_kernel<true><<<grid, 192, SMEM_BYTES, stream>>>(tA, tB, tA2, tB2, static_cast<int>(a.M),
+                                                            static_cast<int>(a.N), num_k, r_steps, a.D, a.accumulate,
+                                                            a.status);
+  else
+    gemm_tn_kernel<false><<<grid, 192, SMEM_BYTES, stream>>>(tA, tB, tA2, tB2, static_cast<int>(a.M),
+                                                             static_cast<int>(a.N), num_k, r_steps, a.D, a.accumulate,
+                                                             a.status);
   return cudaGetLastError();
 }
 

@@ -36,7 +36,7 @@ constexpr int kSegBatch = 4;   // segments loaded ahead per warp
 
 __global__ void __launch_bounds__(256) small_xa_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A,
                                                        int M, int K, int r, float* __restrict__ U32,
-                                                       uint16_t* __restrict__ U_out) {
+                                                       float* __restrict__ U_out) {
   pdl_launch_dependents();
   __shared__ float s_red[8][kGemvMaxM];
   const int j = blockIdx.x;  // rank index
@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(256) small_xa_kernel(const uint16_t* __restric
     float u = 0.0f;
     for (int w = 0; w < 8; ++w) u += s_red[w][tid];
     U32[tid * kRankPad + j] = u;
-    if (U_out != nullptr) U_out[tid * r + j] = static_cast<uint16_t>(pack_bf16x2(u, 0.0f) & 0xFFFF);
+    if (U_out != nullptr) U_out[tid * r + j] = u;
   }
 }
 
@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(WeightView w, const uint16_t*
   }
 }
 
-cudaError_t launch_small_xa(const uint16_t* X, const uint16_t* A, int M, int K, int r, float* U32, uint16_t* U_out,
+cudaError_t launch_small_xa(const uint16_t* X, const uint16_t* A, int M, int K, int r, float* U32, float* U_out,
                             cudaStream_t stream) {
   small_xa_kernel<<<r, 256, 0, stream>>>(X, A, M, K, r, U32, U_out);
   return cudaGetLastError();

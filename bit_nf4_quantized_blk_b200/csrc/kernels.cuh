@@ -49,8 +49,9 @@ constexpr int kMaxDequantBatch = 128;
 
 struct DequantBatchParams {
   int count;
-  int64_t total16;                          // 16-byte packed chunks in the batch
-  int64_t begin16[kMaxDequantBatch + 1];    // prefix sums of chunks per tensor
+  int64_t total_seg;                        // 512-byte packed segments in the batch
+  int64_t begin_seg[kMaxDequantBatch + 1];  // prefix sums of segments per tensor
+  int64_t n_words[kMaxDequantBatch];        // 32-bit packed words per tensor
   const uint8_t* packed[kMaxDequantBatch];
   const int8_t* qscale[kMaxDequantBatch];
   const float* c2[kMaxDequantBatch];
@@ -68,9 +69,9 @@ cudaError_t launch_dequant_transposed(const WeightView& w, uint16_t* out, cudaSt
 constexpr int kGemvMaxM = 16;
 
 // U[m][j] = sum_k X[m][k] * A[j][k] in fp32 for m < M <= 16 (written to
-// U32 [M][kRankPad]); optionally the bf16 copy U_out [M][r].
+// U32 [M][kRankPad]); optionally the compact copy U_out fp32 [M][r].
 cudaError_t launch_small_xa(const uint16_t* X, const uint16_t* A, int M, int K, int r, float* U32,
-                            uint16_t* U_out, cudaStream_t stream);
+                            float* U_out, cudaStream_t stream);
 // Y[m][n] = sum_k X[m][k] W[n][k] + s * sum_j U32[m][j] B[n][j].
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, int M, const uint16_t* B, int r, float scale,
                         const float* U32, uint16_t* Y, cudaStream_t stream);
@@ -80,21 +81,26 @@ cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, int M, const uin
 // ---------------------------------------------------------------------------
 
 // out[m][j] = sum_c In[m][c] * Wt(j, c) for j < r, with Wt(j, c) = Wr[j][c]
-// (row layout [r, C]) or Wc[c][j] (column layout [C, r]).  Writes
-//   o32   [M][64] fp32 (columns >= r zero)          (may be null)
+// (row layout [r, C]) or Wc[c][j] (column layout [C][ldw], r valid columns;
+// ldw * 2 bytes a multiple of 16).
+// `part` is split scratch of skinny_partial_bytes(M, C).  Writes
+//   o32   fp32 [M][o32_ld] (j < r)                   (may be null)
 //   os    [M][64] bf16 of scale * out, zero padded   (may be null)
 //   ohi / olo [M][64] bf16 split of out (hi + lo ~ fp32) (may be null)
-//   obf   [M][r] bf16 of out                         (may be null)
 struct SkinnyOut {
   float* o32;
+  int64_t o32_ld;
   uint16_t* os;
   uint16_t* ohi;
   uint16_t* olo;
-  uint16_t* obf;
   float scale;
 };
+int skinny_splits(int64_t M, int64_t C);
+size_t skinny_partial_bytes(int64_t M, int64_t C);
 cudaError_t launch_skinny(const uint16_t* In, int64_t M, int64_t C, const uint16_t* Wt, bool wt_is_rc, int r,
-                          const SkinnyOut& out, cudaStream_t stream);
+                          int64_t ldw, float* part, const SkinnyOut& out, int* status, cudaStream_t stream);
+// hi/lo bf16 split of a compact fp32 [M][r] matrix into [M][64] buffers.
+cudaError_t launch_split_hilo(const float* src, int64_t M, int r, uint16_t* hi, uint16_t* lo, cudaStream_t stream);
 
 // Column sums over tokens: out(c, j) = scale * sum_m In[m][c] * (hi[m][j] + lo[m][j]).
 // part: [ms][C][64] fp32 partials; then written to dst as [C][r] (dst_rc = false)
@@ -102,7 +108,7 @@ cudaError_t launch_skinny(const uint16_t* In, int64_t M, int64_t C, const uint16
 int colsum_splits(int64_t M, int64_t C);
 size_t colsum_partial_bytes(int64_t M, int64_t C);
 cudaError_t launch_colsum(const uint16_t* In, int64_t M, int64_t C, const uint16_t* hi, const uint16_t* lo, int r,
-                          float scale, float* part, float* dst, bool dst_rc, cudaStream_t stream);
+                          float scale, float* part, float* dst, bool dst_rc, int* status, cudaStream_t stream);
 
 // Copy a bf16 [rows][r] matrix into [rows][64] zero padded, optionally from
 // the transposed source [r][rows].
@@ -113,20 +119,22 @@ cudaError_t launch_pad_rank(const uint16_t* src, bool src_transposed, int64_t ro
 // tcgen05 GEMM (gemm_tc.cu):  D[M][N] (+)= A[M][K] B[N][K]^T + A2[M][64] B2[N][64]^T
 // ---------------------------------------------------------------------------
 struct GemmArgs {
-  const uint16_t* A;
-  const uint16_t* B;
-  const uint16_t* A2;  // may be null (no extra rank product)
-  const uint16_t* B2;
+  const uint16_t* A;   // [M][K]
+  const uint16_t* B;   // K-major: [N][ldb] (ldb = 0: K);  MN-major: [K][N]
+  const uint16_t* A2;  // [M][64] bf16, zero padded beyond r; null: no rank step
+  const uint16_t* B2;  // K-major: [N][ldb2] with r valid columns;  MN-major: [r][N]
   int64_t M, N, K;
   int r;               // rank of the extra product (<= 64)
   uint16_t* D;
   int accumulate;      // D += ... instead of D = ...
   int* status;
+  int b_mn_major;      // 0: B and B2 K-major; 1: B and B2 MN-major
+  int64_t ldb, ldb2;   // row pitches (elements) of K-major B / B2 (0: dense)
 };
 cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream);
 
 // Driver entry point used to encode TMA descriptors (resolved once).
 bool encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
-                          uint32_t box_cols);
+                          uint32_t box_cols, bool swizzle128 = true, uint64_t ld = 0);
 
 }  // namespace qnf4

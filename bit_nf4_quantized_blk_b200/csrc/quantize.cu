@@ -11,7 +11,9 @@
 //  quantize_chunks  one CTA per chunk of 256 blocks (16384 weights).  Each
 //                   group of 8 lanes owns one 64-weight block: 256-bit loads,
 //                   absmax by three xor-shuffles, IEEE fp32 division by the
-//                   absmax (by 1 for an all-zero block), nearest level from a
+//                   absmax (by 1 for an all-zero block; a reciprocal multiply
+//                   with an exact-division fallback next to a threshold),
+//                   nearest level from a
 //                   129-cell decision table, eight codes packed into one
 //                   32-bit word (even element in the low nibble).  The CTA
 //                   then forms the fp64 sum of its 256 block scales and the
@@ -73,6 +75,22 @@ __device__ __forceinline__ uint32_t nf4_code(float x, const float2* tab) {
   return static_cast<uint32_t>(__float_as_int(e.y) + (x >= e.x ? 1 : 0));
 }
 
+// Code of w / a without a division per weight.  x' = fp32(w * rcp) with
+// rcp = RN(1/a) differs from the correctly rounded quotient fp32(w / a) by
+// less than 2^-22 |x|, so both fall on the same side of every decision
+// threshold unless x' lies within that distance of one.  Every threshold is
+// far (> 2^-14 relative) from the cell edges (checked when the table is
+// built), so the only threshold that can lie that close is the one of x's
+// cell; when |x' - thr| <= 2^-19 |thr| the exact IEEE quotient decides.
+__device__ __forceinline__ uint32_t nf4_code_scaled(float w, float a, float rcp, const float2* tab) {
+  const float xa = w * rcp;
+  const int cell = __float2int_rz(xa * 64.0f) + 64;
+  const float2 e = tab[cell];
+  uint32_t code = static_cast<uint32_t>(__float_as_int(e.y) + (xa >= e.x ? 1 : 0));
+  if (fabsf(xa - e.x) <= fabsf(e.x) * 0x1p-19f) code = nf4_code(__fdiv_rn(w, a), tab);
+  return code;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(256) quantize_chunks_kernel(const __grid_constant__ QuantBatchParams p) {
@@ -126,10 +144,13 @@ __global__ void __launch_bounds__(256) quantize_chunks_kernel(const __grid_const
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
     const float div = (m == 0.0f) ? 1.0f : m;  // zero-block convention
     uint32_t word = 0;
+    if (div >= 0x1p-125f && div <= 0x1p125f) {  // 1/div is a normal fp32
+      const float rcp = __frcp_rn(div);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float x = __fdiv_rn(v[it][i], div);
-      word |= nf4_code(x, s_tab) << (4 * i);
+      for (int i = 7; i >= 0; --i) word = word * 16u + nf4_code_scaled(v[it][i], div, rcp, s_tab);
+    } else {
+#pragma unroll
+      for (int i = 7; i >= 0; --i) word = word * 16u + nf4_code(__fdiv_rn(v[it][i], div), s_tab);
     }
     if (b < nblk) {
       packed[(blk0 + b) * (kBlock / 8) + l] = word;

@@ -191,28 +191,31 @@ size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
  *   r     : 1..64.  scale : s = alpha / r (finite).
  *   ws    : 256-byte aligned workspace of qlora_linear_ws_bytes(M, N, K, r).
  *   Y     : bf16 [M, N] output (overwritten).
- *   U_out : bf16 [M, r] output X A^T (for the backward), or NULL.
+ *   U_out : fp32 [M, r] output U = X A^T (keep it for the backward), or NULL.
  * M <= 16 runs the decode-shaped dequant-GEMV; larger M the tensor-core path.
  * Accumulation is fp32.  N must be a multiple of 8.
  */
 qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t M, const uint16_t *A,
-                              const uint16_t *B, int32_t r, float scale, uint16_t *Y, uint16_t *U_out, void *ws,
+                              const uint16_t *B, int32_t r, float scale, uint16_t *Y, float *U_out, void *ws,
                               size_t ws_bytes, void *stream);
 
 /*
  * LoRA linear backward for upstream gradient dY of Y.
  *   X, dY      : bf16 [M, K] and [M, N].
+ *   U          : fp32 [M, r] = X A^T as saved by qlora_linear_fwd, or NULL to
+ *                recompute it from X and A (one more pass over X).
  *   dX         : bf16 [M, K] output, or NULL to skip.  dX = dY W + s (dY B) A.
  *   accumulate : 0 overwrites dX, 1 adds into it (dX += ...; the sum is
  *                formed in fp32 and rounded once).
  *   dA         : fp32 [r, K] output, or NULL.   dA = s (dY B)^T X.
- *   dB         : fp32 [N, r] output, or NULL.   dB = s dY^T (X A^T).
+ *   dB         : fp32 [N, r] output, or NULL.   dB = s dY^T U.
  * dA and dB are overwritten, never accumulated.  No gradient is produced for
  * the frozen weight.
  */
 qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t M,
-                              const uint16_t *A, const uint16_t *B, int32_t r, float scale, uint16_t *dX,
-                              int32_t accumulate, float *dA, float *dB, void *ws, size_t ws_bytes, void *stream);
+                              const uint16_t *A, const uint16_t *B, int32_t r, float scale, const float *U,
+                              uint16_t *dX, int32_t accumulate, float *dA, float *dB, void *ws, size_t ws_bytes,
+                              void *stream);
 
 /*
  * Kernel timing (instrumentation for benchmarks; off by default).

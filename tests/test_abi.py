@@ -93,8 +93,8 @@ def test_argument_checks_run_before_any_launch(lib):
     assert lib.qlora_nf4_dequantize(ctypes.byref(W2), 16, 2, 0, None) == 1  # bad dtype
     assert lib.qlora_linear_fwd(ctypes.byref(W2), 16, 4, 16, 16, 0, 1.0, 16, None, 256, 1 << 30, None) == 1  # r = 0
     assert lib.qlora_linear_fwd(ctypes.byref(W2), 16, 4, 16, 16, 8, 1.0, 16, None, 256, 16, None) == 4  # small ws
-    assert lib.qlora_linear_bwd(ctypes.byref(W2), 16, 16, 4, 16, 16, 8, 1.0, None, 2, None, None, 256, 1 << 30,
-                                None) == 1  # accumulate must be 0 or 1
+    assert lib.qlora_linear_bwd(ctypes.byref(W2), 16, 16, 4, 16, 16, 8, 1.0, None, None, 2, None, None, 256,
+                                1 << 30, None) == 1  # accumulate must be 0 or 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

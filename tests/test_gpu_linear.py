@@ -35,17 +35,17 @@ def _np(t):
 def _run_fwd(out, X, A, B, r, s, ws, want_u=True):
     M, N = X.shape[0], out.rows
     Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    U = torch.empty((M, r), dtype=torch.bfloat16, device="cuda") if want_u else None
+    U = torch.empty((M, r), dtype=torch.float32, device="cuda") if want_u else None
     binding.qlora_linear_fwd(out, X, A, B, r, s, Y, U, ws)
     return Y, U
 
 
-def _run_bwd(out, X, dY, A, B, r, s, ws, dX_init=None):
+def _run_bwd(out, X, dY, A, B, r, s, ws, dX_init=None, U=None):
     M, K, N = X.shape[0], out.cols, out.rows
     dX = dX_init.clone() if dX_init is not None else torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
     dA = torch.empty((r, K), dtype=torch.float32, device="cuda")
     dB = torch.empty((N, r), dtype=torch.float32, device="cuda")
-    binding.qlora_linear_bwd(out, X, dY, A, B, r, s, dX, 1 if dX_init is not None else 0, dA, dB, ws)
+    binding.qlora_linear_bwd(out, X, dY, A, B, r, s, dX, 1 if dX_init is not None else 0, dA, dB, ws, U=U)
     return dX, dA, dB
 
 
@@ -56,12 +56,12 @@ def test_tiny_config_forward_backward():
     X, A, B, dY = (t.cuda() for t in (c.X, c.A, c.B, c.dY))
     ws = workspace(16, 1024, 1024, c.r)
     Y, U = _run_fwd(out, X, A, B, c.r, c.s, ws)
-    dX, dA, dB = _run_bwd(out, X, dY, A, B, c.r, c.s, ws)
+    dX, dA, dB = _run_bwd(out, X, dY, A, B, c.r, c.s, ws, U=U)
     assert binding.qlora_workspace_status(ws) == 0
     Y_ref, U_ref = lora.lora_forward(_np(c.X), Wh, _np(c.A), _np(c.B), c.s)
     dX_ref, dA_ref, dB_ref, _ = lora.lora_backward(_np(c.X), _np(c.dY), Wh, _np(c.A), _np(c.B), c.s)
     assert_close(bf16_to_np(Y), Y_ref, "Y")
-    assert_close(bf16_to_np(U), U_ref, "U")
+    assert_close(_np(U), U_ref, "U")
     assert_close(bf16_to_np(dX), dX_ref, "dX")
     assert_close(_np(dA), dA_ref, "dA")
     assert_close(_np(dB), dB_ref, "dB")
@@ -98,16 +98,18 @@ def test_tensor_core_path_ragged(M, N, K, r):
     Y, U = _run_fwd(out, Xd, Ad, Bd, r, s, ws)
     dX, dA, dB = _run_bwd(out, Xd, dYd, Ad, Bd, r, s, ws)
     dX0 = workloads.normal_bf16((M, K), 1.0, seed + 5).cuda()
-    dXa, _, _ = _run_bwd(out, Xd, dYd, Ad, Bd, r, s, ws, dX_init=dX0)
+    dXa, dAu, dBu = _run_bwd(out, Xd, dYd, Ad, Bd, r, s, ws, dX_init=dX0, U=U)
     assert binding.qlora_workspace_status(ws) == 0
     Y_ref, U_ref = lora.lora_forward(_np(X), Wh, _np(A), _np(B), s)
     dX_ref, dA_ref, dB_ref, _ = lora.lora_backward(_np(X), _np(dY), Wh, _np(A), _np(B), s)
     assert_close(bf16_to_np(Y), Y_ref, "Y")
-    assert_close(bf16_to_np(U), U_ref, "U")
+    assert_close(_np(U), U_ref, "U")
     assert_close(bf16_to_np(dX), dX_ref, "dX")
     assert_close(bf16_to_np(dXa), dX_ref + _np(dX0), "dX accumulate")
     assert_close(_np(dA), dA_ref, "dA")
     assert_close(_np(dB), dB_ref, "dB")
+    assert_close(_np(dAu), dA_ref, "dA (saved U)")
+    assert_close(_np(dBu), dB_ref, "dB (saved U)")
 
 
 @pytest.fixture(scope="module")
@@ -127,7 +129,7 @@ def test_decode_gemv_full_gate_projection(gate7b, M):
     assert binding.qlora_workspace_status(ws) == 0
     Y_ref, U_ref = lora.lora_forward(_np(X), Wh, _np(case.A), _np(case.B), case.s)
     assert_close(bf16_to_np(Y), Y_ref, f"Y M={M}")
-    assert_close(bf16_to_np(U), U_ref, f"U M={M}")
+    assert_close(_np(U), U_ref, f"U M={M}")
 
 
 def test_decode_gemv_and_tensor_core_path_agree(gate7b):
@@ -152,8 +154,8 @@ def test_layer7b_projection_full_size(t):
     M, N, K = 8192, case.proj.n, case.proj.k
     ws = workspace(M, N, K, case.r)
     X, A, B, dY = (x.cuda() for x in (case.X, case.A, case.B, case.dY))
-    Y, _ = _run_fwd(out, X, A, B, case.r, case.s, ws, want_u=False)
-    dX, dA, dB = _run_bwd(out, X, dY, A, B, case.r, case.s, ws)
+    Y, U = _run_fwd(out, X, A, B, case.r, case.s, ws)
+    dX, dA, dB = _run_bwd(out, X, dY, A, B, case.r, case.s, ws, U=U)
     assert binding.qlora_workspace_status(ws) == 0
     rows = np.random.default_rng(100 + t).choice(M, 64, replace=False)
     Xn, An, Bn, dYn = _np(case.X), _np(case.A), _np(case.B), _np(case.dY)
