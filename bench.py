@@ -179,6 +179,18 @@ class LayerStep:
             db.copy_(dB, non_blocking=True)
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (every rank gets the same answer)."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
+
+
 def timed(fn, steps, warmup, world):
     for _ in range(warmup):
         fn()
@@ -196,9 +208,7 @@ def timed(fn, steps, warmup, world):
         dist.barrier()
     ms = start.elapsed_time(stop) / steps
     if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+        ms = max_over_ranks(ms, "cuda")
     return ms
 
 
@@ -384,12 +394,12 @@ def run_ours(args, rank, world, local_rank):
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
 
     flops = step_flops()
-    value = flops * world / (ms / 1e3) / 1e12
+    value = job_throughput(flops, world, ms) / 1e12
 
     # end-to-end through host buffers
     h2d, d2h = step.host_buffers()
     e2e_ms = timed(step.run_e2e, max(2, args.steps // 4), 1, world)
-    e2e_value = flops * world / (e2e_ms / 1e3) / 1e12
+    e2e_value = job_throughput(flops, world, e2e_ms) / 1e12
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

@@ -73,6 +73,7 @@ void derive_thresholds(float (&T)[16]) {
 bool build_decision_table(Nf4DecisionTable* tab) {
   float T[16];
   derive_thresholds(T);
+  int cells_with_threshold = 0;
   for (int c = 0; c <= 128; ++c) {
     const int t = c - 64;
     float xlo, xhi;
@@ -107,9 +108,11 @@ bool build_decision_table(Nf4DecisionTable* tab) {
       if (code_of(thr) != host_nearest(thr)) return false;
       const float below = std::nextafter(thr, -INFINITY);
       if (code_of(below) != host_nearest(below)) return false;
+      if (thr != T[base + 1]) return false;  // the cell's threshold is the next one above its base
+      ++cells_with_threshold;
     }
   }
-  return true;
+  return cells_with_threshold == 15;  // every threshold sits inside exactly one cell
 }
 
 const Nf4DecisionTable* decision_table() {
@@ -415,7 +418,7 @@ extern "C" qlora_status qlora_nf4_dequantize_batched(const qlora_nf4_weight* wei
     const qlora_status st = check_weight(&weights[i]);
     if (st != QLORA_OK) return st;
     if (outs[i] == nullptr) return QLORA_ERR_INVALID_ARG;
-    if (!aligned(outs[i], 16)) return QLORA_ERR_ALIGNMENT;
+    if (!aligned(outs[i], 32)) return QLORA_ERR_ALIGNMENT;  // 256-bit stores
   }
   qlora_status st = check_device();
   if (st != QLORA_OK) return st;
@@ -429,13 +432,13 @@ extern "C" qlora_status qlora_nf4_dequantize_batched(const qlora_nf4_weight* wei
     for (int i = 0; i < n; ++i) {
       const qlora_nf4_weight& w = weights[g0 + i];
       p.begin_seg[i] = c;
-      p.n_words[i] = w.rows * w.cols / 8;
+      p.n_units[i] = w.rows * w.cols / 32;
       p.packed[i] = w.packed;
       p.qscale[i] = w.qscale;
       p.c2[i] = w.c2;
       p.mu[i] = w.mu;
       p.out[i] = outs[g0 + i];
-      c += (p.n_words[i] + 127) / 128;
+      c += (p.n_units[i] + 127) / 128;
     }
     p.begin_seg[n] = c;
     p.total_seg = c;
@@ -518,8 +521,8 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
   DequantBatchParams p;
   std::memset(&p, 0, sizeof(p));
   p.count = 1;
-  p.n_words[0] = N * K / 8;
-  p.begin_seg[1] = p.total_seg = (p.n_words[0] + 127) / 128;
+  p.n_units[0] = N * K / 32;
+  p.begin_seg[1] = p.total_seg = (p.n_units[0] + 127) / 128;
   p.packed[0] = w->packed;
   p.qscale[0] = w->qscale;
   p.c2[0] = w->c2;
@@ -621,8 +624,8 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
     DequantBatchParams p;
     std::memset(&p, 0, sizeof(p));
     p.count = 1;
-    p.n_words[0] = N * K / 8;
-    p.begin_seg[1] = p.total_seg = (p.n_words[0] + 127) / 128;
+    p.n_units[0] = N * K / 32;
+    p.begin_seg[1] = p.total_seg = (p.n_units[0] + 127) / 128;
     p.packed[0] = w->packed;
     p.qscale[0] = w->qscale;
     p.c2[0] = w->c2;

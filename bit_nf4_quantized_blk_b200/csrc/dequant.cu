@@ -31,9 +31,10 @@ __device__ __forceinline__ int find_tensor_seg(const DequantBatchParams& p, int6
   return lo;
 }
 
-// One warp per 512-byte segment of packed codes (1024 weights, 16 blocks):
-// lane t reads the 32-bit words t, t+32, t+64, t+96 of the segment, so every
-// load and every store instruction of the warp covers one contiguous span.
+// One warp per 2 KB segment of packed codes (4096 weights): lane t loads the
+// 16-byte units t, t+32, t+64, t+96 of the segment (every load instruction of
+// the warp reads 512 contiguous bytes, all four are in flight together) and
+// writes each unit's 32 outputs with 256-bit stores (whole sectors).
 template <bool kFp32>
 __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ DequantBatchParams p) {
   __shared__ float2 s_pair[256];
@@ -44,47 +45,56 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
   if (gseg >= p.total_seg) return;
   const int t = find_tensor_seg(p, gseg);
   const int64_t seg = gseg - p.begin_seg[t];
-  const int64_t n_words = p.n_words[t];
-  const uint32_t* __restrict__ packed = reinterpret_cast<const uint32_t*>(p.packed[t]);
+  const int64_t n_units = p.n_units[t];
+  const uint4* __restrict__ packed = reinterpret_cast<const uint4*>(p.packed[t]);
   const float mu = *p.mu[t];
-  uint32_t words[4];
+  uint4 pk[4];
   float a[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const int64_t w = seg * 128 + lane + 32 * q;
-    words[q] = 0;
+    const int64_t u = seg * 128 + lane + 32 * q;
+    pk[q] = make_uint4(0, 0, 0, 0);
     a[q] = 0.0f;
-    if (w < n_words) {
-      words[q] = __ldcs(packed + w);
-      const int64_t blk = w >> 3;  // 8 words per 64-weight block
+    if (u < n_units) pk[q] = ld_stream_u4(packed + u);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int64_t u = seg * 128 + lane + 32 * q;
+    if (u < n_units) {
+      const int64_t blk = u >> 1;  // two units per 64-weight block
       a[q] = decode_scale(p.qscale[t][blk], p.c2[t][blk / kDqBlock], mu);
     }
   }
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const int64_t w = seg * 128 + lane + 32 * q;
-    if (w >= n_words) continue;
+    const int64_t u = seg * 128 + lane + 32 * q;
+    if (u >= n_units) continue;
+    const uint32_t words[4] = {pk[q].x, pk[q].y, pk[q].z, pk[q].w};
     if constexpr (kFp32) {
-      float vals[8];
+      float* o = static_cast<float*>(p.out[t]) + u * 32;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const float2 lv = s_pair[(words[q] >> (8 * b)) & 0xFF];
-        vals[2 * b] = __fmul_rn(lv.x, a[q]);
-        vals[2 * b + 1] = __fmul_rn(lv.y, a[q]);
+      for (int h = 0; h < 4; ++h) {  // 8 weights (one word) per 32-byte store
+        uint32_t vals[8];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const float2 lv = s_pair[(words[h] >> (8 * b)) & 0xFF];
+          vals[2 * b] = __float_as_uint(__fmul_rn(lv.x, a[q]));
+          vals[2 * b + 1] = __float_as_uint(__fmul_rn(lv.y, a[q]));
+        }
+        st_stream_v8(o + 8 * h, vals);
       }
-      float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out[t]) + w * 8);
-      st_stream_u4(o, make_uint4(__float_as_uint(vals[0]), __float_as_uint(vals[1]), __float_as_uint(vals[2]),
-                                 __float_as_uint(vals[3])));
-      st_stream_u4(o + 1, make_uint4(__float_as_uint(vals[4]), __float_as_uint(vals[5]), __float_as_uint(vals[6]),
-                                     __float_as_uint(vals[7])));
     } else {
-      uint32_t pr[4];
+      uint16_t* o = static_cast<uint16_t*>(p.out[t]) + u * 32;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const float2 lv = s_pair[(words[q] >> (8 * b)) & 0xFF];
-        pr[b] = pack_bf16x2(__fmul_rn(lv.x, a[q]), __fmul_rn(lv.y, a[q]));
+      for (int h = 0; h < 2; ++h) {  // 16 weights (two words) per 32-byte store
+        uint32_t pr[8];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          const float2 lv = s_pair[(words[2 * h + (b >> 2)] >> (8 * (b & 3))) & 0xFF];
+          pr[b] = pack_bf16x2(__fmul_rn(lv.x, a[q]), __fmul_rn(lv.y, a[q]));
+        }
+        st_stream_v8(o + 16 * h, pr);
       }
-      st_stream_u4(static_cast<uint16_t*>(p.out[t]) + w * 8, make_uint4(pr[0], pr[1], pr[2], pr[3]));
     }
   }
 }

@@ -5,33 +5,25 @@
 //   with Quantization", section "4. The LoRA mechanics the API wraps")
 //
 // The packed weight (0.5 B per weight) is the only large operand, so the
-// kernel is HBM-bound: it streams the codes once with 128-bit loads and never
-// writes a dequantized copy.  One CTA owns 16 weight rows; its 8 warps split
-// K into 128-wide segments.  In a segment each lane loads 16 bytes of two
-// rows (rows g and g+8, k = 32t .. 32t+31 of the segment, g = lane/4,
-// t = lane%4) and turns them directly into the A fragments of eight
-// m16n8k16 tensor-core steps; X supplies the B fragments.  Because a dot
-// product is invariant under a common permutation of k, the lane's 32
-// consecutive k values are mapped onto the fragment's k slots in whatever
-// order makes both loads contiguous: step s takes bytes 2s and 2s+1, i.e.
-// physical k = 32t + 4s + {0,1} for fragment slots {2t, 2t+1} and
-// 32t + 4s + {2,3} for slots {2t+8, 2t+9}; the X fragment is read with the
-// same map (four consecutive bf16 per step).  Each lane's 32 k values lie in
-// one 64-weight block, so one decoded scale serves them.
-//
-// Dequantized values are bit-identical to the dequantizer: fp32(L[c] * a)
-// rounded to bf16.  The rank-r term uses fp32 U = X A^T (computed by
-// small_xa_kernel, overlapped through programmatic dependent launch) and is
-// added in the fp32 epilogue after the cross-warp reduction.
+// kernel is HBM-bound: it streams the codes once and never writes a
+// dequantized copy; the tensor cores (warp MMA, m16n8k16) do the products.
+// The dequantized weight it uses is bf16(L[code]) * a, with the block scale a
+// applied in fp32 to each block's partial sum (the training path and the
+// dequantizer round fp32(L[code] * a) to bf16 instead; the difference is one
+// bf16 rounding).  The rank-r term uses fp32 U = X A^T (small_xa_kernel,
+// overlapped through programmatic dependent launch) and is added in the fp32
+// epilogue after the cross-warp reduction.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace qnf4 {
 
 namespace {
-constexpr int kGvWarps = 8;
-constexpr int kSegK = 128;     // k per segment
-constexpr int kSegBatch = 4;   // segments loaded ahead per warp
+__device__ __forceinline__ uint32_t ld_shared_u32_lut(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
 }  // namespace
 
 __global__ void __launch_bounds__(256) small_xa_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A,
@@ -77,115 +69,173 @@ __global__ void __launch_bounds__(256) small_xa_kernel(const uint16_t* __restric
   }
 }
 
-__device__ __forceinline__ uint32_t dq_pair(const float2* lut, uint32_t byte, float a) {
-  const float2 lv = lut[byte];
-  return pack_bf16x2(__fmul_rn(lv.x, a), __fmul_rn(lv.y, a));
-}
-
-template <bool kTwoTiles>
-__global__ void __launch_bounds__(256) gemv_kernel(WeightView w, const uint16_t* __restrict__ X, int M,
+// One CTA owns 32 weight rows (two 16-row MMA tiles); its 4 warps split the
+// row's 64-weight blocks.  Inside a block, lane (g = lane/4, t = lane%4)
+// loads 8 bytes of each of its 4 rows (k = 16t .. 16t+15 of the block) and
+// runs 4 k16 steps per row tile: step s takes bytes 2s and 2s+1, i.e.
+// physical k = 16t + 4s + {0,1} for fragment slots {2t, 2t+1} and
+// 16t + 4s + {2,3} for slots {2t+8, 2t+9}; X is read with the same map.  A
+// block's MMAs accumulate bf16 levels L[code] into a fresh fp32 fragment that
+// is then scaled by the block's decoded scale and added to the running sum.
+// Levels come from a byte -> (L[lo], L[hi]) bf16 pair table replicated once
+// per lane (table[byte][lane]), so the lookups never conflict.
+template <bool kTwoTok>
+__global__ void __launch_bounds__(128) gemv_kernel(WeightView w, const uint16_t* __restrict__ X, int M,
                                                    const uint16_t* __restrict__ B, int r, float scale,
                                                    const float* __restrict__ U32, uint16_t* __restrict__ Y) {
-  __shared__ float2 s_lut[256];
-  __shared__ float s_red[kGvWarps][16][16];  // [warp][row][token]
+  extern __shared__ uint32_t s_lut[];        // [256][32] bf16 pairs (32 KB)
+  __shared__ float s_red[4][32][16];          // [warp][row][token]
+  __shared__ float s_qdiv[256];               // fp32(q / 127) for q = -128 .. 127
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  for (int b = tid; b < 256; b += 256) s_lut[b] = make_float2(nf4_level(b & 15), nf4_level(b >> 4));
+  for (int e = tid; e < 256; e += 128) {
+    const uint32_t pr = pack_bf16x2(nf4_level(e & 15), nf4_level(e >> 4));
+    for (int l = 0; l < 32; ++l) s_lut[e * 32 + l] = pr;
+    s_qdiv[e] = __fdiv_rn(static_cast<float>(e - 128), 127.0f);
+  }
 
   const int64_t N = w.rows, K = w.cols;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 16;
-  const int64_t row0 = n0 + g, row1 = n0 + g + 8;
-  const bool v0 = row0 < N, v1 = row1 < N;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
   const int64_t kb = K / kBlock;  // blocks per row
+  const int64_t b_begin = kb * warp / 4, b_end = kb * (warp + 1) / 4;
   const float mu = *w.mu;
-  const int nseg = static_cast<int>((K + kSegK - 1) / kSegK);
+  // Rows of this lane: g, g+8 (tile 0), 16+g, 24+g (tile 1); row (t) is the one
+  // whose scale this lane decodes and shares.
+  int64_t rows[4];
+  bool rv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    rows[i] = n0 + g + 8 * i;
+    rv[i] = rows[i] < N;
+  }
+  const int64_t my_row = n0 + g + 8 * t;
+  const bool my_rv = my_row < N;
+  const uint32_t lut_lane = smem_u32(s_lut) + lane * 4;
   __syncthreads();
 
-  float acc[2][4];
+  float acc[2][2][4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int a = 0; a < 2; ++a)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.0f;
 
-  for (int sb = warp; sb < nseg; sb += kGvWarps * kSegBatch) {
-    uint4 wr0[kSegBatch], wr1[kSegBatch];
-    float a0[kSegBatch], a1[kSegBatch];
-    // Issue all weight loads of this batch first.
+  // Weights and scale codes of the next kAhead blocks stay in flight.
+  constexpr int kAhead = 4;
+  const int nblk = static_cast<int>(b_end - b_begin);
+  uint2 wv[kAhead][4];
+  int qv[kAhead];
+  float c2v[kAhead];
+  auto prefetch = [&](int j, int slot) {
 #pragma unroll
-    for (int u = 0; u < kSegBatch; ++u) {
-      const int seg = sb + u * kGvWarps;
-      const int64_t k = static_cast<int64_t>(seg) * kSegK + 32 * t;
-      const bool kv = seg < nseg && k < K;
-      wr0[u] = (kv && v0) ? ld_stream_u4(w.packed + (row0 * K + k) / 2) : make_uint4(0, 0, 0, 0);
-      wr1[u] = (kv && v1) ? ld_stream_u4(w.packed + (row1 * K + k) / 2) : make_uint4(0, 0, 0, 0);
-      a0[u] = 0.0f;
-      a1[u] = 0.0f;
-      if (kv && v0) {
-        const int64_t blk = row0 * kb + k / kBlock;
-        a0[u] = decode_scale(w.qscale[blk], w.c2[blk / kDqBlock], mu);
-      }
-      if (kv && v1) {
-        const int64_t blk = row1 * kb + k / kBlock;
-        a1[u] = decode_scale(w.qscale[blk], w.c2[blk / kDqBlock], mu);
+    for (int i = 0; i < 4; ++i) wv[slot][i] = make_uint2(0, 0);
+    qv[slot] = 0;
+    c2v[slot] = 0.0f;
+    if (j >= nblk) return;
+    const int64_t b = b_begin + j;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (rv[i]) {
+        const uint2* src = reinterpret_cast<const uint2*>(w.packed + (rows[i] * K + b * kBlock) / 2) + t;
+        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                     : "=r"(wv[slot][i].x), "=r"(wv[slot][i].y)
+                     : "l"(src));
       }
     }
+    if (my_rv) {
+      const int64_t blk = my_row * kb + b;
+      qv[slot] = w.qscale[blk];
+      c2v[slot] = w.c2[blk / kDqBlock];
+    }
+  };
 #pragma unroll
-    for (int u = 0; u < kSegBatch; ++u) {
-      const int seg = sb + u * kGvWarps;
-      const int64_t k = static_cast<int64_t>(seg) * kSegK + 32 * t;
-      const bool kv = seg < nseg && k < K;
-      // X fragments: 32 consecutive k of token g (tile 0) and token g+8 (tile 1).
-      uint32_t x0[16], x1[16];
+  for (int u = 0; u < kAhead; ++u) prefetch(u, u);
+
+  for (int j0 = 0; j0 < nblk; j0 += kAhead) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (kv && g < M) v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(g) * K + k) + q);
-        x0[4 * q] = v.x; x0[4 * q + 1] = v.y; x0[4 * q + 2] = v.z; x0[4 * q + 3] = v.w;
-        if constexpr (kTwoTiles) {
-          uint4 v2 = make_uint4(0, 0, 0, 0);
-          if (kv && g + 8 < M) v2 = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(g + 8) * K + k) + q);
-          x1[4 * q] = v2.x; x1[4 * q + 1] = v2.y; x1[4 * q + 2] = v2.z; x1[4 * q + 3] = v2.w;
+    for (int u = 0; u < kAhead; ++u) {
+      const int j = j0 + u;
+      if (j < nblk) {
+        const int64_t b = b_begin + j;
+        // Decoded scale of row my_row, shared with the 4 lanes of the quad.
+        const float a_mine = my_rv ? __fadd_rn(__fmul_rn(s_qdiv[qv[u] + 128], c2v[u]), mu) : 0.0f;
+        float av[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) av[i] = __shfl_sync(0xffffffffu, a_mine, (lane & ~3) | i);
+        // X fragments: 16 consecutive k of token g (tile 0) and g+8 (tile 1).
+        uint32_t xf[2][8];
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          const int tok = g + 8 * tt;
+          uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
+          if ((tt == 0 || kTwoTok) && tok < M) {
+            const uint4* xs = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(tok) * K + b * kBlock + 16 * t);
+            x0 = __ldg(xs);
+            x1 = __ldg(xs + 1);
+          }
+          xf[tt][0] = x0.x; xf[tt][1] = x0.y; xf[tt][2] = x0.z; xf[tt][3] = x0.w;
+          xf[tt][4] = x1.x; xf[tt][5] = x1.y; xf[tt][6] = x1.z; xf[tt][7] = x1.w;
         }
-      }
-      const uint32_t w0[4] = {wr0[u].x, wr0[u].y, wr0[u].z, wr0[u].w};
-      const uint32_t w1[4] = {wr1[u].x, wr1[u].y, wr1[u].z, wr1[u].w};
+        uint2 cur[4];
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const uint32_t word0 = w0[s >> 1], word1 = w1[s >> 1];
-        const int sh = (s & 1) * 16;
-        uint32_t afr[4];
-        afr[0] = dq_pair(s_lut, (word0 >> sh) & 0xFF, a0[u]);        // row g,   slots 2t, 2t+1
-        afr[1] = dq_pair(s_lut, (word1 >> sh) & 0xFF, a1[u]);        // row g+8, slots 2t, 2t+1
-        afr[2] = dq_pair(s_lut, (word0 >> (sh + 8)) & 0xFF, a0[u]);  // row g,   slots 2t+8, 2t+9
-        afr[3] = dq_pair(s_lut, (word1 >> (sh + 8)) & 0xFF, a1[u]);  // row g+8, slots 2t+8, 2t+9
-        const uint32_t b0[2] = {x0[2 * s], x0[2 * s + 1]};
-        mma_bf16_16816(acc[0], afr, b0);
-        if constexpr (kTwoTiles) {
-          const uint32_t b1[2] = {x1[2 * s], x1[2 * s + 1]};
-          mma_bf16_16816(acc[1], afr, b1);
+        for (int i = 0; i < 4; ++i) cur[i] = wv[u][i];
+        prefetch(j + kAhead, u);
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt) {
+          float d[2][4];
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) d[tt][c] = 0.0f;
+          const uint2 lo = cur[2 * rt], hi = cur[2 * rt + 1];  // rows g(+16rt), g+8(+16rt)
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const uint32_t wl = s < 2 ? lo.x : lo.y, wh = s < 2 ? hi.x : hi.y;
+            const int sh = (s & 1) * 16;
+            uint32_t afr[4];
+            afr[0] = ld_shared_u32_lut(lut_lane + ((wl >> sh) & 0xFF) * 128);
+            afr[1] = ld_shared_u32_lut(lut_lane + ((wh >> sh) & 0xFF) * 128);
+            afr[2] = ld_shared_u32_lut(lut_lane + ((wl >> (sh + 8)) & 0xFF) * 128);
+            afr[3] = ld_shared_u32_lut(lut_lane + ((wh >> (sh + 8)) & 0xFF) * 128);
+            const uint32_t b0[2] = {xf[0][2 * s], xf[0][2 * s + 1]};
+            mma_bf16_16816(d[0], afr, b0);
+            if constexpr (kTwoTok) {
+              const uint32_t b1[2] = {xf[1][2 * s], xf[1][2 * s + 1]};
+              mma_bf16_16816(d[1], afr, b1);
+            }
+          }
+#pragma unroll
+          for (int tt = 0; tt < (kTwoTok ? 2 : 1); ++tt) {
+            acc[rt][tt][0] = fmaf(av[2 * rt], d[tt][0], acc[rt][tt][0]);
+            acc[rt][tt][1] = fmaf(av[2 * rt], d[tt][1], acc[rt][tt][1]);
+            acc[rt][tt][2] = fmaf(av[2 * rt + 1], d[tt][2], acc[rt][tt][2]);
+            acc[rt][tt][3] = fmaf(av[2 * rt + 1], d[tt][3], acc[rt][tt][3]);
+          }
         }
       }
     }
   }
 
-  // Cross-warp reduction: D fragment (row g / g+8, tokens 2t, 2t+1 of each tile).
+  // Cross-warp reduction.  D fragment: rows g / g+8 of the tile, tokens 2t, 2t+1.
 #pragma unroll
-  for (int tile = 0; tile < 2; ++tile) {
-    s_red[warp][g][tile * 8 + 2 * t] = acc[tile][0];
-    s_red[warp][g][tile * 8 + 2 * t + 1] = acc[tile][1];
-    s_red[warp][g + 8][tile * 8 + 2 * t] = acc[tile][2];
-    s_red[warp][g + 8][tile * 8 + 2 * t + 1] = acc[tile][3];
-  }
+  for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      s_red[warp][16 * rt + g][tt * 8 + 2 * t] = acc[rt][tt][0];
+      s_red[warp][16 * rt + g][tt * 8 + 2 * t + 1] = acc[rt][tt][1];
+      s_red[warp][16 * rt + g + 8][tt * 8 + 2 * t] = acc[rt][tt][2];
+      s_red[warp][16 * rt + g + 8][tt * 8 + 2 * t + 1] = acc[rt][tt][3];
+    }
   __syncthreads();
   // U comes from the preceding small_xa_kernel.
   pdl_wait_prior();
-  const int row = tid & 15, tok = tid >> 4;
-  const int64_t n = n0 + row;
-  if (tok < M && n < N) {
-    float y = 0.0f;
-#pragma unroll
-    for (int wv = 0; wv < kGvWarps; ++wv) y += s_red[wv][row][tok];
+  for (int o = tid; o < 32 * 16; o += 128) {
+    const int row = o & 31, tok = o >> 5;
+    const int64_t n = n0 + row;
+    if (tok >= M || n >= N) continue;
+    float y = s_red[0][row][tok] + s_red[1][row][tok] + s_red[2][row][tok] + s_red[3][row][tok];
     float l = 0.0f;
     for (int j = 0; j < r; ++j) l = fmaf(U32[tok * kRankPad + j], bf16_bits_to_float(B[n * r + j]), l);
     y = fmaf(scale, l, y);
@@ -201,10 +251,19 @@ cudaError_t launch_small_xa(const uint16_t* X, const uint16_t* A, int M, int K, 
 
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, int M, const uint16_t* B, int r, float scale,
                         const float* U32, uint16_t* Y, cudaStream_t stream) {
+  constexpr int kLutBytes = 256 * 32 * 4;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((w.rows + 15) / 16));
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
+  cfg.gridDim = dim3(static_cast<unsigned>((w.rows + 31) / 32));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = kLutBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -49,9 +49,9 @@ constexpr int kMaxDequantBatch = 128;
 
 struct DequantBatchParams {
   int count;
-  int64_t total_seg;                        // 512-byte packed segments in the batch
+  int64_t total_seg;                        // 2 KB packed segments in the batch
   int64_t begin_seg[kMaxDequantBatch + 1];  // prefix sums of segments per tensor
-  int64_t n_words[kMaxDequantBatch];        // 32-bit packed words per tensor
+  int64_t n_units[kMaxDequantBatch];        // 16-byte packed units per tensor
   const uint8_t* packed[kMaxDequantBatch];
   const int8_t* qscale[kMaxDequantBatch];
   const float* c2[kMaxDequantBatch];

@@ -63,176 +63,232 @@ __device__ __forceinline__ bool fp64_sum_is_exact(int emin, int emax, int64_t n)
   return (emax - emin) + 24 + ceil_log2(n) <= 53;
 }
 
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float2 ld_shared_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-__device__ __forceinline__ uint32_t nf4_code(float x, const float2* tab) {
-  const int cell = __float2int_rz(x * 64.0f) + 64;  // x * 64 is exact
-  const float2 e = tab[cell];
-  return static_cast<uint32_t>(__float_as_int(e.y) + (x >= e.x ? 1 : 0));
-}
+constexpr int kQWarps = 16;                   // coding warps: 64 groups of 8 lanes
+constexpr int kQThreads = (kQWarps + 1) * 32;  // + one producer warp
+constexpr int kQStages = 3;                    // chunks in flight per CTA (64 KB each)
 
-// Code of w / a without a division per weight.  x' = fp32(w * rcp) with
-// rcp = RN(1/a) differs from the correctly rounded quotient fp32(w / a) by
-// less than 2^-22 |x|, so both fall on the same side of every decision
-// threshold unless x' lies within that distance of one.  Every threshold is
-// far (> 2^-14 relative) from the cell edges (checked when the table is
-// built), so the only threshold that can lie that close is the one of x's
-// cell; when |x' - thr| <= 2^-19 |thr| the exact IEEE quotient decides.
-__device__ __forceinline__ uint32_t nf4_code_scaled(float w, float a, float rcp, const float2* tab) {
-  const float xa = w * rcp;
-  const int cell = __float2int_rz(xa * 64.0f) + 64;
-  const float2 e = tab[cell];
-  uint32_t code = static_cast<uint32_t>(__float_as_int(e.y) + (xa >= e.x ? 1 : 0));
-  if (fabsf(xa - e.x) <= fabsf(e.x) * 0x1p-19f) code = nf4_code(__fdiv_rn(w, a), tab);
-  return code;
+struct QuantSmem {
+  float stage[kQStages][kChunkWeights];  // bulk-copied chunks of W
+  uint32_t cell_base[129][32];           // per-cell base code, one copy per lane (conflict-free)
+  float2 thr[17];                        // (64 T_j, tolerance) for j = 1..15; 256 beyond the last
+  uint64_t full[kQStages];
+  uint64_t empty[kQStages];
+  int abort_flag;
+};
+
+__device__ __forceinline__ void chunk_bounds(const QuantBatchParams& p, int64_t g, int& t, int64_t& blk0, int& nblk) {
+  t = find_tensor(p, g);
+  blk0 = (g - p.chunk_begin[t]) * kDqBlock;
+  const int64_t rem = p.n_blocks[t] - blk0;
+  nblk = static_cast<int>(rem < kDqBlock ? rem : int64_t{kDqBlock});
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(256) quantize_chunks_kernel(const __grid_constant__ QuantBatchParams p) {
-  __shared__ float2 s_tab[129];
-  __shared__ float s_absmax[kDqBlock];
-  __shared__ double s_red[8];
-  __shared__ int s_ered[16];
-  __shared__ int s_last;
+// Codes and block absmax.  Persistent: one CTA per SM walks the chunks (256
+// blocks = 16384 weights) of the batch; its last warp keeps kQStages chunks in
+// flight with 1-D bulk copies, the other 16 warps code the current one and
+// release it with one mbarrier arrival each.  Each group of 8 lanes owns a
+// block: absmax by three xor-shuffles, then per weight x' = w * (64 / a) with
+// a correctly rounded reciprocal.  x' is within 2^-22 |x| of the correctly
+// rounded 64 * fp32(w / a), so it picks the same code unless it lies within
+// the stored tolerance (2^-19 relative) of the cell's threshold; the lane's
+// block is then recoded from the IEEE quotient (so are blocks whose 64/a is
+// not a normal fp32).  Every threshold is > 2^-14 (relative) from its cell's
+// edges (checked on the host), so no other threshold can be that close.
+__global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __grid_constant__ QuantBatchParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  QuantSmem& S = *reinterpret_cast<QuantSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  const int tid = threadIdx.x;
-  const int64_t g = blockIdx.x;
-  const int t = find_tensor(p, g);
-  const int64_t local_chunk = g - p.chunk_begin[t];
-  const int64_t nb = p.n_blocks[t];
-  const int64_t blk0 = local_chunk * kDqBlock;
-  const int nblk = static_cast<int>(((nb - blk0) < kDqBlock ? (nb - blk0) : int64_t{kDqBlock}));
-  const float* __restrict__ W = p.W[t];
-  uint32_t* __restrict__ packed = reinterpret_cast<uint32_t*>(p.packed[t]);
-
-  if (tid < 129) s_tab[tid] = make_float2(p.table.thr[tid], __int_as_float(p.table.base[tid]));
-
-  const int grp = tid >> 3;  // 32 groups of 8 lanes
-  const int l = tid & 7;     // lane in group: weights 8l .. 8l+7 of the block
-
-  // Issue every load of this thread first (8 blocks x 32 bytes).
-  float v[8][8];
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int b = it * 32 + grp;
-    if (b < nblk) {
-      ld_stream_v8(W + (blk0 + b) * kBlock + l * 8, v[it]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[it][i] = 0.0f;
+  for (int i = tid; i < 129 * 32; i += kQThreads) S.cell_base[i >> 5][i & 31] = static_cast<uint32_t>(p.table.base[i >> 5]);
+  if (tid < 17) S.thr[tid] = make_float2(256.0f, 0.0f);
+  if (tid == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], kQWarps);
     }
+    S.abort_flag = 0;
+    fence_mbar_init();
   }
-  __syncthreads();  // decision table ready
+  __syncthreads();
+  if (tid < 129 && p.table.thr[tid] < 2.0f) {
+    const float t64 = p.table.thr[tid] * 64.0f;
+    S.thr[p.table.base[tid] + 1] = make_float2(t64, fabsf(t64) * 0x1p-19f);
+  }
+  __syncthreads();
 
+  if (warp == kQWarps) {  // producer
+    if (lane == 0) {
+      int it = 0;
+      for (int64_t g = blockIdx.x; g < p.total_chunks; g += gridDim.x, ++it) {
+        const int s = it % kQStages, u = it / kQStages;
+        if (it >= kQStages && !mbar_wait(&S.empty[s], (u - 1) & 1, &S.abort_flag, p.status)) break;
+        int t, nblk;
+        int64_t blk0;
+        chunk_bounds(p, g, t, blk0, nblk);
+        const uint32_t bytes = static_cast<uint32_t>(nblk) * kBlock * sizeof(float);
+        mbar_arrive_expect_tx(&S.full[s], bytes);
+        bulk_load(S.stage[s], p.W[t] + blk0 * kBlock, bytes, &S.full[s]);
+      }
+      // Copies still in flight must land before the CTA exits.
+      for (int i = (it > kQStages ? it - kQStages : 0); i < it; ++i)
+        mbar_wait_teardown(&S.full[i % kQStages], (i / kQStages) & 1, p.status);
+    }
+    return;
+  }
+
+  const int grp = tid >> 3;  // 64 groups of 8 lanes
+  const int l = tid & 7;     // lane in group: weights 8l .. 8l+7 of the block
+  const uint32_t cell_addr0 = smem_u32(&S.cell_base[64][lane]);  // cell 64 <-> x64 in (-1, 1)
+  const uint32_t thr_addr1 = smem_u32(&S.thr[1]);
   float nonfinite = 0.0f;  // becomes NaN if any input is NaN or +-Inf
+  int it = 0;
+  for (int64_t g = blockIdx.x; g < p.total_chunks; g += gridDim.x, ++it) {
+    const int s = it % kQStages;
+    int t, nblk;
+    int64_t blk0;
+    chunk_bounds(p, g, t, blk0, nblk);
+    if (!mbar_wait(&S.full[s], (it / kQStages) & 1, &S.abort_flag, p.status)) break;
+    uint32_t* __restrict__ packed = reinterpret_cast<uint32_t*>(p.packed[t]);
+#pragma unroll 1
+    for (int rep = 0; rep < kDqBlock / 64; ++rep) {
+      const int b = rep * 64 + grp;
+      float v[8];
+      if (b < nblk) {
+        const float4 v0 = *reinterpret_cast<const float4*>(&S.stage[s][b * kBlock + l * 8]);
+        const float4 v1 = *reinterpret_cast<const float4*>(&S.stage[s][b * kBlock + l * 8 + 4]);
+        v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w; v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
+      } else {
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int b = it * 32 + grp;
-    float m = 0.0f;
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+      }
+      float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      m = fmaxf(m, fabsf(v[it][i]));
-      nonfinite = fmaf(v[it][i], 0.0f, nonfinite);
-    }
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    const float div = (m == 0.0f) ? 1.0f : m;  // zero-block convention
-    uint32_t word = 0;
-    if (div >= 0x1p-125f && div <= 0x1p125f) {  // 1/div is a normal fp32
-      const float rcp = __frcp_rn(div);
+      for (int i = 0; i < 8; ++i) {
+        m = fmaxf(m, fabsf(v[i]));
+        nonfinite = fmaf(v[i], 0.0f, nonfinite);
+      }
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      const float div = (m == 0.0f) ? 1.0f : m;  // zero-block convention
+      uint32_t word = 0;
+      float slack = -1.0f;  // > 0 once some weight came within tolerance of a threshold
+      const bool fast = div >= 0x1p-121f && div <= 0x1p119f;  // 64 / div is a normal fp32
+      const float rcp64 = fast ? __frcp_rn(div) * 64.0f : 0.0f;
 #pragma unroll
-      for (int i = 7; i >= 0; --i) word = word * 16u + nf4_code_scaled(v[it][i], div, rcp, s_tab);
-    } else {
+      for (int i = 7; i >= 0; --i) {
+        const float x64 = v[i] * rcp64;
+        const uint32_t base = ld_shared_u32(cell_addr0 + static_cast<uint32_t>(__float2int_rz(x64)) * 128u);
+        const float2 thr = ld_shared_f2(thr_addr1 + base * 8u);
+        word = word * 16u + base + (x64 >= thr.x ? 1u : 0u);
+        slack = fmaxf(slack, thr.y - fabsf(x64 - thr.x));
+      }
+      if (__any_sync(0xffffffffu, !fast || slack >= 0.0f)) {
+        if (!fast || slack >= 0.0f) {
+          // Recode this lane's 8 weights from the IEEE quotients.
+          word = 0;
 #pragma unroll
-      for (int i = 7; i >= 0; --i) word = word * 16u + nf4_code(__fdiv_rn(v[it][i], div), s_tab);
-    }
-    if (b < nblk) {
-      packed[(blk0 + b) * (kBlock / 8) + l] = word;
-      if (l == 0) {
-        s_absmax[b] = m;
-        p.absmax[g * kDqBlock + b] = m;
+          for (int i = 7; i >= 0; --i) {
+            const float x64 = __fdiv_rn(v[i], div) * 64.0f;  // exact scaling
+            const uint32_t base = ld_shared_u32(cell_addr0 + static_cast<uint32_t>(__float2int_rz(x64)) * 128u);
+            const float2 thr = ld_shared_f2(thr_addr1 + base * 8u);
+            word = word * 16u + base + (x64 >= thr.x ? 1u : 0u);
+          }
+        }
+      }
+      if (b < nblk) {
+        packed[(blk0 + b) * (kBlock / 8) + l] = word;
+        if (l == 0) p.absmax[g * kDqBlock + b] = m;
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.empty[s]);  // this warp is done with stage s
   }
   if (!(nonfinite == 0.0f)) raise_status(p.status, QLORA_ERR_NONFINITE);
-  __syncthreads();
+}
 
-  // ---- fp64 sum of this chunk's block scales -------------------------------
-  const float av = tid < nblk ? s_absmax[tid] : 0.0f;
-  int emin = av > 0.0f ? exp_field(av) : 1 << 20;
-  int emax = av > 0.0f ? exp_field(av) : -(1 << 20);
+// fp64 sums of the block scales, one warp per chunk, then the tensor's mean
+// offset by the last warp to finish a chunk of that tensor.  The definition
+// is the left-to-right sum; the tree sums here are taken only when every
+// partial sum is exact (see fp64_sum_is_exact), otherwise one lane loops.
+__global__ void __launch_bounds__(256) chunk_sums_kernel(const __grid_constant__ QuantBatchParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (g >= p.total_chunks) return;
+  int t, nblk;
+  int64_t blk0;
+  chunk_bounds(p, g, t, blk0, nblk);
+  const float* a = p.absmax + g * kDqBlock;
+  double part = 0.0;
+  int emin = 1 << 20, emax = -(1 << 20);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = lane * 8 + i;
+    const float v = b < nblk ? __ldcg(a + b) : 0.0f;
+    part += static_cast<double>(v);
+    if (v > 0.0f) {
+      emin = min(emin, exp_field(v));
+      emax = max(emax, exp_field(v));
+    }
+  }
+  // Each lane's 8-term partial is exact whenever the whole chunk's sum is.
+  part = warp_sum_f64(part);
   emin = __reduce_min_sync(0xffffffffu, emin);
   emax = __reduce_max_sync(0xffffffffu, emax);
-  const double wsum = warp_sum_f64(static_cast<double>(av));
-  const int warp = tid >> 5, lane = tid & 31;
+  unsigned last = 0;
   if (lane == 0) {
-    s_red[warp] = wsum;
-    s_ered[warp] = emin;
-    s_ered[8 + warp] = emax;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int cmin = s_ered[0], cmax = s_ered[8];
-    double s = 0.0;
-    for (int w = 0; w < 8; ++w) {
-      cmin = min(cmin, s_ered[w]);
-      cmax = max(cmax, s_ered[8 + w]);
-      s += s_red[w];
+    if (!fp64_sum_is_exact(emin, emax, nblk)) {
+      part = 0.0;  // the definition: left to right
+      for (int b = 0; b < nblk; ++b) part += static_cast<double>(__ldcg(a + b));
     }
-    if (!fp64_sum_is_exact(cmin, cmax, nblk)) {
-      s = 0.0;  // the definition: left to right
-      for (int b = 0; b < nblk; ++b) s += static_cast<double>(s_absmax[b]);
-    }
-    p.chunk_sum[g] = s;
-    p.chunk_exp[2 * g] = cmin;
-    p.chunk_exp[2 * g + 1] = cmax;
+    p.chunk_sum[g] = part;
+    p.chunk_exp[2 * g] = emin;
+    p.chunk_exp[2 * g + 1] = emax;
     __threadfence();
     const unsigned n_chunks = static_cast<unsigned>(p.chunk_begin[t + 1] - p.chunk_begin[t]);
-    const unsigned ticket = atomicAdd(&p.counters[t], 1u);
-    s_last = (ticket == n_chunks - 1) ? 1 : 0;
+    last = atomicAdd(&p.counters[t], 1u) == n_chunks - 1 ? 1u : 0u;
   }
-  __syncthreads();
-  if (!s_last) return;
-
-  // ---- last CTA of tensor t: the mean offset ---------------------------------
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
   __threadfence();
   const int64_t c0 = p.chunk_begin[t], c1 = p.chunk_begin[t + 1];
-  double part = 0.0;
+  const int64_t nb = p.n_blocks[t];
+  double sum = 0.0;
   int tmin = 1 << 20, tmax = -(1 << 20);
-  for (int64_t c = c0 + tid; c < c1; c += 256) {
-    part += __ldcg(&p.chunk_sum[c]);
+  for (int64_t c = c0 + lane; c < c1; c += 32) {
+    sum += __ldcg(&p.chunk_sum[c]);
     tmin = min(tmin, __ldcg(&p.chunk_exp[2 * c]));
     tmax = max(tmax, __ldcg(&p.chunk_exp[2 * c + 1]));
   }
-  part = warp_sum_f64(part);
+  sum = warp_sum_f64(sum);
   tmin = __reduce_min_sync(0xffffffffu, tmin);
   tmax = __reduce_max_sync(0xffffffffu, tmax);
-  __syncthreads();
   if (lane == 0) {
-    s_red[warp] = part;
-    s_ered[warp] = tmin;
-    s_ered[8 + warp] = tmax;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int gmin = s_ered[0], gmax = s_ered[8];
-    double s = 0.0;
-    for (int w = 0; w < 8; ++w) {
-      gmin = min(gmin, s_ered[w]);
-      gmax = max(gmax, s_ered[8 + w]);
-      s += s_red[w];
+    if (!fp64_sum_is_exact(tmin, tmax, nb)) {
+      sum = 0.0;  // the definition: chunk sums left to right
+      for (int64_t c = c0; c < c1; ++c) sum += __ldcg(&p.chunk_sum[c]);
     }
-    if (!fp64_sum_is_exact(gmin, gmax, nb)) {
-      s = 0.0;  // the definition: chunk sums left to right
-      for (int64_t c = c0; c < c1; ++c) s += __ldcg(&p.chunk_sum[c]);
-    }
-    *p.mu[t] = __double2float_rn(s / static_cast<double>(nb));
+    *p.mu[t] = __double2float_rn(sum / static_cast<double>(nb));
     p.counters[t] = 0u;
   }
 }
@@ -281,10 +337,25 @@ __global__ void __launch_bounds__(256) dq_chunks_kernel(const __grid_constant__ 
 
 cudaError_t launch_quantize_batch(const QuantBatchParams& p, cudaStream_t stream) {
   if (p.total_chunks <= 0) return cudaSuccess;
-  quantize_chunks_kernel<<<static_cast<unsigned>(p.total_chunks), 256, 0, stream>>>(p);
+  const int smem = static_cast<int>(sizeof(QuantSmem)) + 128;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+    cudaError_t e = cudaFuncSetAttribute(quantize_codes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  const unsigned grid = static_cast<unsigned>(p.total_chunks < sms ? p.total_chunks : sms);
+  quantize_codes_kernel<<<grid, kQThreads, smem, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dq_chunks_kernel<<<static_cast<unsigned>((p.total_chunks + 7) / 8), 256, 0, stream>>>(p);
+  const unsigned warps_grid = static_cast<unsigned>((p.total_chunks + 7) / 8);
+  chunk_sums_kernel<<<warps_grid, 256, 0, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dq_chunks_kernel<<<warps_grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

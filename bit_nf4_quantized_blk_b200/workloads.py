@@ -174,3 +174,33 @@ def layer7b_case(t: int, m: int = 8192, device="cpu", layer: int = 0, config: in
                  outliers: bool = False) -> LinearCase:
     """Projection ``t`` of the training-shaped 7B layer at ``m`` tokens, r = 16, alpha = 32."""
     return linear_case(LAYER7B[t], m, 16, 32.0, config, layer, t, device, outliers=outliers)
+
+
+# ---------------------------------------------------------------------------
+# 32-layer stack of the 7B layer's projections (weights with 0.1% outliers)
+# ---------------------------------------------------------------------------
+
+STACK_CONFIG = 5
+
+
+def stack_projection(layer: int, t: int, device="cpu", r: int = 16, ab_std: float = 0.02):
+    """(W fp32, A bf16, B bf16) of projection ``t`` of stack layer ``layer``."""
+    p = LAYER7B[t]
+    seed = weight_seed(STACK_CONFIG, layer, t)
+    W = with_outliers(normal_f32((p.n, p.k), W_STD, seed, device), seed)
+    A = normal_bf16((r, p.k), ab_std, SEED_A + seed, device)
+    B = normal_bf16((p.n, r), ab_std, SEED_B + seed, device)
+    return W, A, B
+
+
+def stack_input(m: int, device="cpu") -> torch.Tensor:
+    """The stack's input activations h_0, bf16 [m, 4096] ~ N(0, 1)."""
+    return normal_bf16((m, 4096), 1.0, SEED_X + weight_seed(STACK_CONFIG, 99, 0), device)
+
+
+def stack_leaf_grad(layer: int, which: str, m: int, device="cpu") -> torch.Tensor:
+    """Seeded upstream gradients: the k and v outputs of each layer are leaves
+    ("k", "v": [m, 1024]); "top" is the gradient of the last layer's output [m, 4096]."""
+    cols = {"k": 1024, "v": 1024, "top": 4096}[which]
+    idx = {"k": 1, "v": 2, "top": 7}[which]
+    return normal_bf16((m, cols), 1.0, SEED_DY + weight_seed(STACK_CONFIG, layer, idx), device)

@@ -34,8 +34,9 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *     enqueued on it and the call returns without waiting, except where a
  *     status must be read back (see qlora_nf4_quantize).
- *   - Alignment: fp32 weights to quantize 32 bytes; packed codes, scale codes,
- *     bf16 activations and outputs 16 bytes; fp32 scalars and gradients 4.
+ *   - Alignment: fp32 weights to quantize and dense dequantize outputs 32
+ *     bytes; packed codes, scale codes, bf16 activations and outputs 16 bytes;
+ *     fp32 scalars and gradients 4.
  *     A misaligned pointer returns QLORA_ERR_ALIGNMENT.
  *   - Argument checks run on the host before anything is enqueued; a failed
  *     check returns an error status and enqueues nothing.
