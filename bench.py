@@ -22,6 +22,7 @@ number with pinned host buffers, and the CPU oracle baseline.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -43,6 +44,9 @@ R = 16
 ALPHA = 32.0
 M_TOKENS = 8192
 METRIC = "QLoRA linear fwd+bwd TFLOP/s @8192 tok; dequant-GEMV & quantize GB/s vs HBM"
+WORKLOAD = ("7B decoder layer, 7 NF4+DQ projections (q 4096x4096, k/v 1024x4096, o 4096x4096, "
+            "gate/up 14336x4096, down 4096x14336), 8192 tokens, r=16 alpha=32: "
+            "quantize+DQ, forward, backward (dX, dA, dB)")
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -70,7 +74,11 @@ def load_peaks():
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock / throttle-reason samples every 50 ms; `stop(window)`
+    keeps those stamped inside the host wall-clock window of the timed region
+    (all samples under load if none fall inside it)."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -85,11 +93,19 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.5)  # let the first samples arrive before the load starts
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def stop(self):
+    @staticmethod
+    def _stamp(text):
+        try:
+            return datetime.datetime.strptime(text.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
+
+    def stop(self, window=None):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -97,26 +113,33 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, mx, reasons = [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
+                    rows.append((self._stamp(parts[0]), float(parts[2]), float(parts[3]), parts[6:10]))
                 except ValueError:
                     continue
-                for name, val in zip(names, parts[5:9]):
-                    if val.lower() == "active":
-                        reasons.add(name)
         os.unlink(self.path)
-        if not sm:
+        inside = rows
+        scope = "all samples"
+        if window is not None:
+            sel = [r for r in rows if r[0] is not None and window[0] <= r[0] <= window[1]]
+            if sel:
+                inside, scope = sel, "timed region"
+        if not inside:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for r in inside:
+            for name, val in zip(names, r[3]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "scope": scope, "interval_ms": 50}
 
 
 # ---------------------------------------------------------------------------
@@ -191,7 +214,10 @@ def job_throughput(units_per_rank: float, world: int, ms: float) -> float:
     return units_per_rank * world / (ms / 1e3)
 
 
-def timed(fn, steps, warmup, world):
+def timed(fn, steps, warmup, world, window=None):
+    """Device time per step of `steps` calls after `warmup` untimed ones,
+    bracketed by a barrier and a synchronize; the max over ranks.  `window`
+    (a list) receives the host wall-clock span of the timed calls."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -199,11 +225,15 @@ def timed(fn, steps, warmup, world):
         dist.barrier()
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
     start.record()
     for _ in range(steps):
         fn()
     stop.record()
     torch.cuda.synchronize()
+    t1 = time.time()
+    if window is not None:
+        window[:] = [t0, t1]
     if world > 1:
         dist.barrier()
     ms = start.elapsed_time(stop) / steps
@@ -359,7 +389,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_flops() / (value * 1e12) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "7B decoder layer, 7 NF4+DQ projections, 8192 tokens, r=16 alpha=32, quantize+fwd+bwd"},
+        "config": {"workload": WORKLOAD, "flops_per_step_per_gpu": step_flops(), "parallelism": "replicas x1"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": wall,
@@ -381,8 +411,9 @@ def run_ours(args, rank, world, local_rank):
     clock = ClockSampler(int(vis.split(",")[local_rank]) if vis and vis.split(",")[0].isdigit() else local_rank)
     binding.qlora_timing_enable(True)
     clock.start()
-    ms = timed(step.run, args.steps, args.warmup, world)
-    clocks = clock.stop()
+    window = []
+    ms = timed(step.run, args.steps, args.warmup, world, window)
+    clocks = clock.stop(window)
     fam = {f: binding.qlora_timing_read(f) for f in ("quantize", "dequant", "gemv", "side", "gemm")}
     binding.qlora_timing_enable(False)
     step.check_status()
@@ -405,9 +436,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "7B decoder layer, 7 NF4+DQ projections (q 4096x4096, k/v 1024x4096, o 4096x4096, "
-                               "gate/up 14336x4096, down 4096x14336), 8192 tokens, r=16 alpha=32: "
-                               "quantize+DQ, forward, backward (dX, dA, dB)",
+        "config": {"workload": WORKLOAD,
                    "flops_per_step_per_gpu": flops, "l2": "inputs larger than L2 (GBs per step)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "gemm_tn_kernel (tcgen05 128x256 tile)",
@@ -446,7 +475,7 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")

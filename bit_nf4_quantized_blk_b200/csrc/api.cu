@@ -250,7 +250,7 @@ int64_t max_group_chunks(const qlora_nf4_weight* outs, int32_t count) {
 
 // Linear workspace layout.
 struct LinearWs {
-  size_t wbf, u32, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, total;
+  size_t wbf, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, gu, gy, total;
 };
 
 LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
@@ -263,7 +263,6 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
   };
   const size_t mr = static_cast<size_t>(M) * kRankPad;
   l.wbf = take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
-  l.u32 = take(mr * 4);
   l.us = take(mr * 2);
   l.uhi = take(mr * 2);
   l.ulo = take(mr * 2);
@@ -275,6 +274,12 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
   l.part = take(p1 > p2 ? p1 : p2);
   const size_t s1 = skinny_partial_bytes(M, N), s2 = skinny_partial_bytes(M, K);
   l.skpart = take(s1 > s2 ? s1 : s2);
+  // Decode path (M <= 16): U partials and, for K > 4096, per-chunk fp32 outputs.
+  const bool decode = M <= kGemvMaxM;
+  l.gu = take(decode ? static_cast<size_t>(gemv_upart_count(K)) * kGemvMaxM * kRankPad * 4 : 0);
+  l.gy = take(decode && gemv_chunks(K) > 1
+                  ? static_cast<size_t>(gemv_chunks(K)) * kGemvMaxM * static_cast<size_t>(N) * 4
+                  : 0);
   l.total = off;
   return l;
 }
@@ -509,13 +514,36 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
   int* status = at<int>(ws, 0);
   cudaError_t e;
   if (M <= kGemvMaxM) {
-    {
+    GemvParams gp{};
+    gp.packed = w->packed;
+    gp.qscale = w->qscale;
+    gp.c2 = w->c2;
+    gp.mu = w->mu;
+    gp.N = N;
+    gp.K = K;
+    gp.X = X;
+    gp.M = static_cast<int>(M);
+    gp.A = A;
+    gp.r = r;
+    gp.scale = scale;
+    gp.upart = at<float>(ws, lay.gu);
+    gp.n_upart = gemv_upart_count(K);
+    gp.U_out = U_out;
+    gp.Y = Y;
+    gp.ypart = at<float>(ws, lay.gy);
+    gp.status = status;
+    // B rows travel with each weight tile as one bulk copy, which needs a
+    // 16-byte aligned source; otherwise a zero-padded copy [N][64] is used.
+    const bool b_direct = aligned(B, 16) || gemv_chunks(K) > 1;
+    gp.B = b_direct ? B : at<uint16_t>(ws, lay.bpad);
+    gp.ldb = b_direct ? r : kRankPad;
+    if (!b_direct) {
       Timed tm(kFamSide, s);
-      e = launch_small_xa(X, A, static_cast<int>(M), static_cast<int>(K), r, at<float>(ws, lay.u32), U_out, s);
+      e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
+      if (e != cudaSuccess) return from_cuda(e);
     }
-    if (e != cudaSuccess) return from_cuda(e);
-    Timed tm(kFamGemv, s);
-    return from_cuda(launch_gemv(view_of(w), X, static_cast<int>(M), B, r, scale, at<float>(ws, lay.u32), Y, s));
+    Timed tm(kFamGemv, s, gemv_launches(K));
+    return from_cuda(launch_gemv(gp, s));
   }
   // Tensor-core path: dense bf16 weight, U = X A^T, padded B, GEMM with the rank-r step.
   DequantBatchParams p;

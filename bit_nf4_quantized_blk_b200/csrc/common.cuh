@@ -126,11 +126,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase of parity `parity` of `bar` has completed.  Gives up
 // after kWaitLimitNs or as soon as another thread of the CTA raised `abort`;
 // on a timeout it records QLORA_ERR_TIMEOUT and raises `abort` itself.
+// The abort flag and the clock are looked at once per 32 failed tries, so a
+// waiting warp spends its issue slots on the barrier, not on the bookkeeping.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;

@@ -34,13 +34,14 @@ __device__ __forceinline__ int find_tensor_seg(const DequantBatchParams& p, int6
 // One warp per 2 KB segment of packed codes (4096 weights): lane t loads the
 // 16-byte units t, t+32, t+64, t+96 of the segment (every load instruction of
 // the warp reads 512 contiguous bytes, all four are in flight together) and
-// writes each unit's 32 outputs with 256-bit stores (whole sectors).
+// writes each unit's 32 outputs with 256-bit stores (whole sectors).  Level
+// lookup by shuffle: lane l holds L[l % 16], and a shuffle reads its source
+// lane modulo 32, so `word >> 4i` selects L[nibble i] with no masking and no
+// shared-memory table.
 template <bool kFp32>
 __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ DequantBatchParams p) {
-  __shared__ float2 s_pair[256];
-  fill_pair_table(s_pair);
-  __syncthreads();
   const int lane = threadIdx.x & 31;
+  const float level = nf4_level(lane & 15);
   const int64_t gseg = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (gseg >= p.total_seg) return;
   const int t = find_tensor_seg(p, gseg);
@@ -65,10 +66,12 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
       a[q] = decode_scale(p.qscale[t][blk], p.c2[t][blk / kDqBlock], mu);
     }
   }
+  // Every lane takes part in the shuffles; units past the end are skipped
+  // only at the stores.
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int64_t u = seg * 128 + lane + 32 * q;
-    if (u >= n_units) continue;
+    const bool live = u < n_units;
     const uint32_t words[4] = {pk[q].x, pk[q].y, pk[q].z, pk[q].w};
     if constexpr (kFp32) {
       float* o = static_cast<float*>(p.out[t]) + u * 32;
@@ -76,12 +79,11 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
       for (int h = 0; h < 4; ++h) {  // 8 weights (one word) per 32-byte store
         uint32_t vals[8];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const float2 lv = s_pair[(words[h] >> (8 * b)) & 0xFF];
-          vals[2 * b] = __float_as_uint(__fmul_rn(lv.x, a[q]));
-          vals[2 * b + 1] = __float_as_uint(__fmul_rn(lv.y, a[q]));
+        for (int i = 0; i < 8; ++i) {
+          const float lv = __shfl_sync(0xffffffffu, level, static_cast<int>(words[h] >> (4 * i)));
+          vals[i] = __float_as_uint(__fmul_rn(lv, a[q]));
         }
-        st_stream_v8(o + 8 * h, vals);
+        if (live) st_stream_v8(o + 8 * h, vals);
       }
     } else {
       uint16_t* o = static_cast<uint16_t*>(p.out[t]) + u * 32;
@@ -90,10 +92,12 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
         uint32_t pr[8];
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
-          const float2 lv = s_pair[(words[2 * h + (b >> 2)] >> (8 * (b & 3))) & 0xFF];
-          pr[b] = pack_bf16x2(__fmul_rn(lv.x, a[q]), __fmul_rn(lv.y, a[q]));
+          const uint32_t w = words[2 * h + (b >> 2)] >> (8 * (b & 3));
+          const float lo = __shfl_sync(0xffffffffu, level, static_cast<int>(w));
+          const float hi = __shfl_sync(0xffffffffu, level, static_cast<int>(w >> 4));
+          pr[b] = pack_bf16x2(__fmul_rn(lo, a[q]), __fmul_rn(hi, a[q]));
         }
-        st_stream_v8(o + 16 * h, pr);
+        if (live) st_stream_v8(o + 16 * h, pr);
       }
     }
   }

@@ -4,274 +4,517 @@
 //   local integration", FrozenNF4LoRA.forward; "FT-02: QLoRA -- Fine-Tuning
 //   with Quantization", section "4. The LoRA mechanics the API wraps")
 //
-// The packed weight (0.5 B per weight) is the only large operand, so the
-// kernel is HBM-bound: it streams the codes once and never writes a
-// dequantized copy; the tensor cores (warp MMA, m16n8k16) do the products.
-// The dequantized weight it uses is bf16(L[code]) * a, with the block scale a
-// applied in fp32 to each block's partial sum (the training path and the
-// dequantizer round fp32(L[code] * a) to bf16 instead; the difference is one
-// bf16 rounding).  The rank-r term uses fp32 U = X A^T (small_xa_kernel,
-// overlapped through programmatic dependent launch) and is added in the fp32
-// epilogue after the cross-warp reduction.
+// The packed weight (0.5 B per weight) is the only large operand, so the path
+// is HBM-bound: it streams the codes once and never writes a dequantized
+// copy.  Three kernels:
+//
+//   xa_part_kernel   U partials: each CTA reduces X A^T over 1024 of K with
+//                    warp MMAs ([P][16][64] fp32); it releases the next
+//                    kernel at once (programmatic dependent launch).
+//   gemv_kernel      persistent, one CTA per SM, which owns a contiguous
+//                    range of 8-row tiles.  Each of its 16 warps owns one
+//                    quarter-kilo slice of K (4 blocks of 64; X held in
+//                    registers as MMA fragments) and walks every tile of the
+//                    CTA: a private ring of 16-byte cp.async copies keeps its
+//                    next 4 tile slices in flight (rows padded in shared
+//                    memory so the fragment loads never conflict), nibble
+//                    pairs are decoded through a byte -> bf16x2 table,
+//                    m16n8k16 MMAs accumulate each block and the decoded
+//                    block scale is applied to the block's fp32 partial.
+//                    Partials of 4 tiles stay in registers; then one
+//                    cross-warp reduction (two CTA barriers) sums the 16
+//                    slices, adds the rank-r term s U B^T (U from the
+//                    partials of the first kernel, the CTA's B rows copied
+//                    once) and stores Y as bf16.  No barrier sits inside a
+//                    tile, so each warp overlaps the latency of one tile's
+//                    loads, lookups and MMAs with the next.
+//   gemv_finalize    only when K > 4096: sums the per-chunk fp32 partials and
+//                    adds the rank-r term.
+//
+// The dequantized weight used is bf16(L[code]) * a, with the decoded block
+// scale a applied in fp32 to the block's partial sum (the dequantizer and the
+// training path round fp32(L[code] * a) to bf16 instead; the difference is one
+// bf16 rounding of the weight).
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace qnf4 {
 
 namespace {
-__device__ __forceinline__ uint32_t ld_shared_u32_lut(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+
+constexpr int kGvWarps = 16;
+constexpr int kGvThreads = kGvWarps * 32;
+constexpr int kGvRows = 8;                   // weight rows per tile (MMA n = 8)
+constexpr int kGvWarpBlocks = 4;             // 64-blocks of K per warp and chunk
+constexpr int kGvUnitBlocks = kGvWarps * kGvWarpBlocks;  // 64 blocks = 4096 of K per chunk
+constexpr int kGvPass = 4;                   // tiles per cross-warp reduction
+constexpr int kGvDepth = 4;                  // tile slices in flight per warp
+constexpr int kGvSlicePitch = kGvWarpBlocks * kBlock / 2 + 32;  // 160 B per row of a slice
+constexpr int kGvSliceBytes = kGvRows * kGvSlicePitch;          // 1280 B
+constexpr int kGvRedWarpBytes = kGvPass * 32 * 16 + 16;         // one warp's partials, padded
+constexpr int kGvBBytes = 16384;             // B rows of the CTA, when they fit
+
+// Shared memory.  The byte -> bf16x2 table sits at shared-window address
+// 0x10000 (64 KB): entry (byte, lane) is at 0x10000 | byte << 8 | lane << 2,
+// formed from the packed word by one permute, so a lookup is two
+// instructions and every lane reads its own bank.  Region A (below the table,
+// after the dynamic base) holds the reduction buffer, U, small tables and the
+// B rows; region C (above the table) the warps' copy rings.
+constexpr uint32_t kLutWindow = 0x10000;
+constexpr int kRedOff = 0;                                        // [16 warps][kGvRedWarpBytes]
+constexpr int kUOff = kRedOff + kGvWarps * kGvRedWarpBytes;      // [16][64] fp32
+constexpr int kQdivOff = kUOff + kGemvMaxM * kRankPad * 4;        // [256] fp32
+constexpr int kLevOff = kQdivOff + 256 * 4;                       // [16] fp32 levels
+constexpr int kBOff = kLevOff + 16 * 4;                           // [rows][ldb] bf16
+constexpr int kRegionA = kBOff + kGvBBytes;
+constexpr uint32_t kRingWindow = 2 * kLutWindow;                  // [16 warps][depth][slice]
+constexpr int kGvSmemBytes = static_cast<int>(kRingWindow) + kGvWarps * kGvDepth * kGvSliceBytes;
+
+static_assert(kBOff % 16 == 0 && kGvSliceBytes % 16 == 0 && kGvRedWarpBytes % 16 == 0, "copy alignment");
+static_assert(kRegionA + 4096 <= static_cast<int>(kLutWindow), "region A must leave room for the dynamic base");
+static_assert(kGvSmemBytes <= 227 * 1024, "shared memory budget");
+
+constexpr int kXaWarps = 16;  // U partial kernel: one 64-wide K block per warp
+
+
+// Table entry for byte J of `word`: `lane_base` = 0x10000 | 4 * lane; the
+// permute keeps its bytes 0, 2, 3 and puts byte J of `word` in byte 1.  The
+// load is left non-volatile so it schedules freely; its address depends on
+// `word`, which is read after the stage's barrier completes.
+template <int J>
+__device__ __forceinline__ uint32_t lut_pair(uint32_t word, uint32_t lane_base) {
+  uint32_t addr, v;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(addr) : "r"(lane_base), "r"(word), "n"(0x3240 + 0x10 * J));
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
+
+// m16n8k16 bf16 MMA, fp32 accumulate, without `volatile` so loads can be
+// scheduled around it.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// 16 consecutive bf16 of row `row` starting at element k (zeros if !valid).
+__device__ __forceinline__ void load16(const uint16_t* base, int64_t ld, int row, int64_t k, bool valid,
+                                       uint32_t (&w)[8]) {
+  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+  if (valid) {
+    const uint4* p = reinterpret_cast<const uint4*>(base + static_cast<int64_t>(row) * ld + k);
+    a = __ldg(p);
+    b = __ldg(p + 1);
+  }
+  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+  w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(256) small_xa_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A,
-                                                       int M, int K, int r, float* __restrict__ U32,
-                                                       float* __restrict__ U_out) {
+// Fragment k-map shared by both kernels.  In a 64-wide block, lane
+// (g = lane/4, t = lane%4) holds k = 16t .. 16t+15 of its row; k16 step s
+// takes k = 16t + 4s + {0,1} into fragment slots {2t, 2t+1} and
+// 16t + 4s + {2,3} into slots {2t+8, 2t+9}.  Both operands of every MMA use
+// the same map, so each block's 64 products are each taken exactly once.
+
+// U partials: Upart[p][m][j] = sum over k in [1024p, 1024p + 1024) of
+// X[m][k] A[j][k] (m < 16, j < 64; zeros beyond M and r).
+__global__ void __launch_bounds__(kXaWarps * 32) xa_part_kernel(const uint16_t* __restrict__ X,
+                                                                const uint16_t* __restrict__ A, int M, int64_t K,
+                                                                int r, float* __restrict__ Upart) {
   pdl_launch_dependents();
-  __shared__ float s_red[8][kGemvMaxM];
-  const int j = blockIdx.x;  // rank index
-  const int tid = threadIdx.x;
-  float acc[kGemvMaxM];
+  extern __shared__ float s_xa[];  // [16 warps][16][64]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int64_t kb = static_cast<int64_t>(blockIdx.x) * kXaWarps + warp;
+  float acc[8][4];
 #pragma unroll
-  for (int m = 0; m < kGemvMaxM; ++m) acc[m] = 0.0f;
-  for (int k = tid * 8; k < K; k += 256 * 8) {
-    const uint4 av = *reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * K + k);
-    const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+  for (int jt = 0; jt < 8; ++jt)
 #pragma unroll
-    for (int m = 0; m < kGemvMaxM; ++m) {
-      if (m < M) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * K + k);
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    for (int c = 0; c < 4; ++c) acc[jt][c] = 0.0f;
+  if (kb * kBlock < K) {
+    const int64_t k0 = kb * kBlock + 16 * t;
+    uint32_t xa[8], xb[8];
+    load16(X, K, g, k0, g < M, xa);
+    load16(X, K, g + 8, k0, g + 8 < M, xb);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[m] = fmaf(bf16_bits_to_float(xw[q] & 0xFFFF), bf16_bits_to_float(aw[q] & 0xFFFF), acc[m]);
-          acc[m] = fmaf(bf16_bits_to_float(xw[q] >> 16), bf16_bits_to_float(aw[q] >> 16), acc[m]);
+    for (int jt = 0; jt < 8; ++jt) {
+      if (8 * jt < r) {
+        uint32_t aw[8];
+        load16(A, K, 8 * jt + g, k0, 8 * jt + g < r, aw);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint32_t af[4] = {xa[2 * s], xb[2 * s], xa[2 * s + 1], xb[2 * s + 1]};
+          const uint32_t bf[2] = {aw[2 * s], aw[2 * s + 1]};
+          mma_bf16_16816(acc[jt], af, bf);
         }
       }
     }
   }
-  const int warp = tid >> 5, lane = tid & 31;
+  float* mine = s_xa + warp * (kGemvMaxM * kRankPad);
 #pragma unroll
-  for (int m = 0; m < kGemvMaxM; ++m) {
-    float v = acc[m];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) s_red[warp][m] = v;
+  for (int jt = 0; jt < 8; ++jt) {
+    *reinterpret_cast<float2*>(&mine[g * kRankPad + 8 * jt + 2 * t]) = make_float2(acc[jt][0], acc[jt][1]);
+    *reinterpret_cast<float2*>(&mine[(g + 8) * kRankPad + 8 * jt + 2 * t]) = make_float2(acc[jt][2], acc[jt][3]);
   }
   __syncthreads();
-  if (tid < M) {
-    float u = 0.0f;
-    for (int w = 0; w < 8; ++w) u += s_red[w][tid];
-    U32[tid * kRankPad + j] = u;
-    if (U_out != nullptr) U_out[tid * r + j] = u;
+  for (int e = tid; e < kGemvMaxM * kRankPad; e += kXaWarps * 32) {
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kXaWarps; ++w) v += s_xa[w * (kGemvMaxM * kRankPad) + e];
+    Upart[static_cast<int64_t>(blockIdx.x) * (kGemvMaxM * kRankPad) + e] = v;
   }
 }
 
-// One CTA owns 32 weight rows (two 16-row MMA tiles); its 4 warps split the
-// row's 64-weight blocks.  Inside a block, lane (g = lane/4, t = lane%4)
-// loads 8 bytes of each of its 4 rows (k = 16t .. 16t+15 of the block) and
-// runs 4 k16 steps per row tile: step s takes bytes 2s and 2s+1, i.e.
-// physical k = 16t + 4s + {0,1} for fragment slots {2t, 2t+1} and
-// 16t + 4s + {2,3} for slots {2t+8, 2t+9}; X is read with the same map.  A
-// block's MMAs accumulate bf16 levels L[code] into a fresh fp32 fragment that
-// is then scaled by the block's decoded scale and added to the running sum.
-// Levels come from a byte -> (L[lo], L[hi]) bf16 pair table replicated once
-// per lane (table[byte][lane]), so the lookups never conflict.
-template <bool kTwoTok>
-__global__ void __launch_bounds__(128) gemv_kernel(WeightView w, const uint16_t* __restrict__ X, int M,
-                                                   const uint16_t* __restrict__ B, int r, float scale,
-                                                   const float* __restrict__ U32, uint16_t* __restrict__ Y) {
-  extern __shared__ uint32_t s_lut[];        // [256][32] bf16 pairs (32 KB)
-  __shared__ float s_red[4][32][16];          // [warp][row][token]
-  __shared__ float s_qdiv[256];               // fp32(q / 127) for q = -128 .. 127
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-  for (int e = tid; e < 256; e += 128) {
-    const uint32_t pr = pack_bf16x2(nf4_level(e & 15), nf4_level(e >> 4));
-    for (int l = 0; l < 32; ++l) s_lut[e * 32 + l] = pr;
-    s_qdiv[e] = __fdiv_rn(static_cast<float>(e - 128), 127.0f);
+// Sum of the U partials into shared memory U_s[16][64]; the first CTA also
+// writes the caller's fp32 copy U_out [M][r].
+__device__ __forceinline__ void gather_u(const GemvParams& p, float* U_s, int tid, int nthreads) {
+  for (int e = tid; e < kGemvMaxM * kRankPad; e += nthreads) {
+    float v = 0.0f;
+    for (int q = 0; q < p.n_upart; ++q) v += p.upart[static_cast<int64_t>(q) * (kGemvMaxM * kRankPad) + e];
+    U_s[e] = v;
+    const int m = e / kRankPad, j = e % kRankPad;
+    if (blockIdx.x == 0 && p.U_out != nullptr && m < p.M && j < p.r) p.U_out[m * p.r + j] = v;
   }
+}
 
-  const int64_t N = w.rows, K = w.cols;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
-  const int64_t kb = K / kBlock;  // blocks per row
-  const int64_t b_begin = kb * warp / 4, b_end = kb * (warp + 1) / 4;
-  const float mu = *w.mu;
-  // Rows of this lane: g, g+8 (tile 0), 16+g, 24+g (tile 1); row (t) is the one
-  // whose scale this lane decodes and shares.
-  int64_t rows[4];
-  bool rv[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    rows[i] = n0 + g + 8 * i;
-    rv[i] = rows[i] < N;
+// Position of one work item of a CTA: chunk c of K, tile `tile` of rows.
+struct GvCursor {
+  int c, tile;
+  __device__ __forceinline__ void next(int t0, int t1) {
+    if (++tile == t1) {
+      tile = t0;
+      ++c;
+    }
   }
-  const int64_t my_row = n0 + g + 8 * t;
-  const bool my_rv = my_row < N;
-  const uint32_t lut_lane = smem_u32(s_lut) + lane * 4;
+};
+
+template <bool kM16>
+__global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const uint32_t base = smem_u32(smem);
+  if (base + kRegionA > kLutWindow) {  // the layout needs the dynamic base below 0x10000 - kRegionA
+    if (threadIdx.x == 0) raise_status(p.status, QLORA_ERR_UNSUPPORTED);
+    return;
+  }
+  float* const s_u = reinterpret_cast<float*>(smem + kUOff);
+  float* const s_qdiv = reinterpret_cast<float*>(smem + kQdivOff);
+  float* const s_lev = reinterpret_cast<float*>(smem + kLevOff);
+  uint16_t* const s_b = reinterpret_cast<uint16_t*>(smem + kBOff);
+  uint32_t* const lut = reinterpret_cast<uint32_t*>(smem + (kLutWindow - base));
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int64_t N = p.N, K = p.K;
+  const int64_t nbk = K / kBlock;
+  const int nchunk = static_cast<int>((nbk + kGvUnitBlocks - 1) / kGvUnitBlocks);
+  const int tiles = static_cast<int>(N / kGvRows);
+  const int t0 = static_cast<int>(static_cast<int64_t>(tiles) * blockIdx.x / gridDim.x);
+  const int t1 = static_cast<int>(static_cast<int64_t>(tiles) * (blockIdx.x + 1) / gridDim.x);
+  const int nt = t1 - t0;
+  const int items = nt * nchunk;  // chunk-major: all tiles of chunk 0, then chunk 1, ...
+  const bool single = nchunk == 1;
+  const bool b_smem = single && nt * kGvRows * p.ldb * 2 <= kGvBBytes;
+  uint8_t* const ring = smem + (kRingWindow - base) + warp * (kGvDepth * kGvSliceBytes);
+
+  // The CTA's B rows (one commit group, first of every thread).
+  if (b_smem) {
+    const int pieces = nt * p.ldb;  // 16-byte pieces: 8 rows x ldb bf16 per tile
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.B + static_cast<int64_t>(t0) * kGvRows * p.ldb);
+    for (int i = tid; i < pieces; i += kGvThreads) cp_async_16(smem + kBOff + i * 16, src + i * 16, true);
+  }
+  cp_async_commit();
+
+  // This warp's slice of item i: rows tile*8 .. +8, blocks c*64 + 4*warp ..
+  // +4 (fewer at the end of K), 8 x 16-byte pieces per row; one commit group
+  // per item and thread, empty past the last item.
+  GvCursor ic{0, t0};
+  int issued = 0;
+  auto issue_next = [&]() {
+    if (issued < items) {
+      const int64_t blkw = static_cast<int64_t>(ic.c) * kGvUnitBlocks + kGvWarpBlocks * warp;
+      const int64_t rem = nbk - blkw;
+      const int nbw = rem <= 0 ? 0 : (rem < kGvWarpBlocks ? static_cast<int>(rem) : kGvWarpBlocks);
+      uint8_t* slot = ring + (issued % kGvDepth) * kGvSliceBytes;
+      const uint8_t* src = p.packed + static_cast<int64_t>(ic.tile) * kGvRows * (K / 2) + blkw * (kBlock / 2);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int pc = lane + 32 * h, row = pc >> 3, col = pc & 7;
+        if (col < 2 * nbw) cp_async_16(slot + row * kGvSlicePitch + col * 16, src + row * (K / 2) + col * 16, true);
+      }
+      ic.next(t0, t1);
+    }
+    ++issued;
+    cp_async_commit();
+  };
+#pragma unroll 1
+  for (int i = 0; i < kGvDepth; ++i) issue_next();
+
+  if (tid < 16) s_lev[tid] = nf4_level(tid);
+  if (tid < 256) s_qdiv[tid] = __fdiv_rn(static_cast<float>(tid - 128), 127.0f);
   __syncthreads();
+  // lut[byte][64 words]: word `lane` = (L[byte & 15], L[byte >> 4]) as bf16.
+  for (int i = tid; i < 256 * 32; i += kGvThreads) {
+    const int byte = i >> 5, l = i & 31;
+    lut[byte * 64 + l] = pack_bf16x2(s_lev[byte & 15], s_lev[byte >> 4]);
+  }
 
-  float acc[2][2][4];
-#pragma unroll
-  for (int a = 0; a < 2; ++a)
-#pragma unroll
-    for (int b = 0; b < 2; ++b)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.0f;
-
-  // Weights and scale codes of the next kAhead blocks stay in flight.
-  constexpr int kAhead = 4;
-  const int nblk = static_cast<int>(b_end - b_begin);
-  uint2 wv[kAhead][4];
-  int qv[kAhead];
-  float c2v[kAhead];
-  auto prefetch = [&](int j, int slot) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) wv[slot][i] = make_uint2(0, 0);
+  const float mu = *p.mu;
+  const uint32_t lane_base = kLutWindow | (static_cast<uint32_t>(lane) * 4);
+  // Scale this lane decodes per item: row 2(lane%4) + (lane/4)%2, block
+  // 4 warp + lane/8; the quad lanes fetch theirs with two shuffles per block.
+  const int my_row = 2 * t + ((lane >> 2) & 1), my_b = lane >> 3;
+  GvCursor fc{0, t0};
+  int fetched = 0;
+  int qv[kGvDepth];
+  float c2v[kGvDepth];
+  auto fetch = [&](int slot) {
     qv[slot] = 0;
     c2v[slot] = 0.0f;
-    if (j >= nblk) return;
-    const int64_t b = b_begin + j;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (rv[i]) {
-        const uint2* src = reinterpret_cast<const uint2*>(w.packed + (rows[i] * K + b * kBlock) / 2) + t;
-        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-                     : "=r"(wv[slot][i].x), "=r"(wv[slot][i].y)
-                     : "l"(src));
+    if (fetched < items) {
+      const int64_t blk = static_cast<int64_t>(fc.c) * kGvUnitBlocks + kGvWarpBlocks * warp + my_b;
+      if (blk < nbk) {
+        const int64_t gb = (static_cast<int64_t>(fc.tile) * kGvRows + my_row) * nbk + blk;
+        qv[slot] = p.qscale[gb];
+        c2v[slot] = __ldg(p.c2 + (gb >> 8));
       }
+      fc.next(t0, t1);
     }
-    if (my_rv) {
-      const int64_t blk = my_row * kb + b;
-      qv[slot] = w.qscale[blk];
-      c2v[slot] = w.c2[blk / kDqBlock];
-    }
+    ++fetched;
   };
 #pragma unroll
-  for (int u = 0; u < kAhead; ++u) prefetch(u, u);
+  for (int i = 0; i < kGvDepth; ++i) fetch(i);
 
-  for (int j0 = 0; j0 < nblk; j0 += kAhead) {
+  // X fragments of the current chunk, in MMA operand order: xq[b][k4] = A
+  // operand of k16 step k4 of block b (tokens g and g+8).
+  uint32_t xq[kGvWarpBlocks][4][4];
+  int x_chunk = -1;
+  __syncthreads();  // table complete
+
+  GvCursor cc{0, t0};
+  bool first_reduce = true;
+  for (int i0 = 0; i0 < items;) {
+    // A pass: up to kGvPass tiles of one chunk.
+    const int c = cc.c, tile0 = cc.tile;
+    const int np = (t1 - tile0) < kGvPass ? (t1 - tile0) : kGvPass;
+    const int64_t blkw = static_cast<int64_t>(c) * kGvUnitBlocks + kGvWarpBlocks * warp;
+    const int64_t rem = nbk - blkw;
+    const int nbw = rem <= 0 ? 0 : (rem < kGvWarpBlocks ? static_cast<int>(rem) : kGvWarpBlocks);
+    if (c != x_chunk) {
 #pragma unroll
-    for (int u = 0; u < kAhead; ++u) {
-      const int j = j0 + u;
-      if (j < nblk) {
-        const int64_t b = b_begin + j;
-        // Decoded scale of row my_row, shared with the 4 lanes of the quad.
-        const float a_mine = my_rv ? __fadd_rn(__fmul_rn(s_qdiv[qv[u] + 128], c2v[u]), mu) : 0.0f;
-        float av[4];
+      for (int b = 0; b < kGvWarpBlocks; ++b) {
+        const int64_t k0 = (blkw + b) * kBlock + 16 * t;
+        uint32_t lo[8], hi[8];
+        load16(p.X, K, g, k0, b < nbw && g < p.M, lo);
+        if constexpr (kM16) {
+          load16(p.X, K, g + 8, k0, b < nbw && g + 8 < p.M, hi);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) av[i] = __shfl_sync(0xffffffffu, a_mine, (lane & ~3) | i);
-        // X fragments: 16 consecutive k of token g (tile 0) and g+8 (tile 1).
-        uint32_t xf[2][8];
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const int tok = g + 8 * tt;
-          uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
-          if ((tt == 0 || kTwoTok) && tok < M) {
-            const uint4* xs = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(tok) * K + b * kBlock + 16 * t);
-            x0 = __ldg(xs);
-            x1 = __ldg(xs + 1);
-          }
-          xf[tt][0] = x0.x; xf[tt][1] = x0.y; xf[tt][2] = x0.z; xf[tt][3] = x0.w;
-          xf[tt][4] = x1.x; xf[tt][5] = x1.y; xf[tt][6] = x1.z; xf[tt][7] = x1.w;
+          for (int e = 0; e < 8; ++e) hi[e] = 0u;
         }
-        uint2 cur[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cur[i] = wv[u][i];
-        prefetch(j + kAhead, u);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          xq[b][k4][0] = lo[2 * k4];
+          xq[b][k4][1] = hi[2 * k4];
+          xq[b][k4][2] = lo[2 * k4 + 1];
+          xq[b][k4][3] = hi[2 * k4 + 1];
+        }
+      }
+      x_chunk = c;
+    }
+
+    float acc[kGvPass][4];
 #pragma unroll
-        for (int rt = 0; rt < 2; ++rt) {
-          float d[2][4];
+    for (int j = 0; j < kGvPass; ++j) {
 #pragma unroll
-          for (int tt = 0; tt < 2; ++tt)
+      for (int e = 0; e < 4; ++e) acc[j][e] = 0.0f;
+      if (j < np) {
+        const int i = i0 + j;
+        const float a_mine = __fadd_rn(__fmul_rn(s_qdiv[qv[0] + 128], c2v[0]), mu);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) d[tt][c] = 0.0f;
-          const uint2 lo = cur[2 * rt], hi = cur[2 * rt + 1];  // rows g(+16rt), g+8(+16rt)
+        for (int e = 0; e + 1 < kGvDepth; ++e) {
+          qv[e] = qv[e + 1];
+          c2v[e] = c2v[e + 1];
+        }
+        fetch(kGvDepth - 1);
+        cp_async_wait<kGvDepth - 1>();  // item i (this lane's pieces)
+        __syncwarp();                   // ... and the other lanes' pieces
+        const uint8_t* rowp = ring + (i % kGvDepth) * kGvSliceBytes + g * kGvSlicePitch + 8 * t;
 #pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const uint32_t wl = s < 2 ? lo.x : lo.y, wh = s < 2 ? hi.x : hi.y;
-            const int sh = (s & 1) * 16;
-            uint32_t afr[4];
-            afr[0] = ld_shared_u32_lut(lut_lane + ((wl >> sh) & 0xFF) * 128);
-            afr[1] = ld_shared_u32_lut(lut_lane + ((wh >> sh) & 0xFF) * 128);
-            afr[2] = ld_shared_u32_lut(lut_lane + ((wl >> (sh + 8)) & 0xFF) * 128);
-            afr[3] = ld_shared_u32_lut(lut_lane + ((wh >> (sh + 8)) & 0xFF) * 128);
-            const uint32_t b0[2] = {xf[0][2 * s], xf[0][2 * s + 1]};
-            mma_bf16_16816(d[0], afr, b0);
-            if constexpr (kTwoTok) {
-              const uint32_t b1[2] = {xf[1][2 * s], xf[1][2 * s + 1]};
-              mma_bf16_16816(d[1], afr, b1);
+        for (int b = 0; b < kGvWarpBlocks; ++b) {
+          if (b < nbw) {
+            const uint2 wv = *reinterpret_cast<const uint2*>(rowp + b * 32);
+            uint32_t bf[4][2];
+            bf[0][0] = lut_pair<0>(wv.x, lane_base);
+            bf[0][1] = lut_pair<1>(wv.x, lane_base);
+            bf[1][0] = lut_pair<2>(wv.x, lane_base);
+            bf[1][1] = lut_pair<3>(wv.x, lane_base);
+            bf[2][0] = lut_pair<0>(wv.y, lane_base);
+            bf[2][1] = lut_pair<1>(wv.y, lane_base);
+            bf[3][0] = lut_pair<2>(wv.y, lane_base);
+            bf[3][1] = lut_pair<3>(wv.y, lane_base);
+            float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) mma_16816(d, xq[b][k4], bf[k4]);
+            // D columns 2t, 2t+1 are weight rows 2t, 2t+1 of the tile.
+            const float s_even = __shfl_sync(0xffffffffu, a_mine, b * 8 + t);
+            const float s_odd = __shfl_sync(0xffffffffu, a_mine, b * 8 + 4 + t);
+            acc[j][0] = fmaf(s_even, d[0], acc[j][0]);
+            acc[j][1] = fmaf(s_odd, d[1], acc[j][1]);
+            acc[j][2] = fmaf(s_even, d[2], acc[j][2]);
+            acc[j][3] = fmaf(s_odd, d[3], acc[j][3]);
+          }
+        }
+        __syncwarp();  // the slot is read; refill it
+        issue_next();
+      }
+    }
+
+    // Cross-warp reduction of the pass.
+    uint8_t* const red = smem + kRedOff;
+#pragma unroll
+    for (int j = 0; j < kGvPass; ++j)
+      if (j < np)
+        *reinterpret_cast<float4*>(red + warp * kGvRedWarpBytes + (j * 32 + lane) * 16) =
+            make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+    __syncthreads();
+    if (first_reduce) {  // U partials come from the preceding kernel
+      pdl_wait_prior();
+      if (single) {
+        // The B rows were this thread's oldest copy group, complete since the
+        // first item's wait; the barrier above published every thread's.
+        gather_u(p, s_u, tid, kGvThreads);
+        __syncthreads();
+      }
+      first_reduce = false;
+    }
+    // Warp w owns token w; lane = (row pair rp = lane/8, q = lane%8) sums the
+    // partials of warps 2q, 2q+1 and its share j = q, q+8, ... of the
+    // rank-r term, then three xor-shuffles finish the sum.
+    const int tok = warp;
+    if (kM16 || tok < 8) {
+      const int rp = lane >> 3, q = lane & 7;
+      const int src_lane = (tok & 7) * 4 + rp, h = tok >> 3;
+#pragma unroll
+      for (int j = 0; j < kGvPass; ++j) {
+        if (j < np) {
+          float y0 = 0.0f, y1 = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float2 v = *reinterpret_cast<const float2*>(red + (2 * q + e) * kGvRedWarpBytes +
+                                                              (j * 32 + src_lane) * 16 + 8 * h);
+            y0 += v.x;
+            y1 += v.y;
+          }
+          const int64_t n = static_cast<int64_t>(tile0 + j) * kGvRows + 2 * rp;
+          if (single) {
+            float l0 = 0.0f, l1 = 0.0f;
+            const int64_t r0 = b_smem ? (n - static_cast<int64_t>(t0) * kGvRows) : n;
+            const uint16_t* bsrc = b_smem ? s_b : p.B;
+            for (int jj = q; jj < p.r; jj += 8) {
+              const float uj = s_u[tok * kRankPad + jj];
+              l0 = fmaf(uj, bf16_bits_to_float(bsrc[r0 * p.ldb + jj]), l0);
+              l1 = fmaf(uj, bf16_bits_to_float(bsrc[(r0 + 1) * p.ldb + jj]), l1);
             }
+            y0 = fmaf(p.scale, l0, y0);
+            y1 = fmaf(p.scale, l1, y1);
           }
 #pragma unroll
-          for (int tt = 0; tt < (kTwoTok ? 2 : 1); ++tt) {
-            acc[rt][tt][0] = fmaf(av[2 * rt], d[tt][0], acc[rt][tt][0]);
-            acc[rt][tt][1] = fmaf(av[2 * rt], d[tt][1], acc[rt][tt][1]);
-            acc[rt][tt][2] = fmaf(av[2 * rt + 1], d[tt][2], acc[rt][tt][2]);
-            acc[rt][tt][3] = fmaf(av[2 * rt + 1], d[tt][3], acc[rt][tt][3]);
+          for (int o = 1; o < 8; o <<= 1) {
+            y0 += __shfl_xor_sync(0xffffffffu, y0, o);
+            y1 += __shfl_xor_sync(0xffffffffu, y1, o);
+          }
+          if (q == 0 && tok < p.M) {
+            if (single)
+              *reinterpret_cast<uint32_t*>(p.Y + static_cast<int64_t>(tok) * N + n) = pack_bf16x2(y0, y1);
+            else
+              *reinterpret_cast<float2*>(p.ypart + (static_cast<int64_t>(c) * kGemvMaxM + tok) * N + n) =
+                  make_float2(y0, y1);
           }
         }
       }
     }
+    __syncthreads();  // the reduction buffer is free again
+#pragma unroll 1
+    for (int j = 0; j < np; ++j) cc.next(t0, t1);
+    i0 += np;
   }
+  cp_async_wait<0>();
+}
 
-  // Cross-warp reduction.  D fragment: rows g / g+8 of the tile, tokens 2t, 2t+1.
-#pragma unroll
-  for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-      s_red[warp][16 * rt + g][tt * 8 + 2 * t] = acc[rt][tt][0];
-      s_red[warp][16 * rt + g][tt * 8 + 2 * t + 1] = acc[rt][tt][1];
-      s_red[warp][16 * rt + g + 8][tt * 8 + 2 * t] = acc[rt][tt][2];
-      s_red[warp][16 * rt + g + 8][tt * 8 + 2 * t + 1] = acc[rt][tt][3];
-    }
+// K > 4096: Y[m][n] = sum over chunks of the fp32 partials + s (U B^T)[m][n].
+__global__ void __launch_bounds__(256) gemv_finalize_kernel(const __grid_constant__ GemvParams p) {
+  __shared__ float s_u[kGemvMaxM * kRankPad];
+  gather_u(p, s_u, threadIdx.x, 256);
   __syncthreads();
-  // U comes from the preceding small_xa_kernel.
-  pdl_wait_prior();
-  for (int o = tid; o < 32 * 16; o += 128) {
-    const int row = o & 31, tok = o >> 5;
-    const int64_t n = n0 + row;
-    if (tok >= M || n >= N) continue;
-    float y = s_red[0][row][tok] + s_red[1][row][tok] + s_red[2][row][tok] + s_red[3][row][tok];
-    float l = 0.0f;
-    for (int j = 0; j < r; ++j) l = fmaf(U32[tok * kRankPad + j], bf16_bits_to_float(B[n * r + j]), l);
-    y = fmaf(scale, l, y);
-    Y[static_cast<int64_t>(tok) * N + n] = static_cast<uint16_t>(pack_bf16x2(y, 0.0f) & 0xFFFF);
+  const int64_t N = p.N;
+  const int nchunk = static_cast<int>((p.K / kBlock + kGvUnitBlocks - 1) / kGvUnitBlocks);
+  const int64_t pairs = static_cast<int64_t>(p.M) * (N / 2);
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < pairs;
+       e += static_cast<int64_t>(gridDim.x) * 256) {
+    const int m = static_cast<int>(e / (N / 2));
+    const int64_t n = (e % (N / 2)) * 2;
+    float y0 = 0.0f, y1 = 0.0f;
+    for (int cc = 0; cc < nchunk; ++cc) {
+      const float2 v = *reinterpret_cast<const float2*>(p.ypart + (static_cast<int64_t>(cc) * kGemvMaxM + m) * N + n);
+      y0 += v.x;
+      y1 += v.y;
+    }
+    float l0 = 0.0f, l1 = 0.0f;
+    for (int j = 0; j < p.r; ++j) {
+      const float uj = s_u[m * kRankPad + j];
+      l0 = fmaf(uj, bf16_bits_to_float(p.B[n * p.ldb + j]), l0);
+      l1 = fmaf(uj, bf16_bits_to_float(p.B[(n + 1) * p.ldb + j]), l1);
+    }
+    y0 = fmaf(p.scale, l0, y0);
+    y1 = fmaf(p.scale, l1, y1);
+    *reinterpret_cast<uint32_t*>(p.Y + static_cast<int64_t>(m) * N + n) = pack_bf16x2(y0, y1);
   }
 }
 
-cudaError_t launch_small_xa(const uint16_t* X, const uint16_t* A, int M, int K, int r, float* U32, float* U_out,
-                            cudaStream_t stream) {
-  small_xa_kernel<<<r, 256, 0, stream>>>(X, A, M, K, r, U32, U_out);
-  return cudaGetLastError();
-}
+int gemv_upart_count(int64_t K) { return static_cast<int>((K / kBlock + kXaWarps - 1) / kXaWarps); }
+int gemv_chunks(int64_t K) { return static_cast<int>((K / kBlock + kGvUnitBlocks - 1) / kGvUnitBlocks); }
 
-cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, int M, const uint16_t* B, int r, float scale,
-                        const float* U32, uint16_t* Y, cudaStream_t stream) {
-  constexpr int kLutBytes = 256 * 32 * 4;
+int gemv_launches(int64_t K) { return gemv_chunks(K) > 1 ? 3 : 2; }
+
+cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
+      e = cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(xa_part_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kXaWarps * kGemvMaxM * kRankPad * 4);
     if (e != cudaSuccess) return e;
     configured = true;
   }
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+
+  xa_part_kernel<<<p.n_upart, kXaWarps * 32, kXaWarps * kGemvMaxM * kRankPad * 4, stream>>>(p.X, p.A, p.M, p.K, p.r,
+                                                                                          p.upart);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  const int64_t tiles = p.N / kGvRows;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((w.rows + 31) / 32));
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = kLutBytes;
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms));
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = kGvSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (M > 8) return cudaLaunchKernelEx(&cfg, gemv_kernel<true>, w, X, M, B, r, scale, U32, Y);
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<false>, w, X, M, B, r, scale, U32, Y);
+  e = p.M > 8 ? cudaLaunchKernelEx(&cfg, gemv_kernel<true>, p) : cudaLaunchKernelEx(&cfg, gemv_kernel<false>, p);
+  if (e != cudaSuccess || gemv_chunks(p.K) == 1) return e;
+  const int64_t pairs = static_cast<int64_t>(p.M) * (p.N / 2);
+  const int64_t blocks = (pairs + 255) / 256;
+  gemv_finalize_kernel<<<static_cast<unsigned>(blocks < 4 * sms ? blocks : 4 * sms), 256, 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace qnf4

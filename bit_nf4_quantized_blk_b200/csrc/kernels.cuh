@@ -68,13 +68,31 @@ cudaError_t launch_dequant_transposed(const WeightView& w, uint16_t* out, cudaSt
 
 constexpr int kGemvMaxM = 16;
 
-// U[m][j] = sum_k X[m][k] * A[j][k] in fp32 for m < M <= 16 (written to
-// U32 [M][kRankPad]); optionally the compact copy U_out fp32 [M][r].
-cudaError_t launch_small_xa(const uint16_t* X, const uint16_t* A, int M, int K, int r, float* U32,
-                            float* U_out, cudaStream_t stream);
-// Y[m][n] = sum_k X[m][k] W[n][k] + s * sum_j U32[m][j] B[n][j].
-cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, int M, const uint16_t* B, int r, float scale,
-                        const float* U32, uint16_t* Y, cudaStream_t stream);
+struct GemvParams {
+  const uint8_t* packed;
+  const int8_t* qscale;
+  const float* c2;
+  const float* mu;
+  int64_t N, K;          // weight [N][K]; N % 8 == 0, K % 64 == 0
+  const uint16_t* X;     // [M][K] bf16
+  int M;                 // 1 .. 16
+  const uint16_t* A;     // [r][K] bf16
+  const uint16_t* B;     // [N][ldb] bf16, r valid columns; 16-byte aligned
+  int ldb, r;
+  float scale;
+  float* upart;          // [n_upart][16][64] fp32 scratch
+  int n_upart;           // gemv_upart_count(K)
+  float* U_out;          // [M][r] fp32, may be null
+  uint16_t* Y;           // [M][N] bf16
+  float* ypart;          // [gemv_chunks(K)][16][N] fp32 scratch (K > 4096 only)
+  int* status;
+};
+
+int gemv_upart_count(int64_t K);
+int gemv_chunks(int64_t K);
+int gemv_launches(int64_t K);
+// Y[m][n] = sum_k X[m][k] W[n][k] + s * sum_j (X A^T)[m][j] B[n][j].
+cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
 // Skinny LoRA side products (lora_side.cu)

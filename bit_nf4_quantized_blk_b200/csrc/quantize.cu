@@ -6,18 +6,19 @@
 // path"; "QLoRA Deep Dive: 4-bit NormalFloat & Double Quantization
 // Internals", section "2. Squeezing More Memory: Double Quantization (DQ)".
 //
-// Two kernels per batch of tensors:
+// Three kernels per batch of tensors:
 //
-//  quantize_chunks  one CTA per chunk of 256 blocks (16384 weights).  Each
-//                   group of 8 lanes owns one 64-weight block: 256-bit loads,
+//  quantize_codes   persistent, one CTA per SM over the chunks of 256 blocks
+//                   (16384 weights).  Each group of 8 lanes owns one 64-weight
+//                   block: 256-bit streaming loads (the next chunk in flight),
 //                   absmax by three xor-shuffles, IEEE fp32 division by the
 //                   absmax (by 1 for an all-zero block; a reciprocal multiply
 //                   with an exact-division fallback next to a threshold),
 //                   nearest level from a
 //                   129-cell decision table, eight codes packed into one
-//                   32-bit word (even element in the low nibble).  The CTA
-//                   then forms the fp64 sum of its 256 block scales and the
-//                   last CTA of each tensor forms the tensor's mean offset.
+//                   32-bit word (even element in the low nibble).
+//  chunk_sums       one warp per chunk: the fp64 sum of its 256 block scales;
+//                   the last warp of each tensor forms the tensor's mean offset.
 //  dq_chunks        one warp per chunk: d = a - mu, c2 = max|d|,
 //                   q = rint(fp32(fp32(d / c2) * 127)) (0 where c2 == 0).
 //
@@ -81,17 +82,12 @@ __device__ __forceinline__ double warp_sum_f64(double v) {
   return v;
 }
 
-constexpr int kQWarps = 16;                   // coding warps: 64 groups of 8 lanes
-constexpr int kQThreads = (kQWarps + 1) * 32;  // + one producer warp
-constexpr int kQStages = 3;                    // chunks in flight per CTA (64 KB each)
+constexpr int kQWarps = 16;  // 64 groups of 8 lanes
+constexpr int kQThreads = kQWarps * 32;
 
 struct QuantSmem {
-  float stage[kQStages][kChunkWeights];  // bulk-copied chunks of W
-  uint32_t cell_base[129][32];           // per-cell base code, one copy per lane (conflict-free)
-  float2 thr[17];                        // (64 T_j, tolerance) for j = 1..15; 256 beyond the last
-  uint64_t full[kQStages];
-  uint64_t empty[kQStages];
-  int abort_flag;
+  uint32_t cell_base[129][32];  // per-cell base code, one copy per lane (conflict-free)
+  float2 thr[17];               // (64 T_j, tolerance) for j = 1..15; 256 beyond the last
 };
 
 __device__ __forceinline__ void chunk_bounds(const QuantBatchParams& p, int64_t g, int& t, int64_t& blk0, int& nblk) {
@@ -101,34 +97,48 @@ __device__ __forceinline__ void chunk_bounds(const QuantBatchParams& p, int64_t 
   nblk = static_cast<int>(rem < kDqBlock ? rem : int64_t{kDqBlock});
 }
 
+// Weights 8l .. 8l+7 of blocks grp, grp + 64, grp + 128, grp + 192 of chunk
+// g (zeros past the tensor or the batch), with 256-bit streaming loads.
+__device__ __forceinline__ void load_chunk(const QuantBatchParams& p, int64_t g, int grp, int l, float (&v)[4][8]) {
+  int t = 0, nblk = 0;
+  int64_t blk0 = 0;
+  if (g < p.total_chunks) chunk_bounds(p, g, t, blk0, nblk);
+  const float* src = p.W[t] + (blk0 + grp) * kBlock + l * 8;
+#pragma unroll
+  for (int rep = 0; rep < 4; ++rep) {
+    if (rep * 64 + grp < nblk) {
+      ld_stream_v8(src + rep * 64 * kBlock, v[rep]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[rep][i] = 0.0f;
+    }
+  }
+}
+
 }  // namespace
 
 // Codes and block absmax.  Persistent: one CTA per SM walks the chunks (256
-// blocks = 16384 weights) of the batch; its last warp keeps kQStages chunks in
-// flight with 1-D bulk copies, the other 16 warps code the current one and
-// release it with one mbarrier arrival each.  Each group of 8 lanes owns a
-// block: absmax by three xor-shuffles, then per weight x' = w * (64 / a) with
-// a correctly rounded reciprocal.  x' is within 2^-22 |x| of the correctly
-// rounded 64 * fp32(w / a), so it picks the same code unless it lies within
-// the stored tolerance (2^-19 relative) of the cell's threshold; the lane's
-// block is then recoded from the IEEE quotient (so are blocks whose 64/a is
-// not a normal fp32).  Every threshold is > 2^-14 (relative) from its cell's
-// edges (checked on the host), so no other threshold can be that close.
+// blocks = 16384 weights) of the batch.  Every lane streams its share of the
+// next chunk into registers (256-bit loads) while it codes the current one.
+// Each group of 8 lanes owns a block: absmax by three xor-shuffles, then per
+// weight x' = w * (64 / a) with a correctly rounded reciprocal.  x' is
+// within 2^-22 |x| of the correctly rounded 64 * fp32(w / a), so it picks the
+// same code unless it lies within the stored tolerance (2^-19 relative) of
+// the cell's threshold; the lane's block is then recoded from the IEEE
+// quotient (so are blocks whose 64/a is not a normal fp32).  Every threshold
+// is > 2^-14 (relative) from its cell's edges (checked on the host), so no
+// other threshold can be that close.
 __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __grid_constant__ QuantBatchParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  QuantSmem& S = *reinterpret_cast<QuantSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ QuantSmem S;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int grp = tid >> 3;  // 64 groups of 8 lanes
+  const int l = tid & 7;     // lane in group: weights 8l .. 8l+7 of the block
+
+  float cur[4][8], nxt[4][8];
+  load_chunk(p, blockIdx.x, grp, l, cur);
 
   for (int i = tid; i < 129 * 32; i += kQThreads) S.cell_base[i >> 5][i & 31] = static_cast<uint32_t>(p.table.base[i >> 5]);
   if (tid < 17) S.thr[tid] = make_float2(256.0f, 0.0f);
-  if (tid == 0) {
-    for (int s = 0; s < kQStages; ++s) {
-      mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], kQWarps);
-    }
-    S.abort_flag = 0;
-    fence_mbar_init();
-  }
   __syncthreads();
   if (tid < 129 && p.table.thr[tid] < 2.0f) {
     const float t64 = p.table.thr[tid] * 64.0f;
@@ -136,51 +146,19 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
   }
   __syncthreads();
 
-  if (warp == kQWarps) {  // producer
-    if (lane == 0) {
-      int it = 0;
-      for (int64_t g = blockIdx.x; g < p.total_chunks; g += gridDim.x, ++it) {
-        const int s = it % kQStages, u = it / kQStages;
-        if (it >= kQStages && !mbar_wait(&S.empty[s], (u - 1) & 1, &S.abort_flag, p.status)) break;
-        int t, nblk;
-        int64_t blk0;
-        chunk_bounds(p, g, t, blk0, nblk);
-        const uint32_t bytes = static_cast<uint32_t>(nblk) * kBlock * sizeof(float);
-        mbar_arrive_expect_tx(&S.full[s], bytes);
-        bulk_load(S.stage[s], p.W[t] + blk0 * kBlock, bytes, &S.full[s]);
-      }
-      // Copies still in flight must land before the CTA exits.
-      for (int i = (it > kQStages ? it - kQStages : 0); i < it; ++i)
-        mbar_wait_teardown(&S.full[i % kQStages], (i / kQStages) & 1, p.status);
-    }
-    return;
-  }
-
-  const int grp = tid >> 3;  // 64 groups of 8 lanes
-  const int l = tid & 7;     // lane in group: weights 8l .. 8l+7 of the block
   const uint32_t cell_addr0 = smem_u32(&S.cell_base[64][lane]);  // cell 64 <-> x64 in (-1, 1)
   const uint32_t thr_addr1 = smem_u32(&S.thr[1]);
   float nonfinite = 0.0f;  // becomes NaN if any input is NaN or +-Inf
-  int it = 0;
-  for (int64_t g = blockIdx.x; g < p.total_chunks; g += gridDim.x, ++it) {
-    const int s = it % kQStages;
+  for (int64_t g = blockIdx.x; g < p.total_chunks; g += gridDim.x) {
+    load_chunk(p, g + gridDim.x, grp, l, nxt);
     int t, nblk;
     int64_t blk0;
     chunk_bounds(p, g, t, blk0, nblk);
-    if (!mbar_wait(&S.full[s], (it / kQStages) & 1, &S.abort_flag, p.status)) break;
     uint32_t* __restrict__ packed = reinterpret_cast<uint32_t*>(p.packed[t]);
-#pragma unroll 1
+#pragma unroll
     for (int rep = 0; rep < kDqBlock / 64; ++rep) {
       const int b = rep * 64 + grp;
-      float v[8];
-      if (b < nblk) {
-        const float4 v0 = *reinterpret_cast<const float4*>(&S.stage[s][b * kBlock + l * 8]);
-        const float4 v1 = *reinterpret_cast<const float4*>(&S.stage[s][b * kBlock + l * 8 + 4]);
-        v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w; v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      }
+      float (&v)[8] = cur[rep];
       float m = 0.0f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -221,8 +199,10 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
         if (l == 0) p.absmax[g * kDqBlock + b] = m;
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.empty[s]);  // this warp is done with stage s
+#pragma unroll
+    for (int rep = 0; rep < 4; ++rep)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cur[rep][i] = nxt[rep][i];
   }
   if (!(nonfinite == 0.0f)) raise_status(p.status, QLORA_ERR_NONFINITE);
 }
@@ -258,8 +238,15 @@ __global__ void __launch_bounds__(256) chunk_sums_kernel(const __grid_constant__
   unsigned last = 0;
   if (lane == 0) {
     if (!fp64_sum_is_exact(emin, emax, nblk)) {
-      part = 0.0;  // the definition: left to right
-      for (int b = 0; b < nblk; ++b) part += static_cast<double>(__ldcg(a + b));
+      part = 0.0;  // the definition: left to right (loads batched 8 ahead)
+      for (int b0 = 0; b0 < nblk; b0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = b0 + i < nblk ? __ldcg(a + b0 + i) : 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (b0 + i < nblk) part += static_cast<double>(v[i]);
+      }
     }
     p.chunk_sum[g] = part;
     p.chunk_exp[2 * g] = emin;
@@ -275,18 +262,38 @@ __global__ void __launch_bounds__(256) chunk_sums_kernel(const __grid_constant__
   const int64_t nb = p.n_blocks[t];
   double sum = 0.0;
   int tmin = 1 << 20, tmax = -(1 << 20);
-  for (int64_t c = c0 + lane; c < c1; c += 32) {
-    sum += __ldcg(&p.chunk_sum[c]);
-    tmin = min(tmin, __ldcg(&p.chunk_exp[2 * c]));
-    tmax = max(tmax, __ldcg(&p.chunk_exp[2 * c + 1]));
+  // Loads batched 8 deep per lane: the chunk sums sit in L2, and one
+  // dependent round trip per chunk would dominate the kernel.
+  for (int64_t cb = c0 + lane; cb < c1; cb += 32 * 8) {
+    double v[8];
+    int2 e[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t c = cb + 32 * i;
+      v[i] = c < c1 ? __ldcg(&p.chunk_sum[c]) : 0.0;
+      e[i] = c < c1 ? __ldcg(reinterpret_cast<const int2*>(p.chunk_exp) + c) : make_int2(1 << 20, -(1 << 20));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sum += v[i];
+      tmin = min(tmin, e[i].x);
+      tmax = max(tmax, e[i].y);
+    }
   }
   sum = warp_sum_f64(sum);
   tmin = __reduce_min_sync(0xffffffffu, tmin);
   tmax = __reduce_max_sync(0xffffffffu, tmax);
   if (lane == 0) {
     if (!fp64_sum_is_exact(tmin, tmax, nb)) {
-      sum = 0.0;  // the definition: chunk sums left to right
-      for (int64_t c = c0; c < c1; ++c) sum += __ldcg(&p.chunk_sum[c]);
+      sum = 0.0;  // the definition: chunk sums left to right (loads batched 8 ahead)
+      for (int64_t cb = c0; cb < c1; cb += 8) {
+        double v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = cb + i < c1 ? __ldcg(&p.chunk_sum[cb + i]) : 0.0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (cb + i < c1) sum += v[i];
+      }
     }
     *p.mu[t] = __double2float_rn(sum / static_cast<double>(nb));
     p.counters[t] = 0u;
@@ -337,18 +344,15 @@ __global__ void __launch_bounds__(256) dq_chunks_kernel(const __grid_constant__ 
 
 cudaError_t launch_quantize_batch(const QuantBatchParams& p, cudaStream_t stream) {
   if (p.total_chunks <= 0) return cudaSuccess;
-  const int smem = static_cast<int>(sizeof(QuantSmem)) + 128;
   static int sms = 0;
   if (sms == 0) {
     int dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
-    cudaError_t e = cudaFuncSetAttribute(quantize_codes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
   }
   const unsigned grid = static_cast<unsigned>(p.total_chunks < sms ? p.total_chunks : sms);
-  quantize_codes_kernel<<<grid, kQThreads, smem, stream>>>(p);
+  quantize_codes_kernel<<<grid, kQThreads, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const unsigned warps_grid = static_cast<unsigned>((p.total_chunks + 7) / 8);

@@ -144,6 +144,38 @@ def test_decode_gemv_and_tensor_core_path_agree(gate7b):
     assert_close(bf16_to_np(Y16), Y_ref[:16], "Y M=16")
 
 
+@pytest.mark.parametrize(
+    "M,N,K,r,b_off",
+    [
+        (3, 40, 192, 8, 0),        # K below one unit, most warps idle
+        (1, 8, 64, 1, 0),          # one block, rank 1
+        (9, 64, 1024, 64, 1),      # B not 16-byte aligned: padded copy
+        (5, 136, 4160, 24, 1),     # two chunks, the last one block wide
+        (16, 4096, 14336, 16, 0),  # 7B down projection: four chunks
+    ],
+)
+def test_decode_gemv_shapes(M, N, K, r, b_off):
+    """Decode path over ragged K (partial and multiple 4096-wide chunks), rank
+    1 .. 64 and a B whose rows start off a 16-byte boundary."""
+    seed = 7 * M + N + K + r
+    W = workloads.normal_f32((N, K), 0.02, seed)
+    A = workloads.normal_bf16((r, K), 0.02, seed + 1)
+    B = workloads.normal_bf16((N, r), 0.02, seed + 2)
+    X = workloads.normal_bf16((M, K), 1.0, seed + 3)
+    s = 2.0
+    st, Wh = _w_hat(W)
+    out = gpu_quantize(W)
+    Bbuf = torch.zeros(N * r + 8, dtype=torch.bfloat16, device="cuda")
+    Bd = Bbuf[b_off:b_off + N * r].view(N, r)
+    Bd.copy_(B.cuda())
+    ws = workspace(M, N, K, r)
+    Y, U = _run_fwd(out, X.cuda(), A.cuda(), Bd, r, s, ws)
+    assert binding.qlora_workspace_status(ws) == 0
+    Y_ref, U_ref = lora.lora_forward(_np(X), Wh, _np(A), _np(B), s)
+    assert_close(bf16_to_np(Y), Y_ref, f"Y {M}x{N}x{K} r={r}")
+    assert_close(_np(U), U_ref, f"U {M}x{N}x{K} r={r}")
+
+
 @pytest.mark.parametrize("t", range(7))
 def test_layer7b_projection_full_size(t):
     """Training-shaped 7B projection at 8192 tokens, r = 16, alpha = 32:
