@@ -35,6 +35,8 @@
 // scale a applied in fp32 to the block's partial sum (the dequantizer and the
 // training path round fp32(L[code] * a) to bf16 instead; the difference is one
 // bf16 rounding of the weight).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -44,14 +46,14 @@ namespace {
 
 constexpr int kGvWarps = 16;
 constexpr int kGvThreads = kGvWarps * 32;
-constexpr int kGvRows = 8;                   // weight rows per tile (MMA n = 8)
+constexpr int kGvRows = 16;                  // weight rows per tile (MMA m = 16)
 constexpr int kGvWarpBlocks = 4;             // 64-blocks of K per warp and chunk
 constexpr int kGvUnitBlocks = kGvWarps * kGvWarpBlocks;  // 64 blocks = 4096 of K per chunk
-constexpr int kGvPass = 4;                   // tiles per cross-warp reduction
-constexpr int kGvDepth = 4;                  // tile slices in flight per warp
+constexpr int kGvDepth = 2;                  // tile slices in flight per warp
 constexpr int kGvSlicePitch = kGvWarpBlocks * kBlock / 2 + 32;  // 160 B per row of a slice
-constexpr int kGvSliceBytes = kGvRows * kGvSlicePitch;          // 1280 B
-constexpr int kGvRedWarpBytes = kGvPass * 32 * 16 + 16;         // one warp's partials, padded
+constexpr int kGvSliceBytes = kGvRows * kGvSlicePitch;          // 2560 B
+constexpr int kGvPartFloats = 512;           // partials per warp and pass: tiles x token tiles x 32 lanes x 4
+constexpr int kGvRedWarpBytes = kGvPartFloats * 4 + 16;         // one warp's partials, padded
 constexpr int kGvBBytes = 16384;             // B rows of the CTA, when they fit
 
 // Shared memory.  The byte -> bf16x2 table sits at shared-window address
@@ -189,8 +191,17 @@ struct GvCursor {
   }
 };
 
+// Decode-shaped forward.  The weight tile is the MMA's A operand (16 rows x
+// 16 k), X the B operand (8 tokens; two token tiles for 9..16 tokens).  Lane
+// (g, t) reads 8 bytes of rows g and g+8 per block and decodes four nibble
+// pairs per k16 step; every tile runs the same straight-line code (no branch
+// inside a tile: pieces past the end are zero-filled copies, blocks past the
+// end of K meet zero X fragments).
 template <bool kM16>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
+  constexpr int NT = kM16 ? 2 : 1;  // token tiles of 8
+  constexpr int P = kM16 ? 2 : 4;   // tiles per reduction pass
+  static_assert(P * NT * 32 * 4 == kGvPartFloats, "partials layout");
   extern __shared__ __align__(16) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
   if (base + kRegionA > kLutWindow) {  // the layout needs the dynamic base below 0x10000 - kRegionA
@@ -202,47 +213,52 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
   float* const s_lev = reinterpret_cast<float*>(smem + kLevOff);
   uint16_t* const s_b = reinterpret_cast<uint16_t*>(smem + kBOff);
   uint32_t* const lut = reinterpret_cast<uint32_t*>(smem + (kLutWindow - base));
+  float* const red = reinterpret_cast<float*>(smem + kRedOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int64_t N = p.N, K = p.K;
   const int64_t nbk = K / kBlock;
   const int nchunk = static_cast<int>((nbk + kGvUnitBlocks - 1) / kGvUnitBlocks);
-  const int tiles = static_cast<int>(N / kGvRows);
+  const int tiles = static_cast<int>((N + kGvRows - 1) / kGvRows);
   const int t0 = static_cast<int>(static_cast<int64_t>(tiles) * blockIdx.x / gridDim.x);
   const int t1 = static_cast<int>(static_cast<int64_t>(tiles) * (blockIdx.x + 1) / gridDim.x);
-  const int nt = t1 - t0;
-  const int items = nt * nchunk;  // chunk-major: all tiles of chunk 0, then chunk 1, ...
+  const int items = (t1 - t0) * nchunk;  // chunk-major: all tiles of chunk 0, then chunk 1, ...
   const bool single = nchunk == 1;
-  const bool b_smem = single && nt * kGvRows * p.ldb * 2 <= kGvBBytes;
+  const int64_t row_lo = static_cast<int64_t>(t0) * kGvRows;
+  const int64_t row_hi = static_cast<int64_t>(t1) * kGvRows < N ? static_cast<int64_t>(t1) * kGvRows : N;
+  const bool b_smem = single && (row_hi - row_lo) * p.ldb * 2 <= kGvBBytes;
   uint8_t* const ring = smem + (kRingWindow - base) + warp * (kGvDepth * kGvSliceBytes);
 
-  // The CTA's B rows (one commit group, first of every thread).
+  // The CTA's B rows (one commit group, the first of every thread).
   if (b_smem) {
-    const int pieces = nt * p.ldb;  // 16-byte pieces: 8 rows x ldb bf16 per tile
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.B + static_cast<int64_t>(t0) * kGvRows * p.ldb);
+    const int pieces = static_cast<int>((row_hi - row_lo) * p.ldb / 8);  // 16-byte pieces
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.B + row_lo * p.ldb);
     for (int i = tid; i < pieces; i += kGvThreads) cp_async_16(smem + kBOff + i * 16, src + i * 16, true);
   }
   cp_async_commit();
 
-  // This warp's slice of item i: rows tile*8 .. +8, blocks c*64 + 4*warp ..
-  // +4 (fewer at the end of K), 8 x 16-byte pieces per row; one commit group
-  // per item and thread, empty past the last item.
+  // This warp's slice of item i: rows tile*16 .. +16, blocks c*64 + 4*warp
+  // .. +4, eight 16-byte pieces per row (zero-filled past N, past K or past
+  // the last item); one commit group per item and thread.
   GvCursor ic{0, t0};
   int issued = 0;
   auto issue_next = [&]() {
-    if (issued < items) {
-      const int64_t blkw = static_cast<int64_t>(ic.c) * kGvUnitBlocks + kGvWarpBlocks * warp;
-      const int64_t rem = nbk - blkw;
-      const int nbw = rem <= 0 ? 0 : (rem < kGvWarpBlocks ? static_cast<int>(rem) : kGvWarpBlocks);
-      uint8_t* slot = ring + (issued % kGvDepth) * kGvSliceBytes;
-      const uint8_t* src = p.packed + static_cast<int64_t>(ic.tile) * kGvRows * (K / 2) + blkw * (kBlock / 2);
+    const bool live = issued < items;
+    const int64_t blkw = static_cast<int64_t>(ic.c) * kGvUnitBlocks + kGvWarpBlocks * warp;
+    const int64_t rem = nbk - blkw;
+    const int nbw = !live || rem <= 0 ? 0 : (rem < kGvWarpBlocks ? static_cast<int>(rem) : kGvWarpBlocks);
+    const int64_t row0 = static_cast<int64_t>(ic.tile) * kGvRows;
+    const int64_t rows_left = N - row0;
+    const int rows_valid = rows_left < kGvRows ? static_cast<int>(rows_left) : kGvRows;
+    uint8_t* slot = ring + (issued & (kGvDepth - 1)) * kGvSliceBytes;
+    const uint8_t* src = p.packed + row0 * (K / 2) + blkw * (kBlock / 2);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int pc = lane + 32 * h, row = pc >> 3, col = pc & 7;
-        if (col < 2 * nbw) cp_async_16(slot + row * kGvSlicePitch + col * 16, src + row * (K / 2) + col * 16, true);
-      }
-      ic.next(t0, t1);
+    for (int h = 0; h < 4; ++h) {
+      const int pc = lane + 32 * h, row = pc >> 3, col = pc & 7;
+      const bool v = col < 2 * nbw && row < rows_valid;
+      cp_async_16(slot + row * kGvSlicePitch + col * 16, v ? src + row * (K / 2) + col * 16 : p.packed, v);
     }
+    if (live) ic.next(t0, t1);
     ++issued;
     cp_async_commit();
   };
@@ -260,182 +276,177 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
 
   const float mu = *p.mu;
   const uint32_t lane_base = kLutWindow | (static_cast<uint32_t>(lane) * 4);
-  // Scale this lane decodes per item: row 2(lane%4) + (lane/4)%2, block
-  // 4 warp + lane/8; the quad lanes fetch theirs with two shuffles per block.
-  const int my_row = 2 * t + ((lane >> 2) & 1), my_b = lane >> 3;
+  // Scales this lane decodes per item: row lane%16 of the tile, blocks
+  // 4 warp + lane/16 and 4 warp + lane/16 + 2; the lanes holding rows g and
+  // g+8 hand them over by shuffle.
   GvCursor fc{0, t0};
   int fetched = 0;
-  int qv[kGvDepth];
-  float c2v[kGvDepth];
+  int qv[kGvDepth][2];
+  float c2v[kGvDepth][2];
   auto fetch = [&](int slot) {
-    qv[slot] = 0;
-    c2v[slot] = 0.0f;
-    if (fetched < items) {
-      const int64_t blk = static_cast<int64_t>(fc.c) * kGvUnitBlocks + kGvWarpBlocks * warp + my_b;
-      if (blk < nbk) {
-        const int64_t gb = (static_cast<int64_t>(fc.tile) * kGvRows + my_row) * nbk + blk;
-        qv[slot] = p.qscale[gb];
-        c2v[slot] = __ldg(p.c2 + (gb >> 8));
-      }
-      fc.next(t0, t1);
+    const bool live = fetched < items;
+    const int64_t row = static_cast<int64_t>(fc.tile) * kGvRows + (lane & 15);
+    const int64_t blk = static_cast<int64_t>(fc.c) * kGvUnitBlocks + kGvWarpBlocks * warp + (lane >> 4);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const bool v = live && row < N && blk + 2 * e < nbk;
+      const int64_t gb = v ? row * nbk + blk + 2 * e : 0;
+      const int q = p.qscale[gb];
+      const float c2 = __ldg(p.c2 + (gb >> 8));
+      qv[slot][e] = v ? q : 0;
+      c2v[slot][e] = v ? c2 : 0.0f;
     }
+    if (live) fc.next(t0, t1);
     ++fetched;
   };
 #pragma unroll
   for (int i = 0; i < kGvDepth; ++i) fetch(i);
 
-  // X fragments of the current chunk, in MMA operand order: xq[b][k4] = A
-  // operand of k16 step k4 of block b (tokens g and g+8).
-  uint32_t xq[kGvWarpBlocks][4][4];
+  // X fragments of the current chunk (B operand of k16 step s of block b:
+  // words 2s, 2s+1 of the lane's 16 k of token g (+8 for the second tile).
+  uint32_t xf[NT][kGvWarpBlocks][8];
   int x_chunk = -1;
   __syncthreads();  // table complete
 
   GvCursor cc{0, t0};
   bool first_reduce = true;
-  for (int i0 = 0; i0 < items;) {
-    // A pass: up to kGvPass tiles of one chunk.
+  int item = 0;
+  auto run_pass = [&](auto np_const) {
+    constexpr int NP = decltype(np_const)::value;
     const int c = cc.c, tile0 = cc.tile;
-    const int np = (t1 - tile0) < kGvPass ? (t1 - tile0) : kGvPass;
-    const int64_t blkw = static_cast<int64_t>(c) * kGvUnitBlocks + kGvWarpBlocks * warp;
-    const int64_t rem = nbk - blkw;
-    const int nbw = rem <= 0 ? 0 : (rem < kGvWarpBlocks ? static_cast<int>(rem) : kGvWarpBlocks);
-    if (c != x_chunk) {
+    float acc[NP][NT][4];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[j][nt][e] = 0.0f;
+      const float a_lo = __fadd_rn(__fmul_rn(s_qdiv[qv[0][0] + 128], c2v[0][0]), mu);
+      const float a_hi = __fadd_rn(__fmul_rn(s_qdiv[qv[0][1] + 128], c2v[0][1]), mu);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        qv[0][e] = qv[1][e];
+        c2v[0][e] = c2v[1][e];
+      }
+      fetch(1);
+      cp_async_wait<kGvDepth - 1>();  // this item (this lane's pieces)
+      __syncwarp();                   // ... and the other lanes' pieces
+      const uint8_t* sl = ring + (item & (kGvDepth - 1)) * kGvSliceBytes + g * kGvSlicePitch + 8 * t;
 #pragma unroll
       for (int b = 0; b < kGvWarpBlocks; ++b) {
-        const int64_t k0 = (blkw + b) * kBlock + 16 * t;
-        uint32_t lo[8], hi[8];
-        load16(p.X, K, g, k0, b < nbw && g < p.M, lo);
-        if constexpr (kM16) {
-          load16(p.X, K, g + 8, k0, b < nbw && g + 8 < p.M, hi);
-        } else {
+        const uint2 wa = *reinterpret_cast<const uint2*>(sl + b * 32);
+        const uint2 wb = *reinterpret_cast<const uint2*>(sl + 8 * kGvSlicePitch + b * 32);
+        float d[NT][4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) hi[e] = 0u;
-        }
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d[nt][e] = 0.0f;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
-          xq[b][k4][0] = lo[2 * k4];
-          xq[b][k4][1] = hi[2 * k4];
-          xq[b][k4][2] = lo[2 * k4 + 1];
-          xq[b][k4][3] = hi[2 * k4 + 1];
-        }
-      }
-      x_chunk = c;
-    }
-
-    float acc[kGvPass][4];
+          const uint32_t xa = k4 < 2 ? wa.x : wa.y, xb = k4 < 2 ? wb.x : wb.y;
+          uint32_t a[4];
+          if (k4 & 1) {
+            a[0] = lut_pair<2>(xa, lane_base);
+            a[1] = lut_pair<2>(xb, lane_base);
+            a[2] = lut_pair<3>(xa, lane_base);
+            a[3] = lut_pair<3>(xb, lane_base);
+          } else {
+            a[0] = lut_pair<0>(xa, lane_base);
+            a[1] = lut_pair<0>(xb, lane_base);
+            a[2] = lut_pair<1>(xa, lane_base);
+            a[3] = lut_pair<1>(xb, lane_base);
+          }
 #pragma unroll
-    for (int j = 0; j < kGvPass; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[j][e] = 0.0f;
-      if (j < np) {
-        const int i = i0 + j;
-        const float a_mine = __fadd_rn(__fmul_rn(s_qdiv[qv[0] + 128], c2v[0]), mu);
-#pragma unroll
-        for (int e = 0; e + 1 < kGvDepth; ++e) {
-          qv[e] = qv[e + 1];
-          c2v[e] = c2v[e + 1];
-        }
-        fetch(kGvDepth - 1);
-        cp_async_wait<kGvDepth - 1>();  // item i (this lane's pieces)
-        __syncwarp();                   // ... and the other lanes' pieces
-        const uint8_t* rowp = ring + (i % kGvDepth) * kGvSliceBytes + g * kGvSlicePitch + 8 * t;
-#pragma unroll
-        for (int b = 0; b < kGvWarpBlocks; ++b) {
-          if (b < nbw) {
-            const uint2 wv = *reinterpret_cast<const uint2*>(rowp + b * 32);
-            uint32_t bf[4][2];
-            bf[0][0] = lut_pair<0>(wv.x, lane_base);
-            bf[0][1] = lut_pair<1>(wv.x, lane_base);
-            bf[1][0] = lut_pair<2>(wv.x, lane_base);
-            bf[1][1] = lut_pair<3>(wv.x, lane_base);
-            bf[2][0] = lut_pair<0>(wv.y, lane_base);
-            bf[2][1] = lut_pair<1>(wv.y, lane_base);
-            bf[3][0] = lut_pair<2>(wv.y, lane_base);
-            bf[3][1] = lut_pair<3>(wv.y, lane_base);
-            float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) mma_16816(d, xq[b][k4], bf[k4]);
-            // D columns 2t, 2t+1 are weight rows 2t, 2t+1 of the tile.
-            const float s_even = __shfl_sync(0xffffffffu, a_mine, b * 8 + t);
-            const float s_odd = __shfl_sync(0xffffffffu, a_mine, b * 8 + 4 + t);
-            acc[j][0] = fmaf(s_even, d[0], acc[j][0]);
-            acc[j][1] = fmaf(s_odd, d[1], acc[j][1]);
-            acc[j][2] = fmaf(s_even, d[2], acc[j][2]);
-            acc[j][3] = fmaf(s_odd, d[3], acc[j][3]);
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint32_t bx[2] = {xf[nt][b][2 * k4], xf[nt][b][2 * k4 + 1]};
+            mma_16816(d[nt], a, bx);
           }
         }
-        __syncwarp();  // the slot is read; refill it
-        issue_next();
+        // D rows g and g+8 are weight rows g and g+8 of the tile.
+        const float sv = b < 2 ? a_lo : a_hi;
+        const float s_g = __shfl_sync(0xffffffffu, sv, g + 16 * (b & 1));
+        const float s_g8 = __shfl_sync(0xffffffffu, sv, g + 8 + 16 * (b & 1));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          acc[j][nt][0] = fmaf(s_g, d[nt][0], acc[j][nt][0]);
+          acc[j][nt][1] = fmaf(s_g, d[nt][1], acc[j][nt][1]);
+          acc[j][nt][2] = fmaf(s_g8, d[nt][2], acc[j][nt][2]);
+          acc[j][nt][3] = fmaf(s_g8, d[nt][3], acc[j][nt][3]);
+        }
       }
+      __syncwarp();  // the slot is read; refill it
+      issue_next();
+      ++item;
     }
 
-    // Cross-warp reduction of the pass.
-    uint8_t* const red = smem + kRedOff;
+    // Cross-warp reduction: thread tau sums float tau of the 16 warps'
+    // partials ([tile][token tile][lane][4]).
 #pragma unroll
-    for (int j = 0; j < kGvPass; ++j)
-      if (j < np)
-        *reinterpret_cast<float4*>(red + warp * kGvRedWarpBytes + (j * 32 + lane) * 16) =
-            make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+    for (int j = 0; j < NP; ++j)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        *reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(red) + warp * kGvRedWarpBytes +
+                                   ((j * NT + nt) * 32 + lane) * 16) =
+            make_float4(acc[j][nt][0], acc[j][nt][1], acc[j][nt][2], acc[j][nt][3]);
     __syncthreads();
     if (first_reduce) {  // U partials come from the preceding kernel
       pdl_wait_prior();
       if (single) {
-        // The B rows were this thread's oldest copy group, complete since the
+        // The B rows were this thread's oldest copy group, complete since its
         // first item's wait; the barrier above published every thread's.
         gather_u(p, s_u, tid, kGvThreads);
         __syncthreads();
       }
       first_reduce = false;
     }
-    // Warp w owns token w; lane = (row pair rp = lane/8, q = lane%8) sums the
-    // partials of warps 2q, 2q+1 and its share j = q, q+8, ... of the
-    // rank-r term, then three xor-shuffles finish the sum.
-    const int tok = warp;
-    if (kM16 || tok < 8) {
-      const int rp = lane >> 3, q = lane & 7;
-      const int src_lane = (tok & 7) * 4 + rp, h = tok >> 3;
+    if (tid < NP * NT * 128) {
+      float y = 0.0f;
 #pragma unroll
-      for (int j = 0; j < kGvPass; ++j) {
-        if (j < np) {
-          float y0 = 0.0f, y1 = 0.0f;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float2 v = *reinterpret_cast<const float2*>(red + (2 * q + e) * kGvRedWarpBytes +
-                                                              (j * 32 + src_lane) * 16 + 8 * h);
-            y0 += v.x;
-            y1 += v.y;
-          }
-          const int64_t n = static_cast<int64_t>(tile0 + j) * kGvRows + 2 * rp;
-          if (single) {
-            float l0 = 0.0f, l1 = 0.0f;
-            const int64_t r0 = b_smem ? (n - static_cast<int64_t>(t0) * kGvRows) : n;
-            const uint16_t* bsrc = b_smem ? s_b : p.B;
-            for (int jj = q; jj < p.r; jj += 8) {
-              const float uj = s_u[tok * kRankPad + jj];
-              l0 = fmaf(uj, bf16_bits_to_float(bsrc[r0 * p.ldb + jj]), l0);
-              l1 = fmaf(uj, bf16_bits_to_float(bsrc[(r0 + 1) * p.ldb + jj]), l1);
-            }
-            y0 = fmaf(p.scale, l0, y0);
-            y1 = fmaf(p.scale, l1, y1);
-          }
-#pragma unroll
-          for (int o = 1; o < 8; o <<= 1) {
-            y0 += __shfl_xor_sync(0xffffffffu, y0, o);
-            y1 += __shfl_xor_sync(0xffffffffu, y1, o);
-          }
-          if (q == 0 && tok < p.M) {
-            if (single)
-              *reinterpret_cast<uint32_t*>(p.Y + static_cast<int64_t>(tok) * N + n) = pack_bf16x2(y0, y1);
-            else
-              *reinterpret_cast<float2*>(p.ypart + (static_cast<int64_t>(c) * kGemvMaxM + tok) * N + n) =
-                  make_float2(y0, y1);
-          }
+      for (int w = 0; w < kGvWarps; ++w) y += red[w * (kGvRedWarpBytes / 4) + tid];
+      const int comp = tid & 3, ls = (tid >> 2) & 31, rest = tid >> 7;
+      const int nt = rest % NT, j = rest / NT;
+      const int row = (ls >> 2) + 8 * (comp >> 1);
+      const int tok = 2 * (ls & 3) + (comp & 1) + 8 * nt;
+      const int64_t n = static_cast<int64_t>(tile0 + j) * kGvRows + row;
+      if (tok < p.M && n < N) {
+        if (single) {
+          float l = 0.0f;
+          const uint16_t* brow = b_smem ? s_b + (n - row_lo) * p.ldb : p.B + n * p.ldb;
+          for (int jj = 0; jj < p.r; ++jj) l = fmaf(s_u[tok * kRankPad + jj], bf16_bits_to_float(brow[jj]), l);
+          y = fmaf(p.scale, l, y);
+          p.Y[static_cast<int64_t>(tok) * N + n] = static_cast<uint16_t>(pack_bf16x2(y, 0.0f) & 0xFFFFu);
+        } else {
+          p.ypart[(static_cast<int64_t>(c) * kGemvMaxM + tok) * N + n] = y;
         }
       }
     }
     __syncthreads();  // the reduction buffer is free again
 #pragma unroll 1
-    for (int j = 0; j < np; ++j) cc.next(t0, t1);
+    for (int j = 0; j < NP; ++j) cc.next(t0, t1);
+  };
+
+  for (int i0 = 0; i0 < items;) {
+    const int np = (t1 - cc.tile) < P ? (t1 - cc.tile) : P;
+    if (cc.c != x_chunk) {
+      const int64_t blkw = static_cast<int64_t>(cc.c) * kGvUnitBlocks + kGvWarpBlocks * warp;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int b = 0; b < kGvWarpBlocks; ++b) {
+          const int tok = g + 8 * nt;
+          load16(p.X, K, tok, (blkw + b) * kBlock + 16 * t, blkw + b < nbk && tok < p.M, xf[nt][b]);
+        }
+      x_chunk = cc.c;
+    }
+    if (np == P) {
+      run_pass(std::integral_constant<int, P>{});
+    } else if constexpr (P == 4) {
+      if (np == 3) run_pass(std::integral_constant<int, 3>{});
+      else if (np == 2) run_pass(std::integral_constant<int, 2>{});
+      else run_pass(std::integral_constant<int, 1>{});
+    } else {
+      run_pass(std::integral_constant<int, 1>{});
+    }
     i0 += np;
   }
   cp_async_wait<0>();
@@ -498,7 +509,7 @@ cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  const int64_t tiles = p.N / kGvRows;
+  const int64_t tiles = (p.N + kGvRows - 1) / kGvRows;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms));
   cfg.blockDim = dim3(kGvThreads);

@@ -14,9 +14,9 @@
 //                   absmax by three xor-shuffles, IEEE fp32 division by the
 //                   absmax (by 1 for an all-zero block; a reciprocal multiply
 //                   with an exact-division fallback next to a threshold),
-//                   nearest level from a
-//                   129-cell decision table, eight codes packed into one
-//                   32-bit word (even element in the low nibble).
+//                   nearest level from a 129-cell decision table (one 16-byte
+//                   lookup per weight), eight codes packed into one 32-bit
+//                   word (even element in the low nibble).
 //  chunk_sums       one warp per chunk: the fp64 sum of its 256 block scales;
 //                   the last warp of each tensor forms the tensor's mean offset.
 //  dq_chunks        one warp per chunk: d = a - mu, c2 = max|d|,
@@ -64,16 +64,18 @@ __device__ __forceinline__ bool fp64_sum_is_exact(int emin, int emax, int64_t n)
   return (emax - emin) + 24 + ceil_log2(n) <= 53;
 }
 
-__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
 
-__device__ __forceinline__ float2 ld_shared_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
+// Hardware reciprocal (at most 1 ulp from 1/x for a normal x whose
+// reciprocal is normal).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 __device__ __forceinline__ double warp_sum_f64(double v) {
@@ -85,10 +87,12 @@ __device__ __forceinline__ double warp_sum_f64(double v) {
 constexpr int kQWarps = 16;  // 64 groups of 8 lanes
 constexpr int kQThreads = kQWarps * 32;
 
-struct QuantSmem {
-  uint32_t cell_base[129][32];  // per-cell base code, one copy per lane (conflict-free)
-  float2 thr[17];               // (64 T_j, tolerance) for j = 1..15; 256 beyond the last
-};
+// Per decision cell, one 16-byte entry per lane (conflict-free): the band
+// [lo, hi] = 64 T (1 -+ 2^-19) around the cell's threshold T, 64 T itself and
+// the cell's base code; lo = hi = thr = 256 (never reached) in a cell without
+// a threshold.
+constexpr int kCellEntries = 129 * 32;
+constexpr int kQuantSmemBytes = kCellEntries * 16;
 
 __device__ __forceinline__ void chunk_bounds(const QuantBatchParams& p, int64_t g, int& t, int64_t& blk0, int& nblk) {
   t = find_tensor(p, g);
@@ -121,15 +125,15 @@ __device__ __forceinline__ void load_chunk(const QuantBatchParams& p, int64_t g,
 // blocks = 16384 weights) of the batch.  Every lane streams its share of the
 // next chunk into registers (256-bit loads) while it codes the current one.
 // Each group of 8 lanes owns a block: absmax by three xor-shuffles, then per
-// weight x' = w * (64 / a) with a correctly rounded reciprocal.  x' is
-// within 2^-22 |x| of the correctly rounded 64 * fp32(w / a), so it picks the
-// same code unless it lies within the stored tolerance (2^-19 relative) of
-// the cell's threshold; the lane's block is then recoded from the IEEE
-// quotient (so are blocks whose 64/a is not a normal fp32).  Every threshold
-// is > 2^-14 (relative) from its cell's edges (checked on the host), so no
-// other threshold can be that close.
+// weight x' = w * (64 / a) with the hardware reciprocal.  x' is within
+// 2^-21 |x| of the correctly rounded 64 * fp32(w / a), so it lies on the same
+// side of the cell's threshold unless it falls inside the cell's band
+// (2^-19 relative around the threshold); a lane with such a weight recodes
+// its 8 weights from the IEEE quotient (so does a block whose 64/a is not a
+// normal fp32).  Every threshold is > 2^-14 (relative) from its cell's edges
+// (checked on the host), so no other threshold can be that close.
 __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __grid_constant__ QuantBatchParams p) {
-  __shared__ QuantSmem S;
+  extern __shared__ uint4 s_cell[];  // [129 cells][32 lanes]
   const int tid = threadIdx.x, lane = tid & 31;
   const int grp = tid >> 3;  // 64 groups of 8 lanes
   const int l = tid & 7;     // lane in group: weights 8l .. 8l+7 of the block
@@ -137,17 +141,22 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
   float cur[4][8], nxt[4][8];
   load_chunk(p, blockIdx.x, grp, l, cur);
 
-  for (int i = tid; i < 129 * 32; i += kQThreads) S.cell_base[i >> 5][i & 31] = static_cast<uint32_t>(p.table.base[i >> 5]);
-  if (tid < 17) S.thr[tid] = make_float2(256.0f, 0.0f);
-  __syncthreads();
-  if (tid < 129 && p.table.thr[tid] < 2.0f) {
-    const float t64 = p.table.thr[tid] * 64.0f;
-    S.thr[p.table.base[tid] + 1] = make_float2(t64, fabsf(t64) * 0x1p-19f);
+  for (int i = tid; i < kCellEntries; i += kQThreads) {
+    const int c = i >> 5;
+    const float thr = p.table.thr[c];
+    float t64 = 256.0f, lo = 256.0f, hi = 256.0f;
+    if (thr < 2.0f) {
+      t64 = thr * 64.0f;
+      const float tol = fabsf(t64) * 0x1p-19f;
+      lo = t64 - tol;
+      hi = t64 + tol;
+    }
+    s_cell[i] = make_uint4(__float_as_uint(lo), __float_as_uint(hi), __float_as_uint(t64),
+                           static_cast<uint32_t>(p.table.base[c]));
   }
   __syncthreads();
 
-  const uint32_t cell_addr0 = smem_u32(&S.cell_base[64][lane]);  // cell 64 <-> x64 in (-1, 1)
-  const uint32_t thr_addr1 = smem_u32(&S.thr[1]);
+  const uint32_t cell_addr0 = smem_u32(&s_cell[64 * 32 + lane]);  // cell 64 <-> x64 in (-1, 1)
   float nonfinite = 0.0f;  // becomes NaN if any input is NaN or +-Inf
   for (int64_t g = blockIdx.x; g < p.total_chunks; g += gridDim.x) {
     load_chunk(p, g + gridDim.x, grp, l, nxt);
@@ -170,27 +179,27 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
       const float div = (m == 0.0f) ? 1.0f : m;  // zero-block convention
       uint32_t word = 0;
-      float slack = -1.0f;  // > 0 once some weight came within tolerance of a threshold
+      bool risky = false;  // some weight fell inside its cell's band
       const bool fast = div >= 0x1p-121f && div <= 0x1p119f;  // 64 / div is a normal fp32
-      const float rcp64 = fast ? __frcp_rn(div) * 64.0f : 0.0f;
+      const float rcp64 = fast ? rcp_approx(div) * 64.0f : 0.0f;
 #pragma unroll
       for (int i = 7; i >= 0; --i) {
-        const float x64 = v[i] * rcp64;
-        const uint32_t base = ld_shared_u32(cell_addr0 + static_cast<uint32_t>(__float2int_rz(x64)) * 128u);
-        const float2 thr = ld_shared_f2(thr_addr1 + base * 8u);
-        word = word * 16u + base + (x64 >= thr.x ? 1u : 0u);
-        slack = fmaxf(slack, thr.y - fabsf(x64 - thr.x));
+        const float x64 = __fmul_rn(v[i], rcp64);
+        const uint4 e = ld_shared_u4(cell_addr0 + static_cast<uint32_t>(__float2int_rz(x64)) * 512u);
+        const bool above_lo = x64 >= __uint_as_float(e.x);
+        const bool above_hi = x64 > __uint_as_float(e.y);
+        word = word * 16u + e.w + (above_lo ? 1u : 0u);
+        risky |= above_lo != above_hi;
       }
-      if (__any_sync(0xffffffffu, !fast || slack >= 0.0f)) {
-        if (!fast || slack >= 0.0f) {
+      if (__any_sync(0xffffffffu, !fast || risky)) {
+        if (!fast || risky) {
           // Recode this lane's 8 weights from the IEEE quotients.
           word = 0;
 #pragma unroll
           for (int i = 7; i >= 0; --i) {
             const float x64 = __fdiv_rn(v[i], div) * 64.0f;  // exact scaling
-            const uint32_t base = ld_shared_u32(cell_addr0 + static_cast<uint32_t>(__float2int_rz(x64)) * 128u);
-            const float2 thr = ld_shared_f2(thr_addr1 + base * 8u);
-            word = word * 16u + base + (x64 >= thr.x ? 1u : 0u);
+            const uint4 e = ld_shared_u4(cell_addr0 + static_cast<uint32_t>(__float2int_rz(x64)) * 512u);
+            word = word * 16u + e.w + (x64 >= __uint_as_float(e.z) ? 1u : 0u);
           }
         }
       }
@@ -350,9 +359,12 @@ cudaError_t launch_quantize_batch(const QuantBatchParams& p, cudaStream_t stream
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
+    cudaError_t e = cudaFuncSetAttribute(quantize_codes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kQuantSmemBytes);
+    if (e != cudaSuccess) return e;
   }
   const unsigned grid = static_cast<unsigned>(p.total_chunks < sms ? p.total_chunks : sms);
-  quantize_codes_kernel<<<grid, kQThreads, 0, stream>>>(p);
+  quantize_codes_kernel<<<grid, kQThreads, kQuantSmemBytes, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const unsigned warps_grid = static_cast<unsigned>((p.total_chunks + 7) / 8);
