@@ -396,6 +396,29 @@ def run_reference(args, rank, world):
     }))
 
 
+GEMM_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "gemm_tn_layer_step_traffic.md")
+GEMM_SOURCES = ("csrc/gemm_tc.cu", "csrc/common.cuh", "csrc/kernels.cuh")
+
+
+def gemm_traffic_per_launch():
+    """DRAM bytes per gemm_tn launch from the committed ncu summary, or None
+    when the kernel's sources changed since that capture."""
+    import hashlib
+    try:
+        text = open(GEMM_TRAFFIC_PROFILE).read()
+    except OSError:
+        return None
+    fields = dict(line.split(": ", 1) for line in text.splitlines()
+                  if line.startswith(("traffic_bytes_per_launch: ", "source_digest: ")))
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "bit_nf4_quantized_blk_b200", rel), "rb") as f:
+            h.update(f.read())
+    if fields.get("source_digest", "").strip() != h.hexdigest()[:16]:
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 def run_ours(args, rank, world, local_rank):
     from bit_nf4_quantized_blk_b200 import build
 
@@ -441,7 +464,8 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "gemm_tn_kernel (tcgen05 128x256 tile)",
                      "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tflops / peak,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": gemm_traffic_per_launch(),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "share_of_step": gemm_ms_per_step / ms},
         "gpu_launches": int(round(launches_total / steps_recorded * args.steps)),
         "kernel_ms_per_step": {f: v[0] / steps_recorded for f, v in fam.items()},

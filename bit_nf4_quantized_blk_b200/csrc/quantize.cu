@@ -101,12 +101,32 @@ __device__ __forceinline__ void chunk_bounds(const QuantBatchParams& p, int64_t 
   nblk = static_cast<int>(rem < kDqBlock ? rem : int64_t{kDqBlock});
 }
 
-// Weights 8l .. 8l+7 of blocks grp, grp + 64, grp + 128, grp + 192 of chunk
-// g (zeros past the tensor or the batch), with 256-bit streaming loads.
-__device__ __forceinline__ void load_chunk(const QuantBatchParams& p, int64_t g, int grp, int l, float (&v)[4][8]) {
-  int t = 0, nblk = 0;
-  int64_t blk0 = 0;
-  if (g < p.total_chunks) chunk_bounds(p, g, t, blk0, nblk);
+// Tensor, first block and block count of chunk g (nblk = 0 past the batch).
+// A CTA visits its chunks in increasing order, so the tensor index only moves
+// forward from the previous chunk's.
+struct ChunkInfo {
+  int t, nblk;
+  int64_t blk0;
+};
+
+__device__ __forceinline__ ChunkInfo next_chunk_info(const QuantBatchParams& p, int64_t g, int& t_cursor) {
+  ChunkInfo ci{t_cursor, 0, 0};
+  if (g < p.total_chunks) {
+    while (t_cursor + 1 < p.count && p.chunk_begin[t_cursor + 1] <= g) ++t_cursor;
+    ci.t = t_cursor;
+    ci.blk0 = (g - p.chunk_begin[ci.t]) * kDqBlock;
+    const int64_t rem = p.n_blocks[ci.t] - ci.blk0;
+    ci.nblk = static_cast<int>(rem < kDqBlock ? rem : int64_t{kDqBlock});
+  }
+  return ci;
+}
+
+// Weights 8l .. 8l+7 of blocks grp, grp + 64, grp + 128, grp + 192 of a
+// chunk (zeros past the tensor or the batch), with 256-bit streaming loads.
+__device__ __forceinline__ void load_chunk(const QuantBatchParams& p, const ChunkInfo& ci, int grp, int l,
+                                           float (&v)[4][8]) {
+  const int t = ci.t, nblk = ci.nblk;
+  const int64_t blk0 = ci.blk0;
   const float* src = p.W[t] + (blk0 + grp) * kBlock + l * 8;
 #pragma unroll
   for (int rep = 0; rep < 4; ++rep) {
@@ -139,7 +159,9 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
   const int l = tid & 7;     // lane in group: weights 8l .. 8l+7 of the block
 
   float cur[4][8], nxt[4][8];
-  load_chunk(p, blockIdx.x, grp, l, cur);
+  int t_cursor = 0;
+  ChunkInfo cur_ci = next_chunk_info(p, blockIdx.x, t_cursor);
+  load_chunk(p, cur_ci, grp, l, cur);
 
   for (int i = tid; i < kCellEntries; i += kQThreads) {
     const int c = i >> 5;
@@ -159,10 +181,10 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
   const uint32_t cell_addr0 = smem_u32(&s_cell[64 * 32 + lane]);  // cell 64 <-> x64 in (-1, 1)
   float nonfinite = 0.0f;  // becomes NaN if any input is NaN or +-Inf
   for (int64_t g = blockIdx.x; g < p.total_chunks; g += gridDim.x) {
-    load_chunk(p, g + gridDim.x, grp, l, nxt);
-    int t, nblk;
-    int64_t blk0;
-    chunk_bounds(p, g, t, blk0, nblk);
+    const ChunkInfo nxt_ci = next_chunk_info(p, g + gridDim.x, t_cursor);
+    load_chunk(p, nxt_ci, grp, l, nxt);
+    const int t = cur_ci.t, nblk = cur_ci.nblk;
+    const int64_t blk0 = cur_ci.blk0;
     uint32_t* __restrict__ packed = reinterpret_cast<uint32_t*>(p.packed[t]);
 #pragma unroll
     for (int rep = 0; rep < kDqBlock / 64; ++rep) {
@@ -212,6 +234,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
     for (int rep = 0; rep < 4; ++rep)
 #pragma unroll
       for (int i = 0; i < 8; ++i) cur[rep][i] = nxt[rep][i];
+    cur_ci = nxt_ci;
   }
   if (!(nonfinite == 0.0f)) raise_status(p.status, QLORA_ERR_NONFINITE);
 }
