@@ -462,7 +462,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD,
                    "flops_per_step_per_gpu": flops, "l2": "inputs larger than L2 (GBs per step)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_tn_kernel (tcgen05 128x256 tile)",
+        "roofline": {"bound": "tensor", "kernel": "gemm_tn2_kernel (tcgen05 pair-CTA 256x256 tile)",
                      "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tflops / peak,
                      "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": gemm_traffic_per_launch(),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",

@@ -9,6 +9,8 @@
 // The rank-r product is one more pipeline step that issues ceil(r/16)
 // K=16 MMAs into the same accumulator.
 //
+// Two kernels: the pair-CTA kernel below (256 x 256 tiles on CTA pairs, used
+// whenever pair clusters can be scheduled) and this one-CTA kernel.
 // Persistent CTAs (one per SM) compute 128 x 256 tiles with a 4-stage TMA ring:
 //   warp 0      TMA producer (one elected thread), 128B-swizzled tiles
 //   warp 1      TMEM allocation + MMA issue (one thread): tcgen05.mma
@@ -282,6 +284,324 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Pair-CTA variant: a cluster of 2 CTAs computes 256 x 256 tiles with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16).  Each CTA loads its
+// 128 rows of A and its 128 rows (N) of B per stage (32 KB instead of 48 KB,
+// six stages), so the pair reads half of B per CTA and the shared-memory
+// operand traffic per FLOP drops by a third.
+//   warp 0      TMA producer of this CTA's halves; the transaction bytes of
+//               both CTAs complete on the even CTA's stage barrier, which
+//               the even CTA's producer arms with the pair's total
+//   warp 1      TMEM allocation (both CTAs); in the even CTA, MMA issue
+//   warps 2-5   epilogue of this CTA's 128 accumulator rows
+// The MMA's commits reach both CTAs (multicast commit); the epilogue warps of
+// both CTAs hand the accumulator back to the even CTA by remote arrive.
+// ---------------------------------------------------------------------------
+
+namespace {
+constexpr int BM2 = 128;                 // rows of A per CTA (256 per pair)
+constexpr int BN2 = 256;                 // N per tile; each CTA loads 128 rows of B
+constexpr int BNH = BN2 / 2;
+constexpr int STAGES2 = 6;
+constexpr int A_TILE2 = BM2 * BK * 2;    // 16 KB
+constexpr int B_TILE2 = BNH * BK * 2;    // 16 KB
+constexpr size_t kL2PanelBudget = size_t(48) << 20;  // bytes of operand panels kept resident per group
+constexpr int SMEM2_BYTES = 1024 + STAGES2 * (A_TILE2 + B_TILE2) + 512;
+}  // namespace
+
+// Tile order of the pair kernel: groups of `group` consecutive tiles along M
+// (along_n = 0) or N (along_n = 1) sweep the other dimension, so the panels of
+// one group stay in L2 while the other operand streams past once per group.
+__device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles, int group, int along_n, int& mb,
+                                                 int& nb) {
+  const int g_tiles = along_n ? n_tiles : m_tiles, o_tiles = along_n ? m_tiles : n_tiles;
+  const int per_group = group * o_tiles;
+  const int gi = t / per_group, first = gi * group;
+  const int gsize = min(group, g_tiles - first), local = t - gi * per_group;
+  const int gpos = first + local % gsize, opos = local / gsize;
+  mb = along_n ? opos : gpos;
+  nb = along_n ? gpos : opos;
+}
+
+template <bool kBMN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tn2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, int M, int N,
+                    int num_k, int r_steps, uint16_t* __restrict__ D, int accumulate, int* status, int group,
+                    int along_n) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES2 * A_TILE2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES2 * B_TILE2);
+  uint64_t* empty = full + STAGES2;
+  uint64_t* acc_full = empty + STAGES2;    // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2], even CTA
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t rank = cluster_ctarank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (M + 2 * BM2 - 1) / (2 * BM2), n_tiles = (N + BN2 - 1) / BN2;
+  const int total_tiles = m_tiles * n_tiles;
+  const int pair = static_cast<int>(cluster_id_x()), npairs = static_cast<int>(num_clusters_x());
+  const int k_iters = num_k + (r_steps > 0 ? 1 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);  // 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      if (r_steps > 0) {
+        tma_prefetch_desc(&tmA2);
+        tma_prefetch_desc(&tmB2);
+      }
+      // Stage barriers of the even CTA, in the cluster address space.
+      const uint32_t full0 = map_to_cta(&full[0], 0);
+      int it = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += npairs) {
+        int mb, nb;
+        pair_tile_coords(t, m_tiles, n_tiles, group, along_n, mb, nb);
+        const int m0 = mb * 2 * BM2 + static_cast<int>(rank) * BM2;
+        const int n0 = nb * BN2 + static_cast<int>(rank) * BNH;
+        for (int i = 0; i < k_iters; ++i, ++it) {
+          const int s = it % STAGES2, u = it / STAGES2;
+          if (it >= STAGES2 && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
+          if constexpr (!kBMN) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (A_TILE2 + B_TILE2));
+            if (i < num_k) {
+              tma_load_2d_pair(sA + s * A_TILE2, &tmA, fb, i * BK, m0);
+              tma_load_2d_pair(sB + s * B_TILE2, &tmB, fb, i * BK, n0);
+            } else {
+              tma_load_2d_pair(sA + s * A_TILE2, &tmA2, fb, 0, m0);
+              tma_load_2d_pair(sB + s * B_TILE2, &tmB2, fb, 0, n0);
+            }
+          } else {
+            if (i < num_k) {
+              if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (A_TILE2 + B_TILE2));
+              tma_load_2d_pair(sA + s * A_TILE2, &tmA, fb, i * BK, m0);
+              for (int j = 0; j < BNH / 64; ++j)
+                tma_load_2d_pair(sB + s * B_TILE2 + j * 8192, &tmB, fb, n0 + 64 * j, i * BK);
+            } else {
+              if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (A_TILE2 + (BNH / 64) * r_steps * 16 * 128));
+              tma_load_2d_pair(sA + s * A_TILE2, &tmA2, fb, 0, m0);
+              for (int j = 0; j < BNH / 64; ++j)
+                tma_load_2d_pair(sB + s * B_TILE2 + j * 8192, &tmB2, fb, n0 + 64 * j, 0);
+            }
+          }
+        }
+      }
+      // Teardown: the copies into this CTA's shared memory must have landed
+      // before it goes.  The even CTA waits on its stage barriers (they count
+      // both CTAs' bytes).  The odd CTA cannot wait on them; on the normal path
+      // the even CTA consumed every stage before the final handshake, and
+      // after an abort the odd CTA gives its copies in flight 100 us.
+      if (rank == 0) {
+        for (int i = (it > STAGES2 ? it - STAGES2 : 0); i < it; ++i)
+          mbar_wait_teardown(&full[i % STAGES2], (i / STAGES2) & 1, status);
+      } else if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 100000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * BM2, BN2, kBMN);
+      int it = 0, tl = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += npairs, ++tl) {
+        const int buf = tl & 1, use = tl >> 1;
+        if (use > 0 && !mbar_wait_cluster(&acc_empty[buf], (use - 1) & 1, abort_flag, status)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN2);
+        for (int i = 0; i < k_iters; ++i, ++it) {
+          const int s = it % STAGES2, u = it / STAGES2;
+          if (!mbar_wait_cluster(&full[s], u & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nsteps = i < num_k ? BK / 16 : r_steps;
+          const uint64_t adesc = smem_desc_k128(smem_u32(sA + s * A_TILE2));
+          const uint64_t bdesc = kBMN ? smem_desc_mn128(smem_u32(sB + s * B_TILE2), 8192, 1024)
+                                      : smem_desc_k128(smem_u32(sB + s * B_TILE2));
+          const uint32_t bstep = kBMN ? (2048 >> 4) : 2;
+          for (int kk = 0; kk < nsteps; ++kk)
+            tc_mma_bf16_ss_pair(acc, adesc + 2 * kk, bdesc + bstep * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_commit_pair(&empty[s], 0x3);
+        }
+        if (ok) tc_commit_pair(&acc_full[buf], 0x3);
+      }
+      // Every MMA (which also reads the odd CTA's shared memory) must be
+      // complete before the pair's tensor memory and shared memory go.
+      tc_commit_pair(drain, 0x1);
+      mbar_wait_teardown(drain, 0, status);
+    }
+  } else {
+    // Epilogue warps 2..5 own TMEM lane quadrants (warp % 4).
+    const int q = warp & 3;
+    const uint32_t acc_empty0 = map_to_cta(&acc_empty[0], 0);
+    int tl = 0;
+    for (int t = pair; t < total_tiles; t += npairs, ++tl) {
+      const int buf = tl & 1, use = tl >> 1;
+      const bool ok =
+          __all_sync(0xffffffffu, mbar_wait_cluster(&acc_full[buf], use & 1, abort_flag, status) ? 1 : 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      int mb, nb;
+      pair_tile_coords(t, m_tiles, n_tiles, group, along_n, mb, nb);
+      const int row = mb * 2 * BM2 + static_cast<int>(rank) * BM2 + q * 32 + lane;
+      const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN2) + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c = 0; c < BN2 / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(acc + c * 32, v);
+        tmem_wait_ld();
+        const int col = nb * BN2 + c * 32;
+        if (row >= M || col >= N) continue;
+        uint16_t* dst = D + static_cast<int64_t>(row) * N + col;
+        if (col + 32 <= N) {
+          uint32_t pk[16];
+          if (accumulate) {
+            const uint4* old = reinterpret_cast<const uint4*>(dst);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const uint4 o = old[q4];
+              const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int idx = q4 * 8 + e * 2;
+                pk[q4 * 4 + e] = pack_bf16x2(__uint_as_float(v[idx]) + bf16_bits_to_float(ow[e] & 0xFFFF),
+                                             __uint_as_float(v[idx + 1]) + bf16_bits_to_float(ow[e] >> 16));
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (col + e < N) {
+              float val = __uint_as_float(v[e]);
+              if (accumulate) val += bf16_bits_to_float(dst[e]);
+              dst[e] = static_cast<uint16_t>(pack_bf16x2(val, 0.0f) & 0xFFFF);
+            }
+          }
+        }
+      }
+      // Hand the accumulator buffer back to the even CTA's MMA thread.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * static_cast<uint32_t>(buf));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the pair's MMAs are complete; no remote signal is in flight
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+namespace {
+
+// Pair clusters that can be resident at once (0: the pair kernel cannot run).
+template <bool kBMN>
+int max_pair_clusters() {
+  static int cached = -1;
+  if (cached >= 0) return cached;
+  cached = 0;
+  if (cudaFuncSetAttribute(gemm_tn2_kernel<kBMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES) !=
+      cudaSuccess)
+    return cached;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = SMEM2_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tn2_kernel<kBMN>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cached = n;
+  return cached;
+}
+
+template <bool kBMN>
+cudaError_t launch_pair(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tA2, const CUtensorMap& tB2,
+                        const GemmArgs& a, int num_k, int r_steps, int clusters, cudaStream_t stream) {
+  const int64_t m_tiles = (a.M + 2 * BM2 - 1) / (2 * BM2), n_tiles = (a.N + BN2 - 1) / BN2;
+  const int64_t tiles = m_tiles * n_tiles;
+  const int pairs = static_cast<int>(tiles < clusters ? tiles : clusters);
+  // A 256-wide panel of either operand holds 256 x K bf16.  Group as many
+  // panels as the L2 budget keeps resident, along the dimension that makes
+  // the other operand's re-reads fewest: traffic ~ own + other * ceil(own / group).
+  const size_t panel = size_t(256) * static_cast<size_t>(a.K) * 2;
+  const int64_t fit = static_cast<int64_t>(kL2PanelBudget / panel) > 1 ? static_cast<int64_t>(kL2PanelBudget / panel) : 1;
+  const int64_t gm = fit < m_tiles ? fit : m_tiles, gn = fit < n_tiles ? fit : n_tiles;
+  const int64_t traffic_m = m_tiles + n_tiles * ((m_tiles + gm - 1) / gm);
+  const int64_t traffic_n = n_tiles + m_tiles * ((n_tiles + gn - 1) / gn);
+  const int along_n = traffic_n < traffic_m ? 1 : 0;
+  const int group = static_cast<int>(along_n ? gn : gm);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = SMEM2_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_tn2_kernel<kBMN>, tA, tB, tA2, tB2, static_cast<int>(a.M), static_cast<int>(a.N),
+                            num_k, r_steps, a.D, a.accumulate, a.status, group, along_n);
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
@@ -291,12 +611,16 @@ cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
+  const int clusters = a.b_mn_major ? max_pair_clusters<true>() : max_pair_clusters<false>();
+  const bool pair = clusters > 0;
+  // B (and B2) boxes: the pair kernel loads 128 rows of N per CTA.
+  const uint32_t bn_box = pair ? static_cast<uint32_t>(BNH) : static_cast<uint32_t>(BN);
   CUtensorMap tA, tB, tA2, tB2;
   if (!encode_tensor_map_2d(&tA, a.A, a.M, a.K, BM, BK)) return cudaErrorInvalidValue;
   if (a.b_mn_major) {
     if (!encode_tensor_map_2d(&tB, a.B, a.K, a.N, BK, 64)) return cudaErrorInvalidValue;  // B stored [K][N]
   } else {
-    if (!encode_tensor_map_2d(&tB, a.B, a.N, a.K, BN, BK, true, a.ldb)) return cudaErrorInvalidValue;
+    if (!encode_tensor_map_2d(&tB, a.B, a.N, a.K, bn_box, BK, true, a.ldb)) return cudaErrorInvalidValue;
   }
   int r_steps = 0;
   if (a.A2 != nullptr && a.r > 0) {
@@ -308,13 +632,17 @@ cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     } else {
       // B2 stored [N][ldb2] with r valid columns (zero filled up to 64)
-      if (!encode_tensor_map_2d(&tB2, a.B2, a.N, a.r, BN, BK, true, a.ldb2)) return cudaErrorInvalidValue;
+      if (!encode_tensor_map_2d(&tB2, a.B2, a.N, a.r, bn_box, BK, true, a.ldb2)) return cudaErrorInvalidValue;
     }
   } else {
     tA2 = tA;
     tB2 = tB;
   }
   const int num_k = static_cast<int>((a.K + BK - 1) / BK);
+  if (pair) {
+    return a.b_mn_major ? launch_pair<true>(tA, tB, tA2, tB2, a, num_k, r_steps, clusters, stream)
+                        : launch_pair<false>(tA, tB, tA2, tB2, a, num_k, r_steps, clusters, stream);
+  }
   static int sms = 0;
   if (sms == 0) {
     int dev = 0;
