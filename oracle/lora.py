@@ -73,3 +73,19 @@ def lora_adapter_grads(X, dY, A, B, s: float):
     dA = s * ((dY @ B).T @ X)
     dB = s * (dY.T @ (X @ A.T))
     return dA, dB
+
+
+def merge(W_hat, A, B, s: float) -> np.ndarray:
+    """The merged weight ``W_hat + s B A`` in fp64.
+
+    "FT-02: QLoRA -- Fine-Tuning with Quantization", section "4. The LoRA
+    mechanics the API wraps" (the merge proof: one dense layer with weight
+    ``W0 + (alpha/r) B A`` computes the two-branch output); "QLoRA: NF4
+    storage, gradients and local integration", section "Merge changes the
+    operator: test it explicitly" (merging into the dequantized ``Qhat(W)``
+    matches the unmerged quantized layer in exact arithmetic; requantizing
+    the result adds ``Qhat(M) - M``).  ``W_hat`` here is the fp32 dequantized
+    weight (before any bf16 rounding).
+    """
+    W_hat, A, B = _f64(W_hat), _f64(A), _f64(B)
+    return W_hat + F64(s) * (B @ A)

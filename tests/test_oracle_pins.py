@@ -367,6 +367,39 @@ def test_merge_identity():
     assert np.max(np.abs(Y - merged)) <= 1e-12 * np.max(np.abs(Y))
 
 
+def test_merge_reproduces_the_two_branch_layer():
+    """X merge(W, A, B, s)^T equals the unmerged forward (exact arithmetic)."""
+    X, W, A, B, _, s = _small_lora(11)
+    Y, _ = lora.lora_forward(X, W, A, B, s)
+    assert np.max(np.abs(X @ lora.merge(W, A, B, s).T - Y)) <= 1e-12 * np.max(np.abs(Y))
+
+
+def test_merge_special_cases():
+    X, W, A, B, _, s = _small_lora(12, n=12, k=10, r=3)
+    assert np.array_equal(lora.merge(W, A, np.zeros_like(B), s), W)  # B = 0: the base weight
+    delta = lora.merge(W, A, B, s) - W
+    assert np.linalg.matrix_rank(delta) <= 3  # the update lives in an r-dimensional space
+
+
+def test_requantizing_a_dequantized_weight_keeps_its_codes():
+    """Qhat(Qhat(W)) has Qhat(W)'s codes: every block's largest |value| is
+    the decoded scale times a +-1 level, so renormalising returns each level
+    to within an ulp, far from any decision threshold."""
+    rng = np.random.default_rng(13)
+    W = (rng.standard_normal((64, 256)) * 0.02).astype(np.float32)
+    st = nf4.quantize_weight(W)
+    W_hat = nf4.dequantize_weight(st, "fp32")
+    st2 = nf4.quantize_weight(np.asarray(W_hat, dtype=np.float32))
+    assert np.array_equal(st2.packed, st.packed)
+    # ... while the merged-then-requantized weight moves: Qhat(M) - M != 0.
+    A = rng.standard_normal((4, 256)) * 0.02
+    B = rng.standard_normal((64, 4)) * 0.02
+    M = lora.merge(W_hat, A, B, 2.0).astype(np.float32)
+    back = nf4.dequantize_weight(nf4.quantize_weight(M), "fp32")
+    err = np.linalg.norm(back - M) / np.linalg.norm(M)
+    assert 1e-3 < err < 0.2
+
+
 def test_gradients_match_autograd():
     X, W, A, B, G, s = _small_lora(2)
     tX, tA, tB = (torch.tensor(a, requires_grad=True) for a in (X, A, B))
