@@ -243,7 +243,7 @@ def timed(fn, steps, warmup, world, window=None):
 
 
 # ---------------------------------------------------------------------------
-# Secondary measurements (rank 0): quantize / dequant / GEMV rows
+# Secondary measurements (rank 0): quantize / dequant / GEMV / merge rows
 # ---------------------------------------------------------------------------
 
 def l2_flush_buffer():
@@ -304,6 +304,31 @@ def bench_gemv(reps=50):
         res[f"M={M}"] = {"us": ms * 1e3, "GB/s": nbytes / ms / 1e6, "bytes": nbytes}
         assert binding.qlora_workspace_status(ws) == 0
     return res
+
+
+def bench_merge(reps=10):
+    """Merged bf16 weights W_hat + s B A of the 7B layer's seven projections
+    (r = 16): one qlora_merge per projection, the seven timed together."""
+    cases = [workloads.linear_case(p, 1, 16, 32.0, 4, 0, t, "cuda", with_dy=False)
+             for t, p in enumerate(workloads.LAYER7B)]
+    outs = [binding.NF4Weight.empty(c.proj.n, c.proj.k) for c in cases]
+    ws = torch.empty(binding.qlora_nf4_quantize_batched_ws_bytes(outs), dtype=torch.uint8, device="cuda")
+    dstat = torch.zeros(1, dtype=torch.int32, device="cuda")
+    binding.qlora_nf4_quantize_batched([c.W for c in cases], outs, ws, d_status=dstat)
+    for c in cases:
+        c.W = None
+    ys = [torch.empty((c.proj.n, c.proj.k), dtype=torch.bfloat16, device="cuda") for c in cases]
+
+    def run():
+        for c, o, y in zip(cases, outs, ys):
+            binding.qlora_merge(o, c.A, c.B, c.r, c.s, y, 0)
+
+    ms = timed(run, reps, 2, 1)
+    assert dstat.item() == 0
+    n = sum(c.proj.n * c.proj.k for c in cases)
+    nbytes = (n * (0.5 + 1 / 64 + 2) + 4 * sum(o.c2.numel() + 1 for o in outs)
+              + 2 * sum(c.A.numel() + c.B.numel() for c in cases))
+    return {"weights": n, "ms": ms, "GB/s": nbytes / ms / 1e6, "bytes": nbytes, "out": "bf16"}
 
 
 # ---------------------------------------------------------------------------
@@ -478,8 +503,9 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         extras = bench_quantize_dequant()
         extras["gemv_gate_14336x4096"] = bench_gemv()
+        extras["merge_layer7b_r16"] = bench_merge()
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        for k in ("quantize", "dequant_bf16"):
+        for k in ("quantize", "dequant_bf16", "merge_layer7b_r16"):
             extras[k]["frac_hbm"] = extras[k]["GB/s"] / hbm
         for k, v in extras["gemv_gate_14336x4096"].items():
             v["frac_hbm"] = v["GB/s"] / hbm

@@ -39,6 +39,7 @@ EXPORTED = [
     "qlora_nf4_quantize_noalloc",
     "qlora_nf4_dequantize",
     "qlora_nf4_dequantize_batched",
+    "qlora_merge",
     "qlora_workspace_reset",
     "qlora_workspace_status",
     "qlora_linear_ws_bytes",
@@ -92,6 +93,7 @@ def lib() -> ctypes.CDLL:
         "qlora_nf4_quantize_noalloc": (i32, [P, W, P, P]),
         "qlora_nf4_dequantize": (i32, [W, P, i32, i32, P]),
         "qlora_nf4_dequantize_batched": (i32, [W, ctypes.POINTER(P), i32, i32, P]),
+        "qlora_merge": (i32, [W, P, P, i32, f32, P, i32, P]),
         "qlora_workspace_reset": (i32, [P, sz, P]),
         "qlora_workspace_status": (i32, [P, sz, P]),
         "qlora_linear_ws_bytes": (sz, [i64, i64, i64, i32]),
@@ -207,6 +209,13 @@ def qlora_nf4_dequantize_batched(weights, outs, out_dtype: int = 0, stream=None)
     ptrs = (ctypes.c_void_p * len(outs))(*[o.data_ptr() for o in outs])
     _check("qlora_nf4_dequantize_batched",
            lib().qlora_nf4_dequantize_batched(arr, ptrs, len(weights), out_dtype, _stream(stream)))
+
+
+def qlora_merge(w: NF4Weight, A, B, r: int, scale: float, out, out_dtype: int = 0, stream=None) -> None:
+    st = w.c_struct()
+    _check("qlora_merge",
+           lib().qlora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(scale), out.data_ptr(),
+                             out_dtype, _stream(stream)))
 
 
 def qlora_workspace_reset(ws: torch.Tensor, stream=None) -> None:

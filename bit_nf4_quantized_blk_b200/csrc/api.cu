@@ -127,8 +127,8 @@ const Nf4DecisionTable* decision_table() {
 // Kernel timing (instrumentation): CUDA events around each launch family.
 // ---------------------------------------------------------------------------
 
-enum Family { kFamQuant, kFamDequant, kFamGemv, kFamSide, kFamGemm, kFamCount };
-const char* const kFamNames[kFamCount] = {"quantize", "dequant", "gemv", "side", "gemm"};
+enum Family { kFamQuant, kFamDequant, kFamGemv, kFamSide, kFamGemm, kFamMerge, kFamCount };
+const char* const kFamNames[kFamCount] = {"quantize", "dequant", "gemv", "side", "gemm", "merge"};
 
 struct TimingState {
   bool enabled = false;
@@ -473,6 +473,20 @@ extern "C" qlora_status qlora_nf4_dequantize(const qlora_nf4_weight* w, void* ou
   if (st != QLORA_OK) return st;
   Timed tm(kFamDequant, static_cast<cudaStream_t>(stream));
   return from_cuda(launch_dequant_transposed(view_of(w), static_cast<uint16_t*>(out), static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int32_t r,
+                                    float scale, void* out, int32_t out_dtype, void* stream) {
+  qlora_status st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  if (A == nullptr || B == nullptr || out == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (r < 1 || r > kMaxRank || (out_dtype != 0 && out_dtype != 1) || !std::isfinite(scale))
+    return QLORA_ERR_INVALID_ARG;
+  if (!aligned(A, 2) || !aligned(B, 2) || !aligned(out, 16)) return QLORA_ERR_ALIGNMENT;
+  st = check_device();
+  if (st != QLORA_OK) return st;
+  Timed tm(kFamMerge, static_cast<cudaStream_t>(stream));
+  return from_cuda(launch_merge(view_of(w), A, B, r, scale, out, out_dtype, static_cast<cudaStream_t>(stream)));
 }
 
 extern "C" size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r) {

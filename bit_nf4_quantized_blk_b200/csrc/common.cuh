@@ -461,6 +461,18 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait_prior() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// m16n8k16 bf16 MMA (warp-synchronous legacy tensor path), fp32 accumulate,
+// d += a b.  Fragments (g = lane / 4, t = lane % 4; low half of a register =
+// lower k): a0 (row g, k 2t..2t+1), a1 (row g+8, same k), a2 (row g,
+// k 2t+8..2t+9), a3 (row g+8, same k); b0 (k 2t..2t+1, col g), b1 (k 2t+8..
+// 2t+9, col g); d0, d1 (row g, cols 2t, 2t+1), d2, d3 (row g+8, same cols).
+// Not `volatile`, so loads can be scheduled around it.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // ---------------------------------------------------------------------------
 // The NF4 codebook: the 16 levels of "QLoRA: NF4 storage, gradients and local
 // integration", section "Exact CPU teaching quantizer and adapter gradient

@@ -91,14 +91,6 @@ __device__ __forceinline__ uint32_t lut_pair(uint32_t word, uint32_t lane_base) 
   return v;
 }
 
-// m16n8k16 bf16 MMA, fp32 accumulate, without `volatile` so loads can be
-// scheduled around it.
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
 // 16 consecutive bf16 of row `row` starting at element k (zeros if !valid).
 __device__ __forceinline__ void load16(const uint16_t* base, int64_t ld, int row, int64_t k, bool valid,
                                        uint32_t (&w)[8]) {

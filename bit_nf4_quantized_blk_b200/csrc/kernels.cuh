@@ -63,6 +63,13 @@ cudaError_t launch_dequant_batch(const DequantBatchParams& p, int out_fp32, cuda
 cudaError_t launch_dequant_transposed(const WeightView& w, uint16_t* out, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
+// Merged weight W + s B A (merge.cu)
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_merge(const WeightView& w, const uint16_t* A, const uint16_t* B, int r, float scale, void* out,
+                         int out_fp32, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
 // Decode-shaped dequant-GEMV (gemv.cu), M <= 16
 // ---------------------------------------------------------------------------
 

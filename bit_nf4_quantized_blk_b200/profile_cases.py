@@ -5,7 +5,8 @@ sets up one realistic case (inputs larger than L2, a few hundred MB on the
 device at most), runs the library call ``reps`` times and exits; a profiler
 pointed at it with a kernel filter and a launch count captures the kernel of
 interest.  The cases use the 7B gate projection (14336 x 4096) at 8192
-tokens, or the decode shape (16 tokens) for the GEMV.
+tokens, the decode shape (16 tokens) for the GEMV, and the bf16 merged
+weight (r = 16) for the merge.
 """
 
 from __future__ import annotations
@@ -16,7 +17,7 @@ import torch
 
 from bit_nf4_quantized_blk_b200 import binding, workloads
 
-CASES = ("gemm", "gemm_bwd", "quantize", "dequant", "gemv", "side")
+CASES = ("gemm", "gemm_bwd", "quantize", "dequant", "gemv", "side", "merge")
 
 
 def main():
@@ -26,8 +27,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=8192)
     args = ap.parse_args()
     torch.cuda.set_device(0)
-    M = 16 if args.case == "gemv" else args.tokens
-    case = workloads.linear_case(workloads.GATE7B, M, 16, 32.0, 4, 0, 4, device="cuda", with_dy=args.case != "gemv")
+    M = 16 if args.case in ("gemv", "merge") else args.tokens
+    case = workloads.linear_case(workloads.GATE7B, M, 16, 32.0, 4, 0, 4, device="cuda", with_dy=args.case not in ("gemv", "merge"))
     out = binding.NF4Weight.empty(case.proj.n, case.proj.k)
     qws = torch.empty(binding.qlora_nf4_sizes(case.proj.n, case.proj.k)["ws_bytes"], dtype=torch.uint8, device="cuda")
     binding.qlora_nf4_quantize(case.W, out, qws)
@@ -46,6 +47,9 @@ def main():
         elif args.case == "dequant":
             dense = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
             binding.qlora_nf4_dequantize(out, dense, 0, 0)
+        elif args.case == "merge":
+            merged = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+            binding.qlora_merge(out, case.A, case.B, 16, case.s, merged, 0)
         elif args.case == "side":
             dA = torch.empty((16, K), dtype=torch.float32, device="cuda")
             dB = torch.empty((N, 16), dtype=torch.float32, device="cuda")

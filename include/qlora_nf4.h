@@ -166,6 +166,30 @@ qlora_status qlora_nf4_dequantize_batched(const qlora_nf4_weight *weights, void 
                                           int32_t out_dtype, void *stream);
 
 /*
+ * Merged dense weight of a LoRA-adapted layer:
+ *     out = W + scale * B A          ([rows, cols], W the dequantized weight)
+ * The dense layer that computes the same output as the two-branch forward
+ * (Y = X out^T up to rounding).  Requantizing a merged layer is this call
+ * with out_dtype = 1 followed by qlora_nf4_quantize on `out`.
+ * Source: "FT-02: QLoRA -- Fine-Tuning with Quantization", section "4. The
+ * LoRA mechanics the API wraps" (merge of W0 + (alpha / r) B A);
+ * "QLoRA: NF4 storage, gradients and local integration", section "Merge
+ * changes the operator: test it explicitly" (the merge uses the dequantized
+ * weight; requantizing the merge moves it by Qhat(M) - M).
+ *   w         : quantized weight, rows = N (d_out), cols = K (d_in).
+ *   A         : bf16 [r, K].   B : bf16 [N, r] (both 2-byte aligned).
+ *   r         : 1..64.  scale : s = alpha / r (finite).
+ *   out       : [N, K] output, 16-byte aligned; out_dtype 0 = bf16, 1 = fp32.
+ * Arithmetic: W[n][k] is the fp32 decode (bit-identical to
+ * qlora_nf4_dequantize with out_dtype = 1); sum_j B[n][j] A[j][k] is a
+ * tensor-core product of the bf16 operands with fp32 accumulation;
+ * out = fma(scale, sum, W) in fp32, rounded to nearest-even for bf16.
+ * No workspace.
+ */
+qlora_status qlora_merge(const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                         void *out, int32_t out_dtype, void *stream);
+
+/*
  * Device-side status of a linear-layer workspace.  Kernels record the first
  * device-detected error (QLORA_ERR_TIMEOUT: a barrier wait ran past its one
  * second limit, the kernel gave up and returned) in the first word of the
@@ -223,7 +247,8 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
  * While enabled, every kernel the library enqueues is bracketed by CUDA
  * events recorded on the launching stream, grouped by family:
  *   "quantize" (quantize + double quant), "dequant", "gemv", "side" (rank-r
- *   products, gradient column sums, padding), "gemm" (tensor-core GEMM).
+ *   products, gradient column sums, padding), "gemm" (tensor-core GEMM),
+ *   "merge" (qlora_merge).
  *   qlora_timing_enable : 1 starts recording (clearing earlier records), 0 stops.
  *   qlora_timing_read   : waits for the recorded events of `family` and returns
  *                         the summed device time in milliseconds and the number
