@@ -28,6 +28,22 @@ Each function follows one step of the method as the pages give it:
   cast to the compute dtype.  "QLoRA Deep Dive ...", section "The
   Quantization Process in QLoRA"; "QLoRA: NF4 storage ...", ``dequantize_nf4``.
 
+Variants of the stored format (same steps, other tables):
+
+* FP4 codebook: "FT-02: QLoRA -- Fine-Tuning with Quantization", section
+  "Exercise 3: NF4 vs FP4 at equal memory": a floating E2M1 grid (sign bit,
+  two exponent bits, one mantissa bit) whose positive levels are printed as
+  0, 0.0052, 0.1667, 0.25, 0.3333, 0.5, 0.6667, 1.
+* FP8 scale codes: FT-02, section "2c. Double quantization" (the constants
+  are quantized in FP8); "QLoRA Deep Dive ...", section "2. Squeezing More
+  Memory: Double Quantization (DQ)" (normalize each block of constants by its
+  absmax and quantize to 8-bit floats, a standard, not quantile, quantization).
+* No double quantization: one fp32 absmax per block, (256 + 32) / 64 = 4.5
+  bits per weight ("QLoRA Deep Dive ...", "Memory Savings Analysis"; FT-02
+  guided example 3, double quantization on/off).
+* 16-bit input weights: FT-02, section "3. BitsAndBytesConfig in practice"
+  (each FP16 weight is converted to 4-bit NormalFloat at load time).
+
 Readings of what the pages leave open (each is also listed in the design
 notes of the repository):
 
@@ -45,6 +61,18 @@ notes of the repository):
   operations in that order, no fused multiply-add.
 * Dequantized weight: ``w_hat = fp32(L[code] * a')``; the bf16 output is that
   value rounded to nearest even.
+* FP4 levels: the printed four-digit values are k/12 for k in {0, 1/16, 2, 3,
+  4, 6, 8, 12} (0.0052 is 1/192 rounded); the levels are those fractions
+  rounded to fp32.  The pages give no bit assignment: code bit 3 is the sign,
+  bits 2..0 the magnitude in increasing order (a float's bit pattern orders
+  its magnitudes), so code 8 is -0.  The nearest-level rule is NF4's (lowest
+  code on a tie), which never picks code 8 and sends ties between two levels
+  of one sign to the smaller magnitude.  An odd count is padded with code 0.
+* FP8 scale codes: E4M3 (bias 7, three mantissa bits, subnormals, no
+  infinities), the normalized value ``fp32(d / c2)`` rounded to the nearest
+  E4M3 value, ties to even; code 0 where ``c2 == 0``.  Decoded scale:
+  ``a' = fp32(fp32(E4M3(q) * c2) + mu)``.
+* 16-bit inputs are widened to fp32 exactly and quantized as fp32.
 """
 
 from __future__ import annotations
@@ -80,6 +108,18 @@ NF4_LEVELS = np.array(
     dtype=np.float32,
 )
 
+# The FP4 (E2M1) levels in code order: codes 0..7 are the magnitudes k / 12,
+# k in {0, 1/16, 2, 3, 4, 6, 8, 12}, ascending; code 8 + c is the negative of
+# code c ("FT-02: QLoRA -- Fine-Tuning with Quantization", "Exercise 3: NF4 vs
+# FP4 at equal memory").
+FP4_TWELFTHS = (0.0, 1.0 / 16.0, 2.0, 3.0, 4.0, 6.0, 8.0, 12.0)
+FP4_LEVELS = np.array([F32(k / 12.0) for k in FP4_TWELFTHS] + [-F32(k / 12.0) for k in FP4_TWELFTHS],
+                      dtype=np.float32)
+
+CODEBOOKS = {"nf4": NF4_LEVELS, "fp4": FP4_LEVELS}
+PAD_CODES = {"nf4": 7, "fp4": 0}  # the +0 level: pad code of an odd count
+SCALE_FORMATS = ("dq_int8", "dq_fp8", "fp32")
+
 BLOCK = 64  # weights per first-level block
 DQ_BLOCK = 256  # first-level scales per double-quant chunk
 ZERO_CODE = 7  # index of the exact 0.0 level; also the odd-count pad code
@@ -100,32 +140,33 @@ def assert_ieee_subnormals() -> None:
         raise RuntimeError("host FPU flushes fp32 subnormals; oracle results would be wrong")
 
 
-def nearest_level(x: np.ndarray) -> np.ndarray:
-    """Step Q3: index of the nearest NF4 level of each fp32 value.
+def nearest_level(x: np.ndarray, levels: np.ndarray = NF4_LEVELS) -> np.ndarray:
+    """Step Q3: index of the nearest level of each fp32 value.
 
     ``code = argmin_j |x - L_j|`` with every difference and absolute value in
     fp32, ties going to the lowest index (numpy ``argmin`` returns the first
     minimum), exactly as the teaching quantizer's ``argmin`` over the level
-    axis.
+    axis.  ``levels`` is the codebook in code order (NF4 by default).
     """
     x = np.asarray(x, dtype=F32).ravel()
+    levels = np.asarray(levels, dtype=F32)
     out = np.empty(x.size, dtype=np.uint8)
     for s in range(0, x.size, _CHUNK):
         xs = x[s : s + _CHUNK]
-        dist = np.abs(xs[:, None] - NF4_LEVELS[None, :])  # fp32 array
+        dist = np.abs(xs[:, None] - levels[None, :])  # fp32 array
         out[s : s + _CHUNK] = dist.argmin(axis=1).astype(np.uint8)
     return out
 
 
-def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+def pack_nibbles(codes: np.ndarray, pad_code: int = ZERO_CODE) -> np.ndarray:
     """Step Q4: two 4-bit codes per byte, element ``2i`` in the low nibble.
 
-    An odd number of codes is padded with code 7 (the zero level), as the
-    teaching quantizer does.
+    An odd number of codes is padded with the zero level's code (7 for NF4),
+    as the teaching quantizer does.
     """
     c = np.asarray(codes, dtype=np.uint8).ravel()
     if c.size % 2:
-        c = np.append(c, np.uint8(ZERO_CODE))
+        c = np.append(c, np.uint8(pad_code))
     return (c[0::2] | (c[1::2] << 4)).astype(np.uint8)
 
 
@@ -147,7 +188,7 @@ def blocks_of(w: np.ndarray, block: int = BLOCK) -> np.ndarray:
     return flat.reshape(-1, block)
 
 
-def quantize_nf4(w: np.ndarray, block: int = BLOCK):
+def quantize_nf4(w: np.ndarray, block: int = BLOCK, codebook: str = "nf4"):
     """Steps Q0-Q4: fp32 weights -> (codes, fp32 block absmax, packed bytes).
 
     Q0 rejects an empty or non-finite input (the teaching quantizer raises
@@ -155,7 +196,8 @@ def quantize_nf4(w: np.ndarray, block: int = BLOCK):
     overflow nor underflow, so its second range guard cannot fire.
     Q1 ``a_b = max |w|`` per block.  Q2 ``x = fp32(w / a_b)``, dividing by 1
     for an all-zero block (the zero-block convention), so that block's codes
-    are all 7 and its stored scale is 0.  Q3 nearest level.  Q4 packing.
+    are all the zero level's code and its stored scale is 0.  Q3 nearest
+    level of ``codebook`` ("nf4" or "fp4").  Q4 packing.
     """
     assert_ieee_subnormals()
     w = np.asarray(w)
@@ -169,8 +211,8 @@ def quantize_nf4(w: np.ndarray, block: int = BLOCK):
     absmax = np.max(np.abs(blocks), axis=1).astype(F32)
     divisor = np.where(absmax == 0, F32(1.0), absmax).astype(F32)
     x = (blocks / divisor[:, None]).astype(F32)
-    codes = nearest_level(x)
-    return codes, absmax, pack_nibbles(codes)
+    codes = nearest_level(x, CODEBOOKS[codebook])
+    return codes, absmax, pack_nibbles(codes, PAD_CODES[codebook])
 
 
 def sequential_sum_f64(values: np.ndarray) -> float:
@@ -198,35 +240,84 @@ def mean_offset(absmax: np.ndarray, dq_block: int = DQ_BLOCK) -> np.float32:
     return F32(np.float64(total) / np.float64(nb))
 
 
-def double_quantize(absmax: np.ndarray, dq_block: int = DQ_BLOCK):
-    """Steps D1-D4: fp32 block scales -> (int8 codes q, fp32 c2 per chunk, fp32 mu).
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """fp32 -> E4M3 codes (uint8), round to nearest, ties to even, saturating.
+
+    E4M3: sign bit, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0
+    holds the subnormals m * 2^-9; the largest finite magnitude is 448
+    (code 0x7E; 0x7F is NaN; no infinities).  In binade [2^E, 2^(E+1)),
+    E >= -6, the spacing is 2^(E-3); below 2^-6 it is 2^-9 (the subnormals
+    continue the lowest binade's spacing).  So the magnitude code is
+    8 E + 48 + rint(|x| / 2^(E-3)) with E = max(floor(log2 |x|), -6): a
+    rounding up to the next power of two carries into the exponent field by
+    itself.  Magnitudes past 448 saturate to 0x7E.  The sign bit is the
+    input's (-0 gives 0x80).
+    """
+    x = np.asarray(x, dtype=F32)
+    if not np.isfinite(x).all():
+        raise ValueError("e4m3_encode takes finite values")
+    a = np.abs(x).astype(np.float64)
+    _, ex = np.frexp(a)  # a = f 2^ex, f in [0.5, 1)
+    E = np.where(a >= 2.0 ** -6, ex - 1, -6).astype(np.int64)
+    k = np.rint(np.ldexp(a, -(E - 3)))  # exact scaling; rint is half-to-even
+    mag = np.minimum(8 * E + 48 + k.astype(np.int64), 0x7E)
+    sign = np.signbit(x).astype(np.int64) << 7
+    return (sign | mag).astype(np.uint8)
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """E4M3 codes -> fp32 values (exact): (8 + m) 2^(e-10) for e >= 1,
+    m 2^-9 for e = 0; NaN for magnitude 0x7F."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    e, m = (c >> 3) & 0xF, c & 0x7
+    mag = np.where(e == 0, np.ldexp(m.astype(np.float64), -9),
+                   np.ldexp((8 + m).astype(np.float64), (e - 10).astype(np.int64)))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return np.where(c >> 7 == 1, -mag, mag).astype(F32)
+
+
+def double_quantize(absmax: np.ndarray, dq_block: int = DQ_BLOCK, scale_format: str = "dq_int8"):
+    """Steps D1-D4: fp32 block scales -> (8-bit codes q, fp32 c2 per chunk, fp32 mu).
 
     D2 ``d_b = fp32(a_b - mu)``.  D3 ``c2_j = max |d_b|`` over the (possibly
-    partial, last) chunk ``j``.  D4 ``q_b = rint(fp32(fp32(d_b / c2_j) * 127))``
-    with ties to even, or 0 where ``c2_j == 0``.
+    partial, last) chunk ``j``.  D4, "dq_int8": ``q_b = rint(fp32(fp32(d_b /
+    c2_j) * 127))`` with ties to even (int8); "dq_fp8": ``q_b =
+    E4M3(fp32(d_b / c2_j))`` (uint8 codes).  ``q_b = 0`` where ``c2_j == 0``.
     """
+    if scale_format not in ("dq_int8", "dq_fp8"):
+        raise ValueError(scale_format)
     a = np.asarray(absmax, dtype=F32).ravel()
     mu = mean_offset(a, dq_block)
     d = (a - mu).astype(F32)
     n_chunks = -(-a.size // dq_block)
     c2 = np.empty(n_chunks, dtype=F32)
-    q = np.zeros(a.size, dtype=np.int8)
+    q = np.zeros(a.size, dtype=np.int8 if scale_format == "dq_int8" else np.uint8)
     for j in range(n_chunks):
         dj = d[j * dq_block : (j + 1) * dq_block]
         c = F32(np.max(np.abs(dj)))
         c2[j] = c
         if c != 0:
             ratio = (dj / c).astype(F32)
-            scaled = (ratio * F32(127.0)).astype(F32)
-            q[j * dq_block : (j + 1) * dq_block] = np.rint(scaled).astype(np.int8)
+            if scale_format == "dq_int8":
+                scaled = (ratio * F32(127.0)).astype(F32)
+                q[j * dq_block : (j + 1) * dq_block] = np.rint(scaled).astype(np.int8)
+            else:
+                q[j * dq_block : (j + 1) * dq_block] = e4m3_encode(ratio)
     return q, c2, mu
 
 
-def decode_scales(q: np.ndarray, c2: np.ndarray, mu, dq_block: int = DQ_BLOCK) -> np.ndarray:
-    """Step R1: ``a'_b = fp32(fp32(fp32(q_b / 127) * c2_j) + mu)``."""
-    q = np.asarray(q, dtype=np.int8).ravel()
-    c = np.repeat(np.asarray(c2, dtype=F32), dq_block)[: q.size]
-    t = (q.astype(F32) / F32(127.0)).astype(F32)
+def decode_scales(q: np.ndarray, c2: np.ndarray, mu, dq_block: int = DQ_BLOCK,
+                  scale_format: str = "dq_int8") -> np.ndarray:
+    """Step R1: ``a'_b = fp32(fp32(t_b * c2_j) + mu)`` with ``t_b = fp32(q_b /
+    127)`` ("dq_int8") or the E4M3 value of ``q_b`` ("dq_fp8")."""
+    c = np.repeat(np.asarray(c2, dtype=F32), dq_block)[: np.asarray(q).size]
+    if scale_format == "dq_int8":
+        q = np.asarray(q, dtype=np.int8).ravel()
+        t = (q.astype(F32) / F32(127.0)).astype(F32)
+    elif scale_format == "dq_fp8":
+        t = e4m3_decode(np.asarray(q).view(np.uint8).ravel())
+    else:
+        raise ValueError(scale_format)
     t = (t * c).astype(F32)
     return (t + F32(mu)).astype(F32)
 
@@ -243,11 +334,12 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(F32)
 
 
-def dequantize_codes(codes: np.ndarray, scales: np.ndarray, block: int = BLOCK) -> np.ndarray:
+def dequantize_codes(codes: np.ndarray, scales: np.ndarray, block: int = BLOCK,
+                     levels: np.ndarray = NF4_LEVELS) -> np.ndarray:
     """Step R2 in fp32: ``w_hat = fp32(L[code] * a'_b)`` for every code."""
     codes = np.asarray(codes, dtype=np.uint8).ravel()
     per = np.repeat(np.asarray(scales, dtype=F32), block)[: codes.size]
-    return (NF4_LEVELS[codes] * per).astype(F32)
+    return (np.asarray(levels, dtype=F32)[codes] * per).astype(F32)
 
 
 @dataclass
@@ -256,34 +348,59 @@ class NF4DQState:
 
     shape: tuple
     packed: np.ndarray  # uint8 [n/2]
-    qscale: np.ndarray  # int8  [n/64]
+    qscale: np.ndarray  # int8 (dq_int8) or uint8 E4M3 (dq_fp8) [n/64]; unused for fp32 scales
     c2: np.ndarray  # fp32  [ceil(n/16384)]
     mu: np.float32  # fp32 scalar
-    absmax: np.ndarray  # fp32 [n/64] first-level scales (kept for diagnostics)
+    absmax: np.ndarray  # fp32 [n/64] first-level scales (the stored scales for "fp32")
+    codebook: str = "nf4"
+    scale_format: str = "dq_int8"
 
     @property
     def n(self) -> int:
         return int(np.prod(self.shape))
 
 
-def quantize_weight(w: np.ndarray) -> NF4DQState:
-    """Steps Q0-Q4 then D1-D4 on one tensor."""
+def widen_16bit(bits: np.ndarray, dtype: str) -> np.ndarray:
+    """16-bit weights (bit patterns, uint16) -> the fp32 values they denote.
+
+    "bf16": the bits are the top half of an fp32; "fp16": IEEE half.  Both
+    widenings are exact.
+    """
+    b = np.asarray(bits, dtype=np.uint16)
+    if dtype == "bf16":
+        return (b.astype(np.uint32) << 16).view(F32)
+    if dtype == "fp16":
+        return b.view(np.float16).astype(F32)
+    raise ValueError(dtype)
+
+
+def quantize_weight(w: np.ndarray, codebook: str = "nf4", scale_format: str = "dq_int8") -> NF4DQState:
+    """Steps Q0-Q4 then D1-D4 (none for fp32 scales) on one fp32 tensor."""
     w = np.asarray(w)
-    _, absmax, packed = quantize_nf4(w)
-    q, c2, mu = double_quantize(absmax)
-    return NF4DQState(tuple(w.shape), packed, q, c2, mu, absmax)
+    if scale_format not in SCALE_FORMATS:
+        raise ValueError(scale_format)
+    _, absmax, packed = quantize_nf4(w, codebook=codebook)
+    if scale_format == "fp32":
+        q, c2, mu = np.zeros(0, dtype=np.int8), np.zeros(0, dtype=F32), F32(0.0)
+    else:
+        q, c2, mu = double_quantize(absmax, scale_format=scale_format)
+    return NF4DQState(tuple(w.shape), packed, q, c2, mu, absmax, codebook, scale_format)
 
 
 def dequantize_weight(state: NF4DQState, dtype: str = "fp32", double_quant: bool = True) -> np.ndarray:
     """Steps R1-R2: the reconstructed tensor, fp32 values or bf16 bit patterns.
 
-    ``double_quant=False`` uses the fp32 first-level scales directly (the
-    4.5-bit storage without double quantization).
+    The state's scale format decides the scale decode; ``double_quant=False``
+    uses the fp32 first-level scales of a double-quantized state directly
+    (the 4.5-bit storage without double quantization).
     """
     n = state.n
     codes = unpack_nibbles(state.packed, n)
-    scales = decode_scales(state.qscale, state.c2, state.mu) if double_quant else state.absmax
-    w_hat = dequantize_codes(codes, scales)[:n].reshape(state.shape)
+    if state.scale_format == "fp32" or not double_quant:
+        scales = state.absmax
+    else:
+        scales = decode_scales(state.qscale, state.c2, state.mu, scale_format=state.scale_format)
+    w_hat = dequantize_codes(codes, scales, levels=CODEBOOKS[state.codebook])[:n].reshape(state.shape)
     if dtype == "fp32":
         return w_hat
     if dtype == "bf16":
@@ -301,23 +418,35 @@ def _from_key(k: int) -> np.float32:
     return np.array([u], dtype=np.uint32).view(F32)[0]
 
 
-def decision_thresholds() -> np.ndarray:
+def decision_thresholds(codebook: str = "nf4") -> np.ndarray:
     """The 15 fp32 decision boundaries of :func:`nearest_level` on [-1, 1].
 
-    ``T_j`` (j = 1..15) is the smallest fp32 value whose nearest level has
-    index ``j``, found by bisection over the ordered fp32 bit patterns between
-    ``L[j-1]`` and ``L[j]``.  On that interval only those two levels can be
-    nearest (the other levels are at least one level gap away), the rounded
-    distance to ``L[j-1]`` never decreases and the one to ``L[j]`` never
-    increases as ``x`` grows, so the choice switches once: for every fp32
-    ``x`` in [-1, 1], ``nearest_level(x) = #{ j : x >= T_j }``.
+    Let ``order`` list the codes by increasing level (for a tie in value, the
+    higher code first) and ``rank(x)`` be the position in ``order`` of
+    ``nearest_level(x)``.  ``T_j`` (j = 1..15) is the smallest fp32 value with
+    ``rank >= j``, found by bisection over the ordered fp32 bit patterns
+    between the levels at positions ``j - 1`` and ``j``.  On that interval
+    only those two levels can be nearest (the others are at least one level
+    gap away), the rounded distance to the lower one never decreases and the
+    one to the upper one never increases as ``x`` grows, so ``rank`` switches
+    once: for every fp32 ``x`` in [-1, 1], ``rank(x) = #{ j : x >= T_j }``.
+    Two equal levels (FP4's +0 and -0) give ``T_j = T_(j+1)``: the position
+    of the one the tie rule never picks is skipped.  For NF4 ``order`` is the
+    identity.
     """
+    levels = CODEBOOKS[codebook]
+    order = sorted(range(16), key=lambda c: (float(levels[c]), -c))
+    pos = {c: i for i, c in enumerate(order)}
     out = np.empty(15, dtype=F32)
     for j in range(1, 16):
-        lo, hi = _ordered_key(NF4_LEVELS[j - 1]), _ordered_key(NF4_LEVELS[j])
+        lo, hi = _ordered_key(levels[order[j - 1]]), _ordered_key(levels[order[j]])
+        if hi == lo:
+            # Equal levels: position j - 1 is never chosen, so T_j is the
+            # boundary below it; search from the level at position j - 2.
+            lo = _ordered_key(levels[order[j - 2]])
         while hi - lo > 1:
             mid = (lo + hi) // 2
-            if nearest_level(np.array([_from_key(mid)], dtype=F32))[0] >= j:
+            if pos[int(nearest_level(np.array([_from_key(mid)], dtype=F32), levels)[0])] >= j:
                 hi = mid
             else:
                 lo = mid
