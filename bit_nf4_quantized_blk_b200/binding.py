@@ -37,6 +37,8 @@ EXPORTED = [
     "qlora_nf4_quantize_batched_ws_bytes",
     "qlora_nf4_quantize_batched",
     "qlora_nf4_quantize_noalloc",
+    "qlora_nf4_quantize_ex",
+    "qlora_nf4_quantize_batched_ex",
     "qlora_nf4_dequantize",
     "qlora_nf4_dequantize_batched",
     "qlora_merge",
@@ -56,6 +58,13 @@ class QloraError(RuntimeError):
         super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
 
 
+# qlora_codebook, qlora_scale_format and qlora_input_dtype of the header.
+CODEBOOK_NF4, CODEBOOK_FP4 = 0, 1
+SCALES_DQ_INT8, SCALES_DQ_FP8, SCALES_FP32 = 0, 1, 2
+INPUT_FP32, INPUT_BF16, INPUT_FP16 = 0, 1, 2
+_INPUT_OF_DTYPE = {torch.float32: INPUT_FP32, torch.bfloat16: INPUT_BF16, torch.float16: INPUT_FP16}
+
+
 class QloraNf4WeightC(ctypes.Structure):
     _fields_ = [
         ("rows", ctypes.c_int64),
@@ -64,6 +73,9 @@ class QloraNf4WeightC(ctypes.Structure):
         ("qscale", ctypes.c_void_p),
         ("c2", ctypes.c_void_p),
         ("mu", ctypes.c_void_p),
+        ("codebook", ctypes.c_int32),
+        ("scale_format", ctypes.c_int32),
+        ("absmax", ctypes.c_void_p),
     ]
 
 
@@ -91,6 +103,8 @@ def lib() -> ctypes.CDLL:
         "qlora_nf4_quantize_batched_ws_bytes": (sz, [W, i32]),
         "qlora_nf4_quantize_batched": (i32, [ctypes.POINTER(P), W, i32, P, sz, P, P]),
         "qlora_nf4_quantize_noalloc": (i32, [P, W, P, P]),
+        "qlora_nf4_quantize_ex": (i32, [P, i32, W, P, sz, P, P]),
+        "qlora_nf4_quantize_batched_ex": (i32, [ctypes.POINTER(P), i32, W, i32, P, sz, P, P]),
         "qlora_nf4_dequantize": (i32, [W, P, i32, i32, P]),
         "qlora_nf4_dequantize_batched": (i32, [W, ctypes.POINTER(P), i32, i32, P]),
         "qlora_merge": (i32, [W, P, P, i32, f32, P, i32, P]),
@@ -132,25 +146,35 @@ class NF4Weight:
     rows: int
     cols: int
     packed: torch.Tensor  # uint8 [rows*cols/2]
-    qscale: torch.Tensor  # int8  [rows*cols/64]
-    c2: torch.Tensor  # fp32  [n_chunks]
-    mu: torch.Tensor  # fp32  [1]
+    qscale: torch.Tensor | None  # int8 [rows*cols/64] (int8 or E4M3 codes); None for fp32 scales
+    c2: torch.Tensor | None  # fp32 [n_chunks]; None for fp32 scales
+    mu: torch.Tensor | None  # fp32 [1]; None for fp32 scales
+    codebook: int = CODEBOOK_NF4
+    scale_format: int = SCALES_DQ_INT8
+    absmax: torch.Tensor | None = None  # fp32 [rows*cols/64] for fp32 scales
 
     @classmethod
-    def empty(cls, rows: int, cols: int, device="cuda") -> "NF4Weight":
+    def empty(cls, rows: int, cols: int, device="cuda", codebook: int = CODEBOOK_NF4,
+              scale_format: int = SCALES_DQ_INT8) -> "NF4Weight":
         s = qlora_nf4_sizes(rows, cols)
+        packed = torch.empty(s["packed_bytes"], dtype=torch.uint8, device=device)
+        if scale_format == SCALES_FP32:
+            return cls(rows, cols, packed, None, None, None, codebook, scale_format,
+                       torch.empty(s["n_blocks"], dtype=torch.float32, device=device))
         return cls(
             rows,
             cols,
-            torch.empty(s["packed_bytes"], dtype=torch.uint8, device=device),
+            packed,
             torch.empty(s["n_blocks"], dtype=torch.int8, device=device),
             torch.empty(s["n_chunks"], dtype=torch.float32, device=device),
             torch.empty(1, dtype=torch.float32, device=device),
+            codebook,
+            scale_format,
         )
 
     def c_struct(self) -> QloraNf4WeightC:
-        return QloraNf4WeightC(self.rows, self.cols, self.packed.data_ptr(), self.qscale.data_ptr(),
-                               self.c2.data_ptr(), self.mu.data_ptr())
+        return QloraNf4WeightC(self.rows, self.cols, self.packed.data_ptr(), _ptr(self.qscale), _ptr(self.c2),
+                               _ptr(self.mu), self.codebook, self.scale_format, _ptr(self.absmax))
 
 
 def qlora_status_string(status: int) -> str:
@@ -169,6 +193,25 @@ def qlora_nf4_quantize(W: torch.Tensor, out: NF4Weight, ws: torch.Tensor, d_stat
     _check("qlora_nf4_quantize", lib().qlora_nf4_quantize(W.data_ptr(), ctypes.byref(st), ws.data_ptr(),
                                                           ws.numel() * ws.element_size(), _ptr(d_status),
                                                           _stream(stream)))
+
+
+def qlora_nf4_quantize_ex(W: torch.Tensor, out: NF4Weight, ws: torch.Tensor, d_status=None, stream=None) -> None:
+    """Quantize an fp32, bf16 or fp16 tensor (the input dtype follows W.dtype)."""
+    st = out.c_struct()
+    _check("qlora_nf4_quantize_ex",
+           lib().qlora_nf4_quantize_ex(W.data_ptr(), _INPUT_OF_DTYPE[W.dtype], ctypes.byref(st), ws.data_ptr(),
+                                       ws.numel() * ws.element_size(), _ptr(d_status), _stream(stream)))
+
+
+def qlora_nf4_quantize_batched_ex(Ws, outs, ws: torch.Tensor, d_status=None, stream=None) -> None:
+    dtypes = {w.dtype for w in Ws}
+    if len(dtypes) != 1:
+        raise ValueError("one input dtype per call")
+    arr = _weight_array(outs)
+    ptrs = (ctypes.c_void_p * len(Ws))(*[w.data_ptr() for w in Ws])
+    _check("qlora_nf4_quantize_batched_ex",
+           lib().qlora_nf4_quantize_batched_ex(ptrs, _INPUT_OF_DTYPE[dtypes.pop()], arr, len(outs), ws.data_ptr(),
+                                               ws.numel() * ws.element_size(), _ptr(d_status), _stream(stream)))
 
 
 def _weight_array(ws):

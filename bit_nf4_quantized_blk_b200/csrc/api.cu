@@ -7,6 +7,7 @@
 // here from the codebook of "QLoRA: NF4 storage, gradients and local
 // integration" (section "Exact CPU teaching quantizer and adapter gradient
 // path") with the same fp32 rule the definition uses.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -25,12 +26,12 @@ namespace {
 // ---------------------------------------------------------------------------
 
 // Nearest level of x by the definition: fp32 distances |x - L_j|, the lowest
-// index wins a tie.  Host fp32 arithmetic (SSE, no contraction) is IEEE.
-int host_nearest(float x) {
+// code wins a tie.  Host fp32 arithmetic (SSE, no contraction) is IEEE.
+int host_nearest_code(int codebook, float x) {
   int best = 0;
-  volatile float bd = std::fabs(x - nf4_level(0));
+  volatile float bd = std::fabs(x - codebook_level(codebook, 0));
   for (int j = 1; j < 16; ++j) {
-    volatile float d = std::fabs(x - nf4_level(j));
+    volatile float d = std::fabs(x - codebook_level(codebook, j));
     if (d < bd) {
       bd = d;
       best = j;
@@ -52,44 +53,101 @@ float from_key(int64_t k) {
   return f;
 }
 
-// The 15 decision thresholds: T_j is the smallest fp32 x whose nearest level
-// is j (the choice between neighbouring levels flips once between them).
-void derive_thresholds(float (&T)[16]) {
+// The codebook's distinct levels in increasing order, each with the code the
+// tie rule picks for it (NF4: 16 levels, positions = codes; FP4: 15, +0 and
+// -0 being one value whose code is 0).
+struct SortedLevels {
+  int n = 0;
+  float level[16];
+  int code[16];
+  int pos_of_code[16];
+};
+
+SortedLevels sorted_levels(int codebook) {
+  SortedLevels s;
+  int order[16];
+  for (int j = 0; j < 16; ++j) order[j] = j;
+  std::sort(order, order + 16, [&](int a, int b) {
+    const float la = codebook_level(codebook, a), lb = codebook_level(codebook, b);
+    return la < lb || (la == lb && a < b);
+  });
+  for (int i = 0; i < 16; ++i) {
+    const int c = order[i];
+    const float l = codebook_level(codebook, c);
+    if (s.n > 0 && s.level[s.n - 1] == l) {  // equal value: the lower code (first in order) stays
+      s.pos_of_code[c] = s.n - 1;
+      continue;
+    }
+    s.level[s.n] = l;
+    s.code[s.n] = c;
+    s.pos_of_code[c] = s.n;
+    ++s.n;
+  }
+  return s;
+}
+
+int host_position(int codebook, const SortedLevels& s, float x) {
+  return s.pos_of_code[host_nearest_code(codebook, x)];
+}
+
+// The n - 1 decision thresholds: T_j is the smallest fp32 x whose nearest
+// level has position >= j (the choice between neighbouring levels flips once
+// between them).
+void derive_thresholds(int codebook, const SortedLevels& s, float (&T)[16]) {
   T[0] = -INFINITY;
-  for (int j = 1; j < 16; ++j) {
-    int64_t lo = ordered_key(nf4_level(j - 1)), hi = ordered_key(nf4_level(j));
+  for (int j = 1; j < s.n; ++j) {
+    int64_t lo = ordered_key(s.level[j - 1]), hi = ordered_key(s.level[j]);
     while (hi - lo > 1) {
       const int64_t mid = lo + (hi - lo) / 2;
-      if (host_nearest(from_key(mid)) >= j) hi = mid; else lo = mid;
+      if (host_position(codebook, s, from_key(mid)) >= j) hi = mid; else lo = mid;
     }
     T[j] = from_key(hi);
   }
 }
 
-// Cells of x in [-1, 1] by c = trunc(64 x) + 64; each cell is an interval of
-// fp32 values [xlo, xhi] that holds at most one threshold, so
-// code(x) = base[c] + (x >= thr[c]).  Verified against host_nearest at every
-// cell edge and around every threshold.
-bool build_decision_table(Nf4DecisionTable* tab) {
+// Cells of x in [-1, 1]; each is an interval of fp32 values [xlo, xhi] that
+// holds at most one threshold, so pos(x) = base[c] + (x >= thr[c]).
+//   NF4 (trunc cells): c = trunc(64 x) + 64, c = 0 .. 128 (cell 64 is
+//   (-1/64, 1/64)).  FP4 (floor cells): c = floor(64 x) + 65, c = 1 .. 128
+//   cover [k/64, (k+1)/64), k = c - 65; cells 0 and 129 take the products a
+//   rounding below -64 or at 64 (x = -1, x = 1).  Verified against the
+//   definition at every cell edge and around every threshold.
+bool build_decision_table(int codebook, Nf4DecisionTable* tab) {
+  const SortedLevels s = sorted_levels(codebook);
   float T[16];
-  derive_thresholds(T);
+  derive_thresholds(codebook, s, T);
+  const bool floor_cells = codebook == QLORA_CODEBOOK_FP4;
   int cells_with_threshold = 0;
-  for (int c = 0; c <= 128; ++c) {
-    const int t = c - 64;
+  for (int c = 0; c < kDecisionCells; ++c) {
     float xlo, xhi;
-    if (t >= 1) {
-      xlo = static_cast<float>(t) / 64.0f;
-      xhi = t == 64 ? 1.0f : std::nextafter(static_cast<float>(t + 1) / 64.0f, -INFINITY);
-    } else if (t == 0) {
-      xlo = std::nextafter(-1.0f / 64.0f, INFINITY);
-      xhi = std::nextafter(1.0f / 64.0f, -INFINITY);
+    if (floor_cells) {
+      const int k = c - 65;
+      if (k < -64) {
+        xlo = xhi = -1.0f;
+      } else if (k >= 64) {
+        xlo = xhi = 1.0f;
+      } else {
+        xlo = static_cast<float>(k) / 64.0f;
+        xhi = std::nextafter(static_cast<float>(k + 1) / 64.0f, -INFINITY);
+      }
     } else {
-      xlo = t == -64 ? -1.0f : std::nextafter(static_cast<float>(t - 1) / 64.0f, INFINITY);
-      xhi = static_cast<float>(t) / 64.0f;
+      const int t = c - 64;
+      if (t > 64) {  // not addressed by trunc cells
+        xlo = xhi = 1.0f;
+      } else if (t >= 1) {
+        xlo = static_cast<float>(t) / 64.0f;
+        xhi = t == 64 ? 1.0f : std::nextafter(static_cast<float>(t + 1) / 64.0f, -INFINITY);
+      } else if (t == 0) {
+        xlo = std::nextafter(-1.0f / 64.0f, INFINITY);
+        xhi = std::nextafter(1.0f / 64.0f, -INFINITY);
+      } else {
+        xlo = t == -64 ? -1.0f : std::nextafter(static_cast<float>(t - 1) / 64.0f, INFINITY);
+        xhi = static_cast<float>(t) / 64.0f;
+      }
     }
     int base = 0, inside = 0;
     float thr = 4.0f;  // no threshold in this cell: a value no x in [-1, 1] reaches
-    for (int j = 1; j < 16; ++j) {
+    for (int j = 1; j < s.n; ++j) {
       if (T[j] <= xlo) ++base;
       else if (T[j] <= xhi) {
         thr = T[j];
@@ -102,25 +160,31 @@ bool build_decision_table(Nf4DecisionTable* tab) {
     if (inside && (thr - xlo < std::fabs(thr) * 0x1p-14f || xhi - thr < std::fabs(thr) * 0x1p-14f)) return false;
     tab->thr[c] = thr;
     tab->base[c] = base;
-    auto code_of = [&](float x) { return base + (x >= thr ? 1 : 0); };
-    if (code_of(xlo) != host_nearest(xlo) || code_of(xhi) != host_nearest(xhi)) return false;
+    auto pos_of = [&](float x) { return base + (x >= thr ? 1 : 0); };
+    if (pos_of(xlo) != host_position(codebook, s, xlo) || pos_of(xhi) != host_position(codebook, s, xhi)) return false;
     if (inside) {
-      if (code_of(thr) != host_nearest(thr)) return false;
+      if (pos_of(thr) != host_position(codebook, s, thr)) return false;
       const float below = std::nextafter(thr, -INFINITY);
-      if (code_of(below) != host_nearest(below)) return false;
+      if (pos_of(below) != host_position(codebook, s, below)) return false;
       if (thr != T[base + 1]) return false;  // the cell's threshold is the next one above its base
       ++cells_with_threshold;
     }
   }
-  return cells_with_threshold == 15;  // every threshold sits inside exactly one cell
+  // every threshold sits inside exactly one cell
+  if (cells_with_threshold != s.n - 1) return false;
+  // the kernel's position -> code mapping (identity for NF4)
+  for (int i = 0; i < s.n; ++i)
+    if ((floor_cells ? fp4_code_of_position(i) : i) != s.code[i]) return false;
+  return true;
 }
 
-const Nf4DecisionTable* decision_table() {
-  static Nf4DecisionTable tab;
-  static bool ok = false;
-  static std::once_flag once;
-  std::call_once(once, [] { ok = build_decision_table(&tab); });
-  return ok ? &tab : nullptr;
+const Nf4DecisionTable* decision_table(int codebook) {
+  static Nf4DecisionTable tab[2];
+  static bool ok[2] = {false, false};
+  static std::once_flag once[2];
+  if (codebook != QLORA_CODEBOOK_NF4 && codebook != QLORA_CODEBOOK_FP4) return nullptr;
+  std::call_once(once[codebook], [codebook] { ok[codebook] = build_decision_table(codebook, &tab[codebook]); });
+  return ok[codebook] ? &tab[codebook] : nullptr;
 }
 
 // ---------------------------------------------------------------------------
@@ -205,10 +269,27 @@ qlora_status check_weight(const qlora_nf4_weight* w) {
   if (w == nullptr) return QLORA_ERR_INVALID_ARG;
   if (w->rows < 1 || w->cols < kBlock || w->cols % kBlock != 0) return QLORA_ERR_INVALID_ARG;
   if (w->rows > (int64_t{1} << 40) / w->cols) return QLORA_ERR_UNSUPPORTED;
-  if (!w->packed || !w->qscale || !w->c2 || !w->mu) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(w->packed, 16) || !aligned(w->qscale, 16) || !aligned(w->c2, 4) || !aligned(w->mu, 4))
-    return QLORA_ERR_ALIGNMENT;
+  if (w->codebook != QLORA_CODEBOOK_NF4 && w->codebook != QLORA_CODEBOOK_FP4) return QLORA_ERR_INVALID_ARG;
+  if (w->scale_format != kScalesDqInt8 && w->scale_format != kScalesDqFp8 && w->scale_format != kScalesFp32)
+    return QLORA_ERR_INVALID_ARG;
+  if (!w->packed) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(w->packed, 16)) return QLORA_ERR_ALIGNMENT;
+  if (w->scale_format == kScalesFp32) {
+    if (!w->absmax) return QLORA_ERR_INVALID_ARG;
+    if (!aligned(w->absmax, 16)) return QLORA_ERR_ALIGNMENT;
+    return QLORA_OK;
+  }
+  if (!w->qscale || !w->c2 || !w->mu) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(w->qscale, 16) || !aligned(w->c2, 4) || !aligned(w->mu, 4)) return QLORA_ERR_ALIGNMENT;
   return QLORA_OK;
+}
+
+// Input weights: fp32 needs 32-byte alignment (256-bit loads), bf16 / fp16 16.
+qlora_status check_input(const void* W, int32_t in_dtype) {
+  if (W == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (in_dtype != QLORA_INPUT_FP32 && in_dtype != QLORA_INPUT_BF16 && in_dtype != QLORA_INPUT_FP16)
+    return QLORA_ERR_INVALID_ARG;
+  return aligned(W, in_dtype == QLORA_INPUT_FP32 ? 32 : 16) ? QLORA_OK : QLORA_ERR_ALIGNMENT;
 }
 
 int64_t n_chunks_of(int64_t rows, int64_t cols) {
@@ -289,8 +370,29 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+// Tensor i of a dequant batch.
+void set_dequant_tensor(DequantBatchParams& p, int i, const qlora_nf4_weight& w, void* out) {
+  p.n_units[i] = w.rows * w.cols / 32;
+  p.packed[i] = w.packed;
+  p.qscale[i] = w.qscale;
+  p.c2[i] = w.c2;
+  p.mu[i] = w.mu;
+  p.absmax[i] = w.absmax;
+  p.codebook[i] = w.codebook;
+  p.scale_format[i] = w.scale_format;
+  p.out[i] = out;
+}
+
+// A one-tensor dequant batch (the dense bf16 weight of the linear paths).
+void dequant_one(DequantBatchParams& p, const qlora_nf4_weight* w, void* out) {
+  std::memset(&p, 0, sizeof(p));
+  p.count = 1;
+  set_dequant_tensor(p, 0, *w, out);
+  p.begin_seg[1] = p.total_seg = (p.n_units[0] + 127) / 128;
+}
+
 WeightView view_of(const qlora_nf4_weight* w) {
-  return WeightView{w->packed, w->qscale, w->c2, w->mu, w->rows, w->cols};
+  return WeightView{w->packed, w->qscale, w->c2, w->mu, w->rows, w->cols, w->codebook, w->scale_format, w->absmax};
 }
 
 qlora_status check_linear_args(const qlora_nf4_weight* w, int64_t M, int32_t r, size_t ws_bytes, const void* ws) {
@@ -343,14 +445,17 @@ extern "C" size_t qlora_nf4_quantize_batched_ws_bytes(const qlora_nf4_weight* ou
   return quant_ws_layout(count, max_group_chunks(outs, count)).total;
 }
 
-extern "C" qlora_status qlora_nf4_quantize_batched(const float* const* W, const qlora_nf4_weight* outs, int32_t count,
-                                                   void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+extern "C" qlora_status qlora_nf4_quantize_batched_ex(const void* const* W, int32_t in_dtype,
+                                                      const qlora_nf4_weight* outs, int32_t count, void* ws,
+                                                      size_t ws_bytes, int32_t* d_status, void* stream) {
   if (W == nullptr || outs == nullptr || count < 1) return QLORA_ERR_INVALID_ARG;
   for (int32_t i = 0; i < count; ++i) {
-    const qlora_status st = check_weight(&outs[i]);
+    qlora_status st = check_weight(&outs[i]);
     if (st != QLORA_OK) return st;
-    if (W[i] == nullptr) return QLORA_ERR_INVALID_ARG;
-    if (!aligned(W[i], 32)) return QLORA_ERR_ALIGNMENT;
+    if (outs[i].codebook != outs[0].codebook || outs[i].scale_format != outs[0].scale_format)
+      return QLORA_ERR_INVALID_ARG;  // one format per call
+    st = check_input(W[i], in_dtype);
+    if (st != QLORA_OK) return st;
   }
   if (ws == nullptr) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
@@ -359,7 +464,7 @@ extern "C" qlora_status qlora_nf4_quantize_batched(const float* const* W, const 
   if (d_status != nullptr && !aligned(d_status, 4)) return QLORA_ERR_ALIGNMENT;
   qlora_status st = check_device();
   if (st != QLORA_OK) return st;
-  const Nf4DecisionTable* tab = decision_table();
+  const Nf4DecisionTable* tab = decision_table(outs[0].codebook);
   if (tab == nullptr) return QLORA_ERR_UNSUPPORTED;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -386,7 +491,12 @@ extern "C" qlora_status qlora_nf4_quantize_batched(const float* const* W, const 
     }
     p.chunk_begin[n] = c;
     p.total_chunks = c;
+    p.in_dtype = in_dtype;
+    p.codebook = outs[0].codebook;
+    p.scale_format = outs[0].scale_format;
     p.absmax = at<float>(ws, lay.absmax);
+    for (int i = 0; i < n; ++i)
+      p.absmax_dst[i] = p.scale_format == kScalesFp32 ? outs[g0 + i].absmax : p.absmax + p.chunk_begin[i] * kDqBlock;
     p.chunk_sum = at<double>(ws, lay.sums);
     p.chunk_exp = at<int>(ws, lay.exps);
     p.counters = at<unsigned>(ws, lay.counters);
@@ -408,11 +518,22 @@ extern "C" qlora_status qlora_nf4_quantize_batched(const float* const* W, const 
   return static_cast<qlora_status>(h);
 }
 
+extern "C" qlora_status qlora_nf4_quantize_batched(const float* const* W, const qlora_nf4_weight* outs, int32_t count,
+                                                   void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  return qlora_nf4_quantize_batched_ex(reinterpret_cast<const void* const*>(W), QLORA_INPUT_FP32, outs, count, ws,
+                                       ws_bytes, d_status, stream);
+}
+
+extern "C" qlora_status qlora_nf4_quantize_ex(const void* W, int32_t in_dtype, const qlora_nf4_weight* out, void* ws,
+                                              size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (out == nullptr) return QLORA_ERR_INVALID_ARG;
+  const void* const ws_list[1] = {W};
+  return qlora_nf4_quantize_batched_ex(ws_list, in_dtype, out, 1, ws, ws_bytes, d_status, stream);
+}
+
 extern "C" qlora_status qlora_nf4_quantize(const float* W, const qlora_nf4_weight* out, void* ws, size_t ws_bytes,
                                            int32_t* d_status, void* stream) {
-  if (out == nullptr) return QLORA_ERR_INVALID_ARG;
-  const float* const ws_list[1] = {W};
-  return qlora_nf4_quantize_batched(ws_list, out, 1, ws, ws_bytes, d_status, stream);
+  return qlora_nf4_quantize_ex(W, QLORA_INPUT_FP32, out, ws, ws_bytes, d_status, stream);
 }
 
 extern "C" qlora_status qlora_nf4_dequantize_batched(const qlora_nf4_weight* weights, void* const* outs, int32_t count,
@@ -437,12 +558,7 @@ extern "C" qlora_status qlora_nf4_dequantize_batched(const qlora_nf4_weight* wei
     for (int i = 0; i < n; ++i) {
       const qlora_nf4_weight& w = weights[g0 + i];
       p.begin_seg[i] = c;
-      p.n_units[i] = w.rows * w.cols / 32;
-      p.packed[i] = w.packed;
-      p.qscale[i] = w.qscale;
-      p.c2[i] = w.c2;
-      p.mu[i] = w.mu;
-      p.out[i] = outs[g0 + i];
+      set_dequant_tensor(p, i, w, outs[g0 + i]);
       c += (p.n_units[i] + 127) / 128;
     }
     p.begin_seg[n] = c;
@@ -531,8 +647,10 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
     GemvParams gp{};
     gp.packed = w->packed;
     gp.qscale = w->qscale;
-    gp.c2 = w->c2;
+    gp.c2 = w->scale_format == kScalesFp32 ? w->absmax : w->c2;  // fp32 scales: the absmax array
     gp.mu = w->mu;
+    gp.codebook = w->codebook;
+    gp.scale_format = w->scale_format;
     gp.N = N;
     gp.K = K;
     gp.X = X;
@@ -561,15 +679,7 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
   }
   // Tensor-core path: dense bf16 weight, U = X A^T, padded B, GEMM with the rank-r step.
   DequantBatchParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.count = 1;
-  p.n_units[0] = N * K / 32;
-  p.begin_seg[1] = p.total_seg = (p.n_units[0] + 127) / 128;
-  p.packed[0] = w->packed;
-  p.qscale[0] = w->qscale;
-  p.c2[0] = w->c2;
-  p.mu[0] = w->mu;
-  p.out[0] = at<uint16_t>(ws, lay.wbf);
+  dequant_one(p, w, at<uint16_t>(ws, lay.wbf));
   {
     Timed tm(kFamDequant, s);
     e = launch_dequant_batch(p, 0, s);
@@ -664,15 +774,7 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
   }
   if (dX != nullptr) {  // dX = dY W_hat + s V A, reading W_hat [N, K] and A [r, K] as MN-major operands
     DequantBatchParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.count = 1;
-    p.n_units[0] = N * K / 32;
-    p.begin_seg[1] = p.total_seg = (p.n_units[0] + 127) / 128;
-    p.packed[0] = w->packed;
-    p.qscale[0] = w->qscale;
-    p.c2[0] = w->c2;
-    p.mu[0] = w->mu;
-    p.out[0] = at<uint16_t>(ws, lay.wbf);
+    dequant_one(p, w, at<uint16_t>(ws, lay.wbf));
     {
       Timed tm(kFamDequant, s);
       e = launch_dequant_batch(p, 0, s);
@@ -801,7 +903,7 @@ extern "C" qlora_status qlora_nf4_quantize_noalloc(const float* W, const qlora_n
   if (d_status != nullptr && !aligned(d_status, 4)) return QLORA_ERR_ALIGNMENT;
   st = check_device();
   if (st != QLORA_OK) return st;
-  const Nf4DecisionTable* tab = decision_table();
+  const Nf4DecisionTable* tab = decision_table(out->codebook);
   if (tab == nullptr) return QLORA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
@@ -825,7 +927,11 @@ extern "C" qlora_status qlora_nf4_quantize_noalloc(const float* W, const qlora_n
   p.qscale[0] = out->qscale;
   p.c2[0] = out->c2;
   p.mu[0] = out->mu;
+  p.in_dtype = QLORA_INPUT_FP32;
+  p.codebook = out->codebook;
+  p.scale_format = out->scale_format;
   p.absmax = at<float>(scratch, kNoAllocLayout.absmax);
+  p.absmax_dst[0] = p.scale_format == kScalesFp32 ? out->absmax : p.absmax;
   p.chunk_sum = at<double>(scratch, kNoAllocLayout.sums);
   p.chunk_exp = at<int>(scratch, kNoAllocLayout.exps);
   p.counters = at<unsigned>(scratch, kNoAllocLayout.counters);

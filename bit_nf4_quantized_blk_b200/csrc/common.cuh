@@ -497,20 +497,97 @@ __host__ __device__ constexpr float nf4_level(int j) {
                    : 1.0f;
 }
 
-// Decision table of the nearest-level search on x in [-1, 1] (built once on
-// the host, see api.cu): cell c = trunc(64 x) + 64 covers a fixed interval of
-// x holding at most one decision threshold; code(x) = base[c] + (x >= thr[c])
-// (thr[c] = 4 where the cell holds none).
+// The FP4 (E2M1) codebook of "FT-02: QLoRA -- Fine-Tuning with
+// Quantization", section "Exercise 3: NF4 vs FP4 at equal memory": codes 0..7
+// are the magnitudes k / 12, k = 0, 1/16, 2, 3, 4, 6, 8, 12 (printed there as
+// 0, 0.0052, 0.1667, 0.25, 0.3333, 0.5, 0.6667, 1), rounded to fp32; code
+// 8 + c is the negative of code c (bit 3 is the sign).
+__host__ __device__ constexpr float fp4_level(int j) {
+  return (j & 8 ? -1.0f : 1.0f) * ((j & 7) == 0   ? 0.0f
+                                   : (j & 7) == 1 ? 0.005208333333333333f
+                                   : (j & 7) == 2 ? 0.16666666666666666f
+                                   : (j & 7) == 3 ? 0.25f
+                                   : (j & 7) == 4 ? 0.3333333333333333f
+                                   : (j & 7) == 5 ? 0.5f
+                                   : (j & 7) == 6 ? 0.6666666666666666f
+                                                  : 1.0f);
+}
+
+// Level j of a codebook (QLORA_CODEBOOK_NF4 or QLORA_CODEBOOK_FP4).
+__host__ __device__ constexpr float codebook_level(int codebook, int j) {
+  return codebook == QLORA_CODEBOOK_FP4 ? fp4_level(j) : nf4_level(j);
+}
+
+// Decision table of the nearest-level search on x in [-1, 1] (built once per
+// codebook on the host, see api.cu).  A cell covers a fixed interval of x
+// holding at most one decision threshold; pos(x) = base[c] + (x >= thr[c])
+// (thr[c] = 4 where the cell holds none) is x's position among the
+// codebook's distinct levels in increasing order.
+//   NF4: cell c = trunc(64 x) + 64 (c = 0 .. 128); positions are the codes.
+//   FP4: cell c = floor(64 x) + 65 (c = 0 .. 129; cells 0 and 129 catch
+//        |64 x| a rounding past 64); positions 0 .. 14 over the 15 distinct
+//        values (-0 is never chosen), mapped to codes by fp4_codes_of.
+constexpr int kDecisionCells = 130;
 struct Nf4DecisionTable {
-  float thr[129];
-  int base[129];
+  float thr[kDecisionCells];
+  int base[kDecisionCells];
 };
 
-// Decoded first-level scale: a = fp32(fp32(fp32(q / 127) * c2) + mu), three
+// Eight FP4 positions (nibbles, 0 .. 14) -> their sign-magnitude codes:
+// positions 7 .. 14 are +0 .. +1 (codes 0 .. 7), positions 0 .. 6 are
+// -1 .. -1/192 (codes 15 .. 9).  Nibble-parallel: first p16 = p + (p >= 7)
+// (the 16-entry order with -0 at 7), then p16 >= 8 -> p16 - 8 and
+// p16 < 8 -> 15 - p16, i.e. p16 ^ 8 ^ (p16 < 8 ? 7 : 0).  No nibble carries:
+// p + 1 <= 15.
+__host__ __device__ __forceinline__ uint32_t fp4_codes_of(uint32_t pos) {
+  const uint32_t ge7 = ((pos + 0x11111111u) >> 3) & 0x11111111u;
+  const uint32_t p16 = pos + ge7;
+  const uint32_t lt8 = (~p16 >> 3) & 0x11111111u;
+  return p16 ^ 0x88888888u ^ (lt8 * 7u);
+}
+
+__host__ __device__ __forceinline__ int fp4_code_of_position(int pos) {
+  return static_cast<int>(fp4_codes_of(static_cast<uint32_t>(pos)) & 0xFu);
+}
+
+// Scale formats of a quantized tensor (qlora_scale_format).
+constexpr int kScalesDqInt8 = QLORA_SCALES_DQ_INT8;
+constexpr int kScalesDqFp8 = QLORA_SCALES_DQ_FP8;
+constexpr int kScalesFp32 = QLORA_SCALES_FP32;
+
+// E4M3 code -> fp32, exact: (1 + m/8) 2^(e-7) for e >= 1 (the fp32 bit
+// pattern with exponent field e + 120 and the top mantissa bits m), m 2^-9
+// for e = 0.  Stored scale codes are finite (never 0x7F / 0xFF).
+__host__ __device__ __forceinline__ float e4m3_to_float(uint32_t code) {
+  const uint32_t e = (code >> 3) & 0xFu, m = code & 7u;
+  float v;
+  if (e != 0) {
+    const uint32_t bits = ((e + 120u) << 23) | (m << 20);
+#ifdef __CUDA_ARCH__
+    v = __uint_as_float(bits);
+#else
+    __builtin_memcpy(&v, &bits, 4);
+#endif
+  } else {
+    v = static_cast<float>(m) * 0x1p-9f;
+  }
+  return (code & 0x80u) ? -v : v;
+}
+
+// The first factor of a double-quantized scale: fp32(q / 127) for int8
+// codes, the E4M3 value for FP8 codes.
+__device__ __forceinline__ float scale_code_value(int format, int8_t q) {
+  return format == kScalesDqFp8 ? e4m3_to_float(static_cast<uint8_t>(q)) : __fdiv_rn(static_cast<float>(q), 127.0f);
+}
+
+// Decoded first-level scale: a = fp32(fp32(t * c2) + mu), t as above; two
 // rounded operations in this order (no contraction into an FMA).
-__device__ __forceinline__ float decode_scale(int q, float c2, float mu) {
-  const float t = __fdiv_rn(static_cast<float>(q), 127.0f);
+__device__ __forceinline__ float decode_scale_value(float t, float c2, float mu) {
   return __fadd_rn(__fmul_rn(t, c2), mu);
+}
+
+__device__ __forceinline__ float decode_scale(int q, float c2, float mu) {
+  return decode_scale_value(__fdiv_rn(static_cast<float>(q), 127.0f), c2, mu);
 }
 
 }  // namespace qnf4

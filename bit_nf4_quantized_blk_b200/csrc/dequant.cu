@@ -1,11 +1,13 @@
-// NF4 + double-quant dequantization to dense bf16 / fp32 (sm_100a).
+// 4-bit dequantization to dense bf16 / fp32 (sm_100a).
 //
 // Method: "QLoRA Deep Dive: 4-bit NormalFloat & Double Quantization
 // Internals", section "The Quantization Process in QLoRA" (load the 4-bit
 // codes and the block constant, multiply, cast to bf16); "QLoRA: NF4 storage,
 // gradients and local integration", ``dequantize_nf4`` of the teaching
-// program.  Block scale decode a = fp32(fp32(fp32(q/127) * c2) + mu); weight
-// fp32(L[code] * a); bf16 output rounds that value to nearest even.
+// program.  Block scale decode a = fp32(fp32(t * c2) + mu) (t = fp32(q/127)
+// for int8 codes, the E4M3 value for FP8 codes) or the stored fp32 absmax;
+// weight fp32(L[code] * a) with L the NF4 or FP4 codebook; bf16 output
+// rounds that value to nearest even.
 //
 // HBM-bound: 0.5 B of codes + 1/64 B of scale codes read and 2 B (bf16) or
 // 4 B (fp32) written per weight.
@@ -16,8 +18,9 @@ namespace qnf4 {
 
 namespace {
 
-__device__ __forceinline__ void fill_pair_table(float2* tab) {
-  for (int b = threadIdx.x; b < 256; b += blockDim.x) tab[b] = make_float2(nf4_level(b & 15), nf4_level(b >> 4));
+__device__ __forceinline__ void fill_pair_table(float2* tab, int codebook) {
+  for (int b = threadIdx.x; b < 256; b += blockDim.x)
+    tab[b] = make_float2(codebook_level(codebook, b & 15), codebook_level(codebook, b >> 4));
 }
 
 }  // namespace
@@ -41,14 +44,15 @@ __device__ __forceinline__ int find_tensor_seg(const DequantBatchParams& p, int6
 template <bool kFp32>
 __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ DequantBatchParams p) {
   const int lane = threadIdx.x & 31;
-  const float level = nf4_level(lane & 15);
   const int64_t gseg = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (gseg >= p.total_seg) return;
   const int t = find_tensor_seg(p, gseg);
+  const float level = codebook_level(p.codebook[t], lane & 15);
   const int64_t seg = gseg - p.begin_seg[t];
   const int64_t n_units = p.n_units[t];
   const uint4* __restrict__ packed = reinterpret_cast<const uint4*>(p.packed[t]);
-  const float mu = *p.mu[t];
+  const int fmt = p.scale_format[t];
+  const float mu = fmt == kScalesFp32 ? 0.0f : *p.mu[t];
   uint4 pk[4];
   float a[4];
 #pragma unroll
@@ -58,12 +62,31 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
     a[q] = 0.0f;
     if (u < n_units) pk[q] = ld_stream_u4(packed + u);
   }
+  // Scales of the four units (two units per 64-weight block); one uniform
+  // branch on the format, the loads of each branch issued together.
+  if (fmt == kScalesFp32) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int64_t u = seg * 128 + lane + 32 * q;
-    if (u < n_units) {
-      const int64_t blk = u >> 1;  // two units per 64-weight block
-      a[q] = decode_scale(p.qscale[t][blk], p.c2[t][blk / kDqBlock], mu);
+    for (int q = 0; q < 4; ++q) {
+      const int64_t u = seg * 128 + lane + 32 * q;
+      if (u < n_units) a[q] = p.absmax[t][u >> 1];
+    }
+  } else {
+    int qv[4];
+    float c2v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t u = seg * 128 + lane + 32 * q;
+      qv[q] = 0;
+      c2v[q] = 0.0f;
+      if (u < n_units) {
+        qv[q] = p.qscale[t][u >> 1];
+        c2v[q] = p.c2[t][(u >> 1) / kDqBlock];
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t u = seg * 128 + lane + 32 * q;
+      if (u < n_units) a[q] = decode_scale_value(scale_code_value(fmt, static_cast<int8_t>(qv[q])), c2v[q], mu);
     }
   }
   // Every lane takes part in the shuffles; units past the end are skipped
@@ -108,7 +131,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
 __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, uint16_t* __restrict__ out) {
   __shared__ float2 s_pair[256];
   __shared__ __align__(16) uint16_t s_t[64][64];  // [k][n]
-  fill_pair_table(s_pair);
+  fill_pair_table(s_pair, w.codebook);
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 64;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * 64;
   const int tid = threadIdx.x;
@@ -120,7 +143,7 @@ __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, u
   float a = 0.0f;
   if (n < w.rows) {
     const int64_t blk = (n * w.cols + k0) / kBlock;
-    a = decode_scale(w.qscale[blk], w.c2[blk / kDqBlock], *w.mu);
+    a = weight_block_scale(w, blk, weight_mu(w));
     const uint2 pk = *reinterpret_cast<const uint2*>(w.packed + (n * w.cols + k0 + kq) / 2);
     lo = pk.x;
     hi = pk.y;

@@ -189,7 +189,7 @@ struct GvCursor {
 // pairs per k16 step; every tile runs the same straight-line code (no branch
 // inside a tile: pieces past the end are zero-filled copies, blocks past the
 // end of K meet zero X fragments).
-template <bool kM16>
+template <bool kM16, bool kScales32>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
   constexpr int NT = kM16 ? 2 : 1;  // token tiles of 8
   constexpr int P = kM16 ? 2 : 4;   // tiles per reduction pass
@@ -257,8 +257,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
 #pragma unroll 1
   for (int i = 0; i < kGvDepth; ++i) issue_next();
 
-  if (tid < 16) s_lev[tid] = nf4_level(tid);
-  if (tid < 256) s_qdiv[tid] = __fdiv_rn(static_cast<float>(tid - 128), 127.0f);
+  if (tid < 16) s_lev[tid] = codebook_level(p.codebook, tid);
+  if (tid < 256) s_qdiv[tid] = scale_table_entry(p.scale_format, tid);
   __syncthreads();
   // lut[byte][64 words]: word `lane` = (L[byte & 15], L[byte >> 4]) as bf16.
   for (int i = tid; i < 256 * 32; i += kGvThreads) {
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
     lut[byte * 64 + l] = pack_bf16x2(s_lev[byte & 15], s_lev[byte >> 4]);
   }
 
-  const float mu = *p.mu;
+  const float mu = kScales32 ? 0.0f : *p.mu;
   const uint32_t lane_base = kLutWindow | (static_cast<uint32_t>(lane) * 4);
   // Scales this lane decodes per item: row lane%16 of the tile, blocks
   // 4 warp + lane/16 and 4 warp + lane/16 + 2; the lanes holding rows g and
@@ -283,8 +283,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
     for (int e = 0; e < 2; ++e) {
       const bool v = live && row < N && blk + 2 * e < nbk;
       const int64_t gb = v ? row * nbk + blk + 2 * e : 0;
-      const int q = p.qscale[gb];
-      const float c2 = __ldg(p.c2 + (gb >> 8));
+      // fp32 scales: t(127) = 1, "c2" is the block's absmax and mu = 0, so
+      // the decode below returns the absmax itself.
+      const int q = kScales32 ? 127 : p.qscale[gb];
+      const float c2 = __ldg(p.c2 + (kScales32 ? gb : gb >> 8));
       qv[slot][e] = v ? q : 0;
       c2v[slot][e] = v ? c2 : 0.0f;
     }
@@ -482,9 +484,10 @@ int gemv_launches(int64_t K) { return gemv_chunks(K) > 1 ? 3 : 2; }
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes);
+    cudaError_t e = cudaSuccess;
+    for (auto fn : {gemv_kernel<true, false>, gemv_kernel<false, false>, gemv_kernel<true, true>,
+                    gemv_kernel<false, true>})
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(xa_part_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kXaWarps * kGemvMaxM * kRankPad * 4);
@@ -512,7 +515,12 @@ cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = p.M > 8 ? cudaLaunchKernelEx(&cfg, gemv_kernel<true>, p) : cudaLaunchKernelEx(&cfg, gemv_kernel<false>, p);
+  if (p.scale_format == kScalesFp32)
+    e = p.M > 8 ? cudaLaunchKernelEx(&cfg, gemv_kernel<true, true>, p)
+                : cudaLaunchKernelEx(&cfg, gemv_kernel<false, true>, p);
+  else
+    e = p.M > 8 ? cudaLaunchKernelEx(&cfg, gemv_kernel<true, false>, p)
+                : cudaLaunchKernelEx(&cfg, gemv_kernel<false, false>, p);
   if (e != cudaSuccess || gemv_chunks(p.K) == 1) return e;
   const int64_t pairs = static_cast<int64_t>(p.M) * (p.N / 2);
   const int64_t blocks = (pairs + 255) / 256;

@@ -17,11 +17,17 @@ struct QuantBatchParams {
   int64_t total_chunks;
   int64_t chunk_begin[kMaxQuantBatch + 1];  // prefix sums of chunks per tensor
   int64_t n_blocks[kMaxQuantBatch];
-  const float* W[kMaxQuantBatch];
+  const void* W[kMaxQuantBatch];          // fp32, bf16 or fp16 (in_dtype)
   uint8_t* packed[kMaxQuantBatch];
   int8_t* qscale[kMaxQuantBatch];
   float* c2[kMaxQuantBatch];
   float* mu[kMaxQuantBatch];
+  float* absmax_dst[kMaxQuantBatch];      // where block b of tensor t goes: the tensor's
+                                          // absmax array (fp32 scales) or the workspace
+                                          // slots of its chunks (absmax + chunk_begin[t] * 256)
+  int in_dtype;                           // QLORA_INPUT_*
+  int codebook;                           // QLORA_CODEBOOK_* (one per launch)
+  int scale_format;                       // QLORA_SCALES_* (one per launch)
   // workspace
   float* absmax;        // [total_chunks * 256] first-level scales, slot per chunk
   double* chunk_sum;    // [total_chunks]
@@ -43,7 +49,32 @@ struct WeightView {
   const float* c2;
   const float* mu;
   int64_t rows, cols;
+  int codebook;          // QLORA_CODEBOOK_*
+  int scale_format;      // QLORA_SCALES_*
+  const float* absmax;   // fp32 block scales (QLORA_SCALES_FP32)
 };
+
+// Block scale blk of a weight; mu is *w.mu read once by the caller (0 for
+// fp32 scales).
+__device__ __forceinline__ float weight_block_scale(const WeightView& w, int64_t blk, float mu) {
+  if (w.scale_format == kScalesFp32) return w.absmax[blk];
+  return decode_scale_value(scale_code_value(w.scale_format, w.qscale[blk]), w.c2[blk / kDqBlock], mu);
+}
+
+__device__ __forceinline__ float weight_mu(const WeightView& w) {
+  return w.scale_format == kScalesFp32 ? 0.0f : *w.mu;
+}
+
+// Entry i of a 256-entry table of scale-code values t(q), q = i - 128 the
+// int8 view of the stored code: fp32(q / 127) for int8 codes, the E4M3 value
+// for FP8 codes.  With fp32 scales the table is the int8 one and the kernels
+// decode with q = 127 (t = 1 exactly), c2 = the block absmax and mu = 0, so
+// that fp32(fp32(t c2) + mu) is the absmax itself.
+__device__ __forceinline__ float scale_table_entry(int format, int i) {
+  const int q = i - 128;
+  return format == kScalesDqFp8 ? e4m3_to_float(static_cast<uint32_t>(q) & 0xFFu)
+                                : __fdiv_rn(static_cast<float>(q), 127.0f);
+}
 
 constexpr int kMaxDequantBatch = 128;
 
@@ -56,6 +87,9 @@ struct DequantBatchParams {
   const int8_t* qscale[kMaxDequantBatch];
   const float* c2[kMaxDequantBatch];
   const float* mu[kMaxDequantBatch];
+  const float* absmax[kMaxDequantBatch];   // fp32 scales
+  int codebook[kMaxDequantBatch];          // QLORA_CODEBOOK_*
+  int scale_format[kMaxDequantBatch];      // QLORA_SCALES_*
   void* out[kMaxDequantBatch];
 };
 
@@ -78,8 +112,10 @@ constexpr int kGemvMaxM = 16;
 struct GemvParams {
   const uint8_t* packed;
   const int8_t* qscale;
-  const float* c2;
+  const float* c2;       // fp32 scales: the block absmax array
   const float* mu;
+  int codebook;          // QLORA_CODEBOOK_*
+  int scale_format;      // QLORA_SCALES_*
   int64_t N, K;          // weight [N][K]; N % 8 == 0, K % 64 == 0
   const uint16_t* X;     // [M][K] bf16
   int M;                 // 1 .. 16

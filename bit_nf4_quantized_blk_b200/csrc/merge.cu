@@ -69,8 +69,13 @@ __device__ __forceinline__ void merge_load_tile(MergeTileIn<kSteps>& in, const W
     const int64_t blk = nn * kb + stripe;
     in.code[h][0] = ok ? __ldg(src) : make_uint4(0, 0, 0, 0);
     in.code[h][1] = ok ? __ldg(src + 1) : make_uint4(0, 0, 0, 0);
-    in.q[h] = ok ? static_cast<int>(w.qscale[blk]) : 0;
-    in.c2[h] = ok ? __ldg(w.c2 + (blk >> 8)) : 0.0f;  // 256 scales per chunk
+    if (w.scale_format == kScalesFp32) {  // t = 1, c2 = the absmax (see scale_table_entry)
+      in.q[h] = 127;
+      in.c2[h] = ok ? __ldg(w.absmax + blk) : 0.0f;
+    } else {
+      in.q[h] = ok ? static_cast<int>(w.qscale[blk]) : 0;
+      in.c2[h] = ok ? __ldg(w.c2 + (blk >> 8)) : 0.0f;  // 256 scales per chunk
+    }
     const uint16_t* brow = B + nn * r;
 #pragma unroll
     for (int s = 0; s < kSteps; ++s) {
@@ -91,7 +96,7 @@ __device__ __forceinline__ void mma_16816_zero(float (&d)[4], const uint32_t (&a
 }  // namespace
 
 template <int kSteps, bool kFp32, bool kPair32>
-__global__ void __launch_bounds__(kMergeThreads, kSteps == 1 ? (kFp32 ? 4 : 5) : (kSteps == 2 ? 3 : 2))
+__global__ void __launch_bounds__(kMergeThreads, kSteps == 1 ? 4 : (kSteps == 2 ? 3 : 2))
     merge_kernel(WeightView w, const uint16_t* __restrict__ A, const uint16_t* __restrict__ B, int r, float scale,
                  void* __restrict__ out) {
   // Output staging: 16 rows per warp, padded so that the fragment stores hit
@@ -99,18 +104,18 @@ __global__ void __launch_bounds__(kMergeThreads, kSteps == 1 ? (kFp32 ? 4 : 5) :
   // in half-warp phases).
   constexpr int kPitch = kFp32 ? 288 : 144;
   __shared__ __align__(16) uint8_t s_out[kMergeWarps][16 * kPitch];
-  __shared__ float s_qdiv[256];  // fp32(q / 127) for q = -128 .. 127
+  __shared__ float s_qdiv[256];  // scale-code values t(q), q = -128 .. 127
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  for (int i = threadIdx.x; i < 256; i += kMergeThreads) s_qdiv[i] = __fdiv_rn(static_cast<float>(i - 128), 127.0f);
+  for (int i = threadIdx.x; i < 256; i += kMergeThreads) s_qdiv[i] = scale_table_entry(w.scale_format, i);
   __syncthreads();
   const int64_t N = w.rows, K = w.cols;
   const int stripe = blockIdx.x * kMergeWarps + warp;
   if (stripe >= K / kBlock) return;  // whole warp; no block-wide barrier below
   const int64_t c0 = static_cast<int64_t>(stripe) * kBlock;
-  const float level = nf4_level(lane & 15);
-  const float mu = *w.mu;
+  const float level = codebook_level(w.codebook, lane & 15);
+  const float mu = weight_mu(w);
 
   // MMA B operand: the stripe's A columns, fragment (k = j, n = column).
   uint32_t af[kSteps][8][2];

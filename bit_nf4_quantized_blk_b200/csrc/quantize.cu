@@ -6,7 +6,7 @@
 // path"; "QLoRA Deep Dive: 4-bit NormalFloat & Double Quantization
 // Internals", section "2. Squeezing More Memory: Double Quantization (DQ)".
 //
-// Three kernels per batch of tensors:
+// Three kernels per batch of tensors (the first alone for fp32 scales):
 //
 //  quantize_codes   persistent, one CTA per SM over the chunks of 256 blocks
 //                   (16384 weights).  Each group of 8 lanes owns one 64-weight
@@ -20,13 +20,20 @@
 //  chunk_sums       one warp per chunk: the fp64 sum of its 256 block scales;
 //                   the last warp of each tensor forms the tensor's mean offset.
 //  dq_chunks        one warp per chunk: d = a - mu, c2 = max|d|,
-//                   q = rint(fp32(fp32(d / c2) * 127)) (0 where c2 == 0).
+//                   q = rint(fp32(fp32(d / c2) * 127)) (int8 codes) or the
+//                   E4M3 code of fp32(d / c2) (FP8 codes); 0 where c2 == 0.
+//
+// Variants: fp32, bf16 or fp16 input weights (16-bit ones widen exactly to
+// fp32 on load); the NF4 or FP4 codebook ("FT-02: QLoRA -- Fine-Tuning with
+// Quantization", "Exercise 3: NF4 vs FP4 at equal memory").
 //
 // The mean is defined as a strictly sequential fp64 sum (inside each chunk,
 // then over chunk sums).  When the exponents of the summed values span few
 // enough binades every partial sum is exact in fp64, so a tree reduction
 // gives the same bits; the kernels check that bound and fall back to a
 // sequential loop when it does not hold.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -89,10 +96,31 @@ constexpr int kQThreads = kQWarps * 32;
 
 // Per decision cell, one 16-byte entry per lane (conflict-free): the band
 // [lo, hi] = 64 T (1 -+ 2^-19) around the cell's threshold T, 64 T itself and
-// the cell's base code; lo = hi = thr = 256 (never reached) in a cell without
-// a threshold.
-constexpr int kCellEntries = 129 * 32;
+// the cell's base position; lo = hi = thr = 256 (never reached) in a cell
+// without a threshold.
+constexpr int kCellEntries = kDecisionCells * 32;
 constexpr int kQuantSmemBytes = kCellEntries * 16;
+
+// 8 consecutive 16-bit weights with one 128-bit streaming load, widened to
+// fp32 exactly (bf16: the bits are the top half of the fp32; fp16: IEEE
+// half to single conversion).
+template <int kIn>
+__device__ __forceinline__ void ld_stream_16bit_v8(const uint16_t* p, float (&v)[8]) {
+  uint32_t u[4];
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+               : "l"(p));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (kIn == QLORA_INPUT_BF16) {
+      v[2 * i] = __uint_as_float(u[i] << 16);
+      v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    } else {
+      v[2 * i] = __half2float(__ushort_as_half(static_cast<unsigned short>(u[i] & 0xFFFFu)));
+      v[2 * i + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(u[i] >> 16)));
+    }
+  }
+}
 
 __device__ __forceinline__ void chunk_bounds(const QuantBatchParams& p, int64_t g, int& t, int64_t& blk0, int& nblk) {
   t = find_tensor(p, g);
@@ -122,16 +150,22 @@ __device__ __forceinline__ ChunkInfo next_chunk_info(const QuantBatchParams& p, 
 }
 
 // Weights 8l .. 8l+7 of blocks grp, grp + 64, grp + 128, grp + 192 of a
-// chunk (zeros past the tensor or the batch), with 256-bit streaming loads.
+// chunk (zeros past the tensor or the batch), with 256-bit (fp32) or 128-bit
+// (16-bit inputs) streaming loads.
+template <int kIn>
 __device__ __forceinline__ void load_chunk(const QuantBatchParams& p, const ChunkInfo& ci, int grp, int l,
                                            float (&v)[4][8]) {
   const int t = ci.t, nblk = ci.nblk;
   const int64_t blk0 = ci.blk0;
-  const float* src = p.W[t] + (blk0 + grp) * kBlock + l * 8;
+  using In = std::conditional_t<kIn == QLORA_INPUT_FP32, float, uint16_t>;
+  const In* src = static_cast<const In*>(p.W[t]) + (blk0 + grp) * kBlock + l * 8;
 #pragma unroll
   for (int rep = 0; rep < 4; ++rep) {
     if (rep * 64 + grp < nblk) {
-      ld_stream_v8(src + rep * 64 * kBlock, v[rep]);
+      if constexpr (kIn == QLORA_INPUT_FP32)
+        ld_stream_v8(src + rep * 64 * kBlock, v[rep]);
+      else
+        ld_stream_16bit_v8<kIn>(src + rep * 64 * kBlock, v[rep]);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[rep][i] = 0.0f;
@@ -152,8 +186,14 @@ __device__ __forceinline__ void load_chunk(const QuantBatchParams& p, const Chun
 // its 8 weights from the IEEE quotient (so does a block whose 64/a is not a
 // normal fp32).  Every threshold is > 2^-14 (relative) from its cell's edges
 // (checked on the host), so no other threshold can be that close.
+//
+// kFp4: the FP4 codebook's table uses floor cells (c = floor(64 x) + 65) and
+// yields positions among its 15 distinct levels; fp4_codes_of maps each
+// word of positions to codes.  NF4: trunc cells (c = trunc(64 x) + 64),
+// positions are the codes.
+template <int kIn, bool kFp4>
 __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __grid_constant__ QuantBatchParams p) {
-  extern __shared__ uint4 s_cell[];  // [129 cells][32 lanes]
+  extern __shared__ uint4 s_cell[];  // [kDecisionCells cells][32 lanes]
   const int tid = threadIdx.x, lane = tid & 31;
   const int grp = tid >> 3;  // 64 groups of 8 lanes
   const int l = tid & 7;     // lane in group: weights 8l .. 8l+7 of the block
@@ -161,7 +201,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
   float cur[4][8], nxt[4][8];
   int t_cursor = 0;
   ChunkInfo cur_ci = next_chunk_info(p, blockIdx.x, t_cursor);
-  load_chunk(p, cur_ci, grp, l, cur);
+  load_chunk<kIn>(p, cur_ci, grp, l, cur);
 
   for (int i = tid; i < kCellEntries; i += kQThreads) {
     const int c = i >> 5;
@@ -178,11 +218,15 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
   }
   __syncthreads();
 
-  const uint32_t cell_addr0 = smem_u32(&s_cell[64 * 32 + lane]);  // cell 64 <-> x64 in (-1, 1)
+  // NF4: cell 64 <-> trunc(x64) = 0; FP4: cell 65 <-> floor(x64) = 0.
+  const uint32_t cell_addr0 = smem_u32(&s_cell[(kFp4 ? 65 : 64) * 32 + lane]);
+  auto cell_of = [](float x64) {
+    return static_cast<uint32_t>(kFp4 ? __float2int_rd(x64) : __float2int_rz(x64)) * 512u;
+  };
   float nonfinite = 0.0f;  // becomes NaN if any input is NaN or +-Inf
   for (int64_t g = blockIdx.x; g < p.total_chunks; g += gridDim.x) {
     const ChunkInfo nxt_ci = next_chunk_info(p, g + gridDim.x, t_cursor);
-    load_chunk(p, nxt_ci, grp, l, nxt);
+    load_chunk<kIn>(p, nxt_ci, grp, l, nxt);
     const int t = cur_ci.t, nblk = cur_ci.nblk;
     const int64_t blk0 = cur_ci.blk0;
     uint32_t* __restrict__ packed = reinterpret_cast<uint32_t*>(p.packed[t]);
@@ -207,7 +251,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
 #pragma unroll
       for (int i = 7; i >= 0; --i) {
         const float x64 = __fmul_rn(v[i], rcp64);
-        const uint4 e = ld_shared_u4(cell_addr0 + static_cast<uint32_t>(__float2int_rz(x64)) * 512u);
+        const uint4 e = ld_shared_u4(cell_addr0 + cell_of(x64));
         const bool above_lo = x64 >= __uint_as_float(e.x);
         const bool above_hi = x64 > __uint_as_float(e.y);
         word = word * 16u + e.w + (above_lo ? 1u : 0u);
@@ -220,14 +264,15 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
 #pragma unroll
           for (int i = 7; i >= 0; --i) {
             const float x64 = __fdiv_rn(v[i], div) * 64.0f;  // exact scaling
-            const uint4 e = ld_shared_u4(cell_addr0 + static_cast<uint32_t>(__float2int_rz(x64)) * 512u);
+            const uint4 e = ld_shared_u4(cell_addr0 + cell_of(x64));
             word = word * 16u + e.w + (x64 >= __uint_as_float(e.z) ? 1u : 0u);
           }
         }
       }
+      if constexpr (kFp4) word = fp4_codes_of(word);
       if (b < nblk) {
         packed[(blk0 + b) * (kBlock / 8) + l] = word;
-        if (l == 0) p.absmax[g * kDqBlock + b] = m;
+        if (l == 0) p.absmax_dst[t][blk0 + b] = m;
       }
     }
 #pragma unroll
@@ -355,12 +400,32 @@ __global__ void __launch_bounds__(256) dq_chunks_kernel(const __grid_constant__ 
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   const float c2 = m;
 
+  uint32_t bytes[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) bytes[i] = 0;
+  if (c2 != 0.0f) {
+    if (p.scale_format == kScalesDqFp8) {
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        // E4M3 pair, round to nearest even (|d / c2| <= 1: no saturation);
+        // the first source operand goes to the upper byte.
+        uint16_t pair;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(pair)
+            : "f"(__fdiv_rn(d[i + 1], c2)), "f"(__fdiv_rn(d[i], c2)));
+        bytes[i] = pair & 0xFFu;
+        bytes[i + 1] = pair >> 8;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        bytes[i] = static_cast<uint32_t>(static_cast<int>(rintf(__fmul_rn(__fdiv_rn(d[i], c2), 127.0f)))) & 0xFFu;
+    }
+  }
   uint32_t lo = 0, hi = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    int q = 0;
-    if (c2 != 0.0f) q = static_cast<int>(rintf(__fmul_rn(__fdiv_rn(d[i], c2), 127.0f)));
-    const uint32_t byte = static_cast<uint32_t>(q) & 0xFFu;
+    const uint32_t byte = bytes[i];
     if (i < 4) lo |= byte << (8 * i); else hi |= byte << (8 * (i - 4));
   }
   int8_t* qs = p.qscale[t] + local_chunk * kDqBlock + lane * 8;
@@ -374,6 +439,29 @@ __global__ void __launch_bounds__(256) dq_chunks_kernel(const __grid_constant__ 
   if (lane == 0) p.c2[t][local_chunk] = c2;
 }
 
+namespace {
+
+template <int kIn, bool kFp4>
+cudaError_t launch_codes(const QuantBatchParams& p, unsigned grid, cudaStream_t stream) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(quantize_codes_kernel<kIn, kFp4>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  quantize_codes_kernel<kIn, kFp4><<<grid, kQThreads, kQuantSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int kIn>
+cudaError_t launch_codes_for(const QuantBatchParams& p, unsigned grid, cudaStream_t stream) {
+  return p.codebook == QLORA_CODEBOOK_FP4 ? launch_codes<kIn, true>(p, grid, stream)
+                                          : launch_codes<kIn, false>(p, grid, stream);
+}
+
+}  // namespace
+
 cudaError_t launch_quantize_batch(const QuantBatchParams& p, cudaStream_t stream) {
   if (p.total_chunks <= 0) return cudaSuccess;
   static int sms = 0;
@@ -382,14 +470,13 @@ cudaError_t launch_quantize_batch(const QuantBatchParams& p, cudaStream_t stream
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
-    cudaError_t e = cudaFuncSetAttribute(quantize_codes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kQuantSmemBytes);
-    if (e != cudaSuccess) return e;
   }
   const unsigned grid = static_cast<unsigned>(p.total_chunks < sms ? p.total_chunks : sms);
-  quantize_codes_kernel<<<grid, kQThreads, kQuantSmemBytes, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = p.in_dtype == QLORA_INPUT_BF16   ? launch_codes_for<QLORA_INPUT_BF16>(p, grid, stream)
+                  : p.in_dtype == QLORA_INPUT_FP16 ? launch_codes_for<QLORA_INPUT_FP16>(p, grid, stream)
+                                                   : launch_codes_for<QLORA_INPUT_FP32>(p, grid, stream);
   if (e != cudaSuccess) return e;
+  if (p.scale_format == kScalesFp32) return cudaSuccess;  // no double quantization
   const unsigned warps_grid = static_cast<unsigned>((p.total_chunks + 7) / 8);
   chunk_sums_kernel<<<warps_grid, 256, 0, stream>>>(p);
   e = cudaGetLastError();

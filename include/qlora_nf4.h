@@ -65,18 +65,63 @@ typedef enum qlora_status {
 } qlora_status;
 
 /*
+ * 4-bit codebooks.
+ *   NF4: the 16 NormalFloat levels, ascending with the code ("QLoRA: NF4
+ *        storage, gradients and local integration", section "Exact CPU
+ *        teaching quantizer and adapter gradient path").
+ *   FP4: the E2M1 grid of "FT-02: QLoRA -- Fine-Tuning with Quantization",
+ *        section "Exercise 3: NF4 vs FP4 at equal memory": code bit 3 is the
+ *        sign, bits 2..0 select the magnitude k/12, k = 0, 1/16, 2, 3, 4, 6,
+ *        8, 12 (fp32-rounded).  Quantization never emits code 8 (-0).
+ * Both quantize to the nearest level (fp32 distances), the lowest code on a
+ * tie.
+ */
+typedef enum qlora_codebook { QLORA_CODEBOOK_NF4 = 0, QLORA_CODEBOOK_FP4 = 1 } qlora_codebook;
+
+/*
+ * Storage of the per-block scales.
+ *   DQ_INT8 : double quantization, int8 codes q in [-127, 127] per block,
+ *             t = fp32(q / 127) (4.127 bits per weight in all).
+ *   DQ_FP8  : double quantization, E4M3 codes per block (stored in the same
+ *             int8 array as bit patterns), q = E4M3(fp32(d / c2)) rounded to
+ *             nearest even, t = the E4M3 value ("QLoRA Deep Dive: 4-bit
+ *             NormalFloat & Double Quantization Internals", section "2.
+ *             Squeezing More Memory: Double Quantization (DQ)": normalize by
+ *             the chunk absmax, quantize to 8-bit floats).
+ *   FP32    : no double quantization, the fp32 block absmax itself (4.5 bits
+ *             per weight; same page, "Memory Savings Analysis").
+ * Double-quantized scales decode as a = fp32(fp32(t * c2) + mu).
+ */
+typedef enum qlora_scale_format {
+  QLORA_SCALES_DQ_INT8 = 0,
+  QLORA_SCALES_DQ_FP8 = 1,
+  QLORA_SCALES_FP32 = 2
+} qlora_scale_format;
+
+/* Element type of the dense weight given to the quantizer. */
+typedef enum qlora_input_dtype { QLORA_INPUT_FP32 = 0, QLORA_INPUT_BF16 = 1, QLORA_INPUT_FP16 = 2 } qlora_input_dtype;
+
+/*
  * One quantized tensor.  The struct itself lives in host memory; its pointers
  * are device memory owned by the caller.
- *   rows, cols : W0 is [rows, cols] row-major (rows = d_out, cols = d_in);
- *                cols must be a multiple of 64 so every block lies in one row.
- *   packed     : rows*cols/2 bytes; byte i holds code 2i (low nibble) and
- *                code 2i+1 (high nibble).
- *   qscale     : rows*cols/64 int8 scale codes in [-127, 127], one per block.
- *   c2         : ceil(rows*cols/16384) fp32 second-level scales, one per chunk
- *                of 256 consecutive blocks.
- *   mu         : one fp32, the per-tensor mean of the block absmax values.
- * The block scale is decoded as a = fp32(fp32(fp32(q/127)*c2) + mu) and the
- * weight as fp32(L[code] * a) (bf16 outputs round that to nearest even).
+ *   rows, cols   : W0 is [rows, cols] row-major (rows = d_out, cols = d_in);
+ *                  cols must be a multiple of 64 so every block lies in one row.
+ *   packed       : rows*cols/2 bytes; byte i holds code 2i (low nibble) and
+ *                  code 2i+1 (high nibble).
+ *   qscale       : rows*cols/64 scale codes, one per block (DQ formats):
+ *                  int8 in [-127, 127] (DQ_INT8) or E4M3 bit patterns (DQ_FP8).
+ *   c2           : ceil(rows*cols/16384) fp32 second-level scales, one per
+ *                  chunk of 256 consecutive blocks (DQ formats).
+ *   mu           : one fp32, the per-tensor mean of the block absmax values
+ *                  (DQ formats).
+ *   codebook     : qlora_codebook (0 = NF4).
+ *   scale_format : qlora_scale_format (0 = DQ_INT8).
+ *   absmax       : rows*cols/64 fp32 block scales (FP32 format only; 16-byte
+ *                  aligned).  qscale, c2 and mu are unused (may be NULL) with
+ *                  FP32 scales; absmax is unused (may be NULL) otherwise.
+ * The weight decodes as fp32(L[code] * a), a the block scale (bf16 outputs
+ * round that to nearest even).  A zero-initialized codebook / scale_format /
+ * absmax is the NF4 double-quantized (int8) format.
  */
 typedef struct qlora_nf4_weight {
   int64_t rows;
@@ -85,6 +130,9 @@ typedef struct qlora_nf4_weight {
   int8_t *qscale;
   float *c2;
   float *mu;
+  int32_t codebook;
+  int32_t scale_format;
+  float *absmax;
 } qlora_nf4_weight;
 
 /* Human-readable name of a status code (static string). */
@@ -93,6 +141,7 @@ const char *qlora_status_string(qlora_status status);
 /*
  * Sizes of the quantized state of a [rows, cols] tensor and the workspace
  * qlora_nf4_quantize needs for it.  Any output pointer may be NULL.
+ * n_blocks is also the length of the fp32 absmax array of QLORA_SCALES_FP32.
  * Errors: INVALID_ARG if rows < 1, cols < 64 or cols % 64 != 0.
  */
 qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, size_t *packed_bytes, size_t *n_blocks,
@@ -100,8 +149,9 @@ qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, size_t *packed_bytes, s
 
 /*
  * Quantize + double-quantize one fp32 tensor W [out->rows, out->cols]
- * (steps: block absmax, normalisation, nearest NF4 level, packing, mean
- * offset, second-level absmax per 256-block chunk, int8 scale codes).
+ * (steps: block absmax, normalisation, nearest level of out->codebook,
+ * packing; then, by out->scale_format, mean offset, second-level absmax per
+ * 256-block chunk and int8 or E4M3 scale codes, or the fp32 absmax alone).
  * Results are bit-identical to the definition: fp32 IEEE division and
  * comparisons, fp64 strictly sequential mean (per chunk, then over chunks).
  *   W        : device fp32 input, not modified.
@@ -127,6 +177,24 @@ qlora_status qlora_nf4_quantize(const float *W, const qlora_nf4_weight *out, voi
 size_t qlora_nf4_quantize_batched_ws_bytes(const qlora_nf4_weight *outs, int32_t count);
 qlora_status qlora_nf4_quantize_batched(const float *const *W, const qlora_nf4_weight *outs, int32_t count,
                                         void *ws, size_t ws_bytes, int32_t *d_status, void *stream);
+
+/*
+ * Quantize dense weights given as fp32, bf16 or fp16 (qlora_input_dtype;
+ * "FT-02: QLoRA -- Fine-Tuning with Quantization", section "3.
+ * BitsAndBytesConfig in practice": checkpoints are 16-bit and are converted
+ * at load time).  16-bit weights are widened to fp32 exactly and then
+ * quantized as fp32 weights, so the result equals qlora_nf4_quantize of the
+ * widened tensor.  Pointers, workspace and status as qlora_nf4_quantize /
+ * qlora_nf4_quantize_batched; W is 32-byte aligned for fp32 and 16-byte
+ * aligned for bf16 / fp16.  The codebook and scale format of the outputs
+ * select the stored format; one call takes one format (every output of a
+ * batch has the same codebook and scale_format, else QLORA_ERR_INVALID_ARG).
+ */
+qlora_status qlora_nf4_quantize_ex(const void *W, int32_t in_dtype, const qlora_nf4_weight *out, void *ws,
+                                   size_t ws_bytes, int32_t *d_status, void *stream);
+qlora_status qlora_nf4_quantize_batched_ex(const void *const *W, int32_t in_dtype, const qlora_nf4_weight *outs,
+                                           int32_t count, void *ws, size_t ws_bytes, int32_t *d_status,
+                                           void *stream);
 
 /*
  * Quantize + double-quantize one tensor exactly as qlora_nf4_quantize does,

@@ -48,23 +48,33 @@ def f32_bits(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a, dtype=np.float32)).view(np.uint32)
 
 
-def gpu_quantize(W: torch.Tensor) -> binding.NF4Weight:
-    """Quantize one fp32 tensor on the GPU through the C ABI (status read back)."""
+def gpu_quantize(W: torch.Tensor, codebook: int = 0, scale_format: int = 0) -> binding.NF4Weight:
+    """Quantize one fp32, bf16 or fp16 tensor on the GPU through the C ABI
+    (status read back)."""
     rows, cols = W.shape
-    Wd = W.to("cuda", torch.float32).contiguous()
-    out = binding.NF4Weight.empty(rows, cols)
+    Wd = W.to("cuda").contiguous()
+    out = binding.NF4Weight.empty(rows, cols, codebook=codebook, scale_format=scale_format)
     ws = torch.empty(binding.qlora_nf4_sizes(rows, cols)["ws_bytes"], dtype=torch.uint8, device="cuda")
-    binding.qlora_nf4_quantize(Wd, out, ws)
+    if Wd.dtype == torch.float32 and codebook == 0 and scale_format == 0:
+        binding.qlora_nf4_quantize(Wd, out, ws)
+    else:
+        binding.qlora_nf4_quantize_ex(Wd, out, ws)
     return out
 
 
 def assert_state_equal(out: binding.NF4Weight, st, what=""):
-    """Bit-exact comparison of the GPU state with the oracle's NF4DQState."""
+    """Bit-exact comparison of the GPU state with the oracle's NF4DQState
+    (any codebook / scale format)."""
     torch.cuda.synchronize()
     packed = out.packed.cpu().numpy()
     assert np.array_equal(packed, st.packed), f"{what}: packed codes differ at {np.flatnonzero(packed != st.packed)[:8]}"
-    q = out.qscale.cpu().numpy()
-    assert np.array_equal(q, st.qscale), f"{what}: scale codes differ at {np.flatnonzero(q != st.qscale)[:8]}"
+    if st.scale_format == "fp32":
+        a = f32_bits(out.absmax.cpu().numpy())
+        assert np.array_equal(a, f32_bits(st.absmax)), f"{what}: absmax differs at {np.flatnonzero(a != f32_bits(st.absmax))[:8]}"
+        return
+    q = out.qscale.cpu().numpy().view(np.uint8)
+    sq = np.asarray(st.qscale).view(np.uint8)
+    assert np.array_equal(q, sq), f"{what}: scale codes differ at {np.flatnonzero(q != sq)[:8]}"
     assert np.array_equal(f32_bits(out.c2.cpu().numpy()), f32_bits(st.c2)), f"{what}: c2 differs"
     assert f32_bits(out.mu.cpu().numpy())[0] == f32_bits([st.mu])[0], f"{what}: mu {out.mu.item()} != {st.mu}"
 
