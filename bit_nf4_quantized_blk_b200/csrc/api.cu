@@ -495,8 +495,7 @@ extern "C" qlora_status qlora_nf4_quantize_batched_ex(const void* const* W, int3
     p.codebook = outs[0].codebook;
     p.scale_format = outs[0].scale_format;
     p.absmax = at<float>(ws, lay.absmax);
-    for (int i = 0; i < n; ++i)
-      p.absmax_dst[i] = p.scale_format == kScalesFp32 ? outs[g0 + i].absmax : p.absmax + p.chunk_begin[i] * kDqBlock;
+    for (int i = 0; i < n; ++i) p.absmax_out[i] = outs[g0 + i].absmax;
     p.chunk_sum = at<double>(ws, lay.sums);
     p.chunk_exp = at<int>(ws, lay.exps);
     p.counters = at<unsigned>(ws, lay.counters);
@@ -931,7 +930,7 @@ extern "C" qlora_status qlora_nf4_quantize_noalloc(const float* W, const qlora_n
   p.codebook = out->codebook;
   p.scale_format = out->scale_format;
   p.absmax = at<float>(scratch, kNoAllocLayout.absmax);
-  p.absmax_dst[0] = p.scale_format == kScalesFp32 ? out->absmax : p.absmax;
+  p.absmax_out[0] = out->absmax;
   p.chunk_sum = at<double>(scratch, kNoAllocLayout.sums);
   p.chunk_exp = at<int>(scratch, kNoAllocLayout.exps);
   p.counters = at<unsigned>(scratch, kNoAllocLayout.counters);

@@ -41,17 +41,20 @@ __device__ __forceinline__ int find_tensor_seg(const DequantBatchParams& p, int6
 // lookup by shuffle: lane l holds L[l % 16], and a shuffle reads its source
 // lane modulo 32, so `word >> 4i` selects L[nibble i] with no masking and no
 // shared-memory table.
-template <bool kFp32>
+//
+// kAnyFormat = false: every tensor of the batch is NF4 with int8 scale codes
+// (the default format), decoded without the per-tensor format dispatch.
+template <bool kFp32, bool kAnyFormat>
 __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ DequantBatchParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t gseg = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (gseg >= p.total_seg) return;
   const int t = find_tensor_seg(p, gseg);
-  const float level = codebook_level(p.codebook[t], lane & 15);
+  const float level = kAnyFormat ? codebook_level(p.codebook[t], lane & 15) : nf4_level(lane & 15);
   const int64_t seg = gseg - p.begin_seg[t];
   const int64_t n_units = p.n_units[t];
   const uint4* __restrict__ packed = reinterpret_cast<const uint4*>(p.packed[t]);
-  const int fmt = p.scale_format[t];
+  const int fmt = kAnyFormat ? p.scale_format[t] : kScalesDqInt8;
   const float mu = fmt == kScalesFp32 ? 0.0f : *p.mu[t];
   uint4 pk[4];
   float a[4];
@@ -64,7 +67,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
   }
   // Scales of the four units (two units per 64-weight block); one uniform
   // branch on the format, the loads of each branch issued together.
-  if (fmt == kScalesFp32) {
+  if (kAnyFormat && fmt == kScalesFp32) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int64_t u = seg * 128 + lane + 32 * q;
@@ -86,7 +89,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int64_t u = seg * 128 + lane + 32 * q;
-      if (u < n_units) a[q] = decode_scale_value(scale_code_value(fmt, static_cast<int8_t>(qv[q])), c2v[q], mu);
+      if (u < n_units)
+        a[q] = kAnyFormat ? decode_scale_value(scale_code_value(fmt, static_cast<int8_t>(qv[q])), c2v[q], mu)
+                          : decode_scale(qv[q], c2v[q], mu);
     }
   }
   // Every lane takes part in the shuffles; units past the end are skipped
@@ -175,10 +180,16 @@ __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, u
 cudaError_t launch_dequant_batch(const DequantBatchParams& p, int out_fp32, cudaStream_t stream) {
   if (p.total_seg <= 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((p.total_seg + 7) / 8);  // 8 warps per CTA
-  if (out_fp32)
-    dequant_kernel<true><<<grid, 256, 0, stream>>>(p);
-  else
-    dequant_kernel<false><<<grid, 256, 0, stream>>>(p);
+  bool any_format = false;
+  for (int i = 0; i < p.count; ++i)
+    any_format |= p.codebook[i] != QLORA_CODEBOOK_NF4 || p.scale_format[i] != kScalesDqInt8;
+  if (out_fp32) {
+    if (any_format) dequant_kernel<true, true><<<grid, 256, 0, stream>>>(p);
+    else dequant_kernel<true, false><<<grid, 256, 0, stream>>>(p);
+  } else {
+    if (any_format) dequant_kernel<false, true><<<grid, 256, 0, stream>>>(p);
+    else dequant_kernel<false, false><<<grid, 256, 0, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 

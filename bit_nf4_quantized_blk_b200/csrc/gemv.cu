@@ -231,26 +231,39 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
 
   // This warp's slice of item i: rows tile*16 .. +16, blocks c*64 + 4*warp
   // .. +4, eight 16-byte pieces per row (zero-filled past N, past K or past
-  // the last item); one commit group per item and thread.
-  GvCursor ic{0, t0};
-  int issued = 0;
+  // the last item); one commit group per item and thread.  Lane piece h is
+  // row (lane >> 3) + 4h, 16-byte column lane & 7 of the slice, so the
+  // source is one running pointer plus fixed strides: it advances by one
+  // tile per item and, after the CTA's last tile, to the next 4096-wide chunk
+  // of K.
+  const int ntile = t1 - t0;
+  const int64_t tile_bytes = static_cast<int64_t>(kGvRows) * (K / 2);
+  const int64_t rows4_bytes = 4 * (K / 2);
+  const int prow = lane >> 3, pcol = lane & 7;
+  const uint8_t* isrc = p.packed + static_cast<int64_t>(t0) * tile_bytes + warp * (kGvWarpBlocks * kBlock / 2) +
+                        prow * (K / 2) + pcol * 16;
+  const uint32_t slot_lane = static_cast<uint32_t>(prow * kGvSlicePitch + pcol * 16);
+  int i_tile = 0, i_chunk = 0, issued = 0;
   auto issue_next = [&]() {
     const bool live = issued < items;
-    const int64_t blkw = static_cast<int64_t>(ic.c) * kGvUnitBlocks + kGvWarpBlocks * warp;
-    const int64_t rem = nbk - blkw;
-    const int nbw = !live || rem <= 0 ? 0 : (rem < kGvWarpBlocks ? static_cast<int>(rem) : kGvWarpBlocks);
-    const int64_t row0 = static_cast<int64_t>(ic.tile) * kGvRows;
-    const int64_t rows_left = N - row0;
-    const int rows_valid = rows_left < kGvRows ? static_cast<int>(rows_left) : kGvRows;
-    uint8_t* slot = ring + (issued & (kGvDepth - 1)) * kGvSliceBytes;
-    const uint8_t* src = p.packed + row0 * (K / 2) + blkw * (kBlock / 2);
+    const int rows_left = static_cast<int>(N - static_cast<int64_t>(t0 + i_tile) * kGvRows);
+    const int rem = static_cast<int>(nbk - i_chunk * kGvUnitBlocks) - kGvWarpBlocks * warp;
+    const bool col_ok = live && pcol < 2 * rem;
+    uint8_t* slot = ring + (issued & (kGvDepth - 1)) * kGvSliceBytes + slot_lane;
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      const int pc = lane + 32 * h, row = pc >> 3, col = pc & 7;
-      const bool v = col < 2 * nbw && row < rows_valid;
-      cp_async_16(slot + row * kGvSlicePitch + col * 16, v ? src + row * (K / 2) + col * 16 : p.packed, v);
+      const bool v = col_ok && prow + 4 * h < rows_left;
+      cp_async_16(slot + h * 4 * kGvSlicePitch, v ? isrc + h * rows4_bytes : p.packed, v);
     }
-    if (live) ic.next(t0, t1);
+    if (live) {
+      if (++i_tile == ntile) {
+        i_tile = 0;
+        ++i_chunk;
+        isrc += kGvUnitBlocks * kBlock / 2 - static_cast<int64_t>(ntile - 1) * tile_bytes;
+      } else {
+        isrc += tile_bytes;
+      }
+    }
     ++issued;
     cp_async_commit();
   };
@@ -270,19 +283,21 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
   const uint32_t lane_base = kLutWindow | (static_cast<uint32_t>(lane) * 4);
   // Scales this lane decodes per item: row lane%16 of the tile, blocks
   // 4 warp + lane/16 and 4 warp + lane/16 + 2; the lanes holding rows g and
-  // g+8 hand them over by shuffle.
-  GvCursor fc{0, t0};
-  int fetched = 0;
+  // g+8 hand them over by shuffle.  The block index runs like the copy
+  // source: + 16 nbk per tile, to the next chunk after the last tile.
+  const int frow = lane & 15, fblk = kGvWarpBlocks * warp + (lane >> 4);
+  int64_t fgb = (static_cast<int64_t>(t0) * kGvRows + frow) * nbk + fblk;
+  int f_tile = 0, f_chunk = 0, fetched = 0;
   int qv[kGvDepth][2];
   float c2v[kGvDepth][2];
   auto fetch = [&](int slot) {
     const bool live = fetched < items;
-    const int64_t row = static_cast<int64_t>(fc.tile) * kGvRows + (lane & 15);
-    const int64_t blk = static_cast<int64_t>(fc.c) * kGvUnitBlocks + kGvWarpBlocks * warp + (lane >> 4);
+    const bool row_ok = live && static_cast<int64_t>(t0 + f_tile) * kGvRows + frow < N;
+    const int blk = f_chunk * kGvUnitBlocks + fblk;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const bool v = live && row < N && blk + 2 * e < nbk;
-      const int64_t gb = v ? row * nbk + blk + 2 * e : 0;
+      const bool v = row_ok && blk + 2 * e < nbk;
+      const int64_t gb = v ? fgb + 2 * e : 0;
       // fp32 scales: t(127) = 1, "c2" is the block's absmax and mu = 0, so
       // the decode below returns the absmax itself.
       const int q = kScales32 ? 127 : p.qscale[gb];
@@ -290,7 +305,15 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
       qv[slot][e] = v ? q : 0;
       c2v[slot][e] = v ? c2 : 0.0f;
     }
-    if (live) fc.next(t0, t1);
+    if (live) {
+      if (++f_tile == ntile) {
+        f_tile = 0;
+        ++f_chunk;
+        fgb += kGvUnitBlocks - static_cast<int64_t>(ntile - 1) * kGvRows * nbk;
+      } else {
+        fgb += kGvRows * nbk;
+      }
+    }
     ++fetched;
   };
 #pragma unroll

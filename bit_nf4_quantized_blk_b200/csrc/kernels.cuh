@@ -22,9 +22,7 @@ struct QuantBatchParams {
   int8_t* qscale[kMaxQuantBatch];
   float* c2[kMaxQuantBatch];
   float* mu[kMaxQuantBatch];
-  float* absmax_dst[kMaxQuantBatch];      // where block b of tensor t goes: the tensor's
-                                          // absmax array (fp32 scales) or the workspace
-                                          // slots of its chunks (absmax + chunk_begin[t] * 256)
+  float* absmax_out[kMaxQuantBatch];      // fp32 scales: the tensor's block absmax array
   int in_dtype;                           // QLORA_INPUT_*
   int codebook;                           // QLORA_CODEBOOK_* (one per launch)
   int scale_format;                       // QLORA_SCALES_* (one per launch)

@@ -190,8 +190,10 @@ __device__ __forceinline__ void load_chunk(const QuantBatchParams& p, const Chun
 // kFp4: the FP4 codebook's table uses floor cells (c = floor(64 x) + 65) and
 // yields positions among its 15 distinct levels; fp4_codes_of maps each
 // word of positions to codes.  NF4: trunc cells (c = trunc(64 x) + 64),
-// positions are the codes.
-template <int kIn, bool kFp4>
+// positions are the codes.  kScales32: the block absmax goes to the tensor's
+// fp32 scale array (no double quantization), else to the chunk's workspace
+// slots.
+template <int kIn, bool kFp4, bool kScales32>
 __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __grid_constant__ QuantBatchParams p) {
   extern __shared__ uint4 s_cell[];  // [kDecisionCells cells][32 lanes]
   const int tid = threadIdx.x, lane = tid & 31;
@@ -272,7 +274,12 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_codes_kernel(const __gr
       if constexpr (kFp4) word = fp4_codes_of(word);
       if (b < nblk) {
         packed[(blk0 + b) * (kBlock / 8) + l] = word;
-        if (l == 0) p.absmax_dst[t][blk0 + b] = m;
+        if (l == 0) {
+          if constexpr (kScales32)
+            p.absmax_out[t][blk0 + b] = m;
+          else
+            p.absmax[g * kDqBlock + b] = m;
+        }
       }
     }
 #pragma unroll
@@ -441,23 +448,29 @@ __global__ void __launch_bounds__(256) dq_chunks_kernel(const __grid_constant__ 
 
 namespace {
 
-template <int kIn, bool kFp4>
+template <int kIn, bool kFp4, bool kScales32>
 cudaError_t launch_codes(const QuantBatchParams& p, unsigned grid, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(quantize_codes_kernel<kIn, kFp4>,
+    cudaError_t e = cudaFuncSetAttribute(quantize_codes_kernel<kIn, kFp4, kScales32>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  quantize_codes_kernel<kIn, kFp4><<<grid, kQThreads, kQuantSmemBytes, stream>>>(p);
+  quantize_codes_kernel<kIn, kFp4, kScales32><<<grid, kQThreads, kQuantSmemBytes, stream>>>(p);
   return cudaGetLastError();
+}
+
+template <int kIn, bool kFp4>
+cudaError_t launch_codes_scales(const QuantBatchParams& p, unsigned grid, cudaStream_t stream) {
+  return p.scale_format == kScalesFp32 ? launch_codes<kIn, kFp4, true>(p, grid, stream)
+                                       : launch_codes<kIn, kFp4, false>(p, grid, stream);
 }
 
 template <int kIn>
 cudaError_t launch_codes_for(const QuantBatchParams& p, unsigned grid, cudaStream_t stream) {
-  return p.codebook == QLORA_CODEBOOK_FP4 ? launch_codes<kIn, true>(p, grid, stream)
-                                          : launch_codes<kIn, false>(p, grid, stream);
+  return p.codebook == QLORA_CODEBOOK_FP4 ? launch_codes_scales<kIn, true>(p, grid, stream)
+                                          : launch_codes_scales<kIn, false>(p, grid, stream);
 }
 
 }  // namespace
