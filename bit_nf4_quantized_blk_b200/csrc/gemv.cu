@@ -91,6 +91,17 @@ __device__ __forceinline__ uint32_t lut_pair(uint32_t word, uint32_t lane_base) 
   return v;
 }
 
+// 16-byte copy global -> shared (32-bit shared address), no predicate.
+__device__ __forceinline__ void cp_async_16_full(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
 // 16 consecutive bf16 of row `row` starting at element k (zeros if !valid).
 __device__ __forceinline__ void load16(const uint16_t* base, int64_t ld, int row, int64_t k, bool valid,
                                        uint32_t (&w)[8]) {
@@ -243,17 +254,30 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
   const uint8_t* isrc = p.packed + static_cast<int64_t>(t0) * tile_bytes + warp * (kGvWarpBlocks * kBlock / 2) +
                         prow * (K / 2) + pcol * 16;
   const uint32_t slot_lane = static_cast<uint32_t>(prow * kGvSlicePitch + pcol * 16);
+  const uint32_t ring_lane = smem_u32(ring) + slot_lane;
+  // An item is full (every piece of the slice valid) unless it is the ragged
+  // last tile of the weight or a chunk where this warp's 4 blocks run past K.
+  const int ragged_tile = N % kGvRows != 0 ? tiles - 1 : -1;
+  const int full_chunks = nbk >= kGvWarpBlocks * (warp + 1)
+                              ? static_cast<int>((nbk - kGvWarpBlocks * (warp + 1)) / kGvUnitBlocks) + 1
+                              : 0;
   int i_tile = 0, i_chunk = 0, issued = 0;
   auto issue_next = [&]() {
     const bool live = issued < items;
-    const int rows_left = static_cast<int>(N - static_cast<int64_t>(t0 + i_tile) * kGvRows);
-    const int rem = static_cast<int>(nbk - i_chunk * kGvUnitBlocks) - kGvWarpBlocks * warp;
-    const bool col_ok = live && pcol < 2 * rem;
-    uint8_t* slot = ring + (issued & (kGvDepth - 1)) * kGvSliceBytes + slot_lane;
+    const uint32_t dst = ring_lane + (issued & (kGvDepth - 1)) * kGvSliceBytes;
+    if (live && t0 + i_tile != ragged_tile && i_chunk < full_chunks) {
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const bool v = col_ok && prow + 4 * h < rows_left;
-      cp_async_16(slot + h * 4 * kGvSlicePitch, v ? isrc + h * rows4_bytes : p.packed, v);
+      for (int h = 0; h < 4; ++h) cp_async_16_full(dst + h * 4 * kGvSlicePitch, isrc + h * rows4_bytes);
+    } else {
+      const int rows_left = static_cast<int>(N - static_cast<int64_t>(t0 + i_tile) * kGvRows);
+      const int rem = static_cast<int>(nbk - i_chunk * kGvUnitBlocks) - kGvWarpBlocks * warp;
+      const bool col_ok = live && pcol < 2 * rem;
+      uint8_t* slot = ring + (issued & (kGvDepth - 1)) * kGvSliceBytes + slot_lane;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const bool v = col_ok && prow + 4 * h < rows_left;
+        cp_async_16(slot + h * 4 * kGvSlicePitch, v ? isrc + h * rows4_bytes : p.packed, v);
+      }
     }
     if (live) {
       if (++i_tile == ntile) {
@@ -281,6 +305,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
 
   const float mu = kScales32 ? 0.0f : *p.mu;
   const uint32_t lane_base = kLutWindow | (static_cast<uint32_t>(lane) * 4);
+  const uint32_t ring_frag = smem_u32(ring) + static_cast<uint32_t>(g * kGvSlicePitch + 8 * t);
   // Scales this lane decodes per item: row lane%16 of the tile, blocks
   // 4 warp + lane/16 and 4 warp + lane/16 + 2; the lanes holding rows g and
   // g+8 hand them over by shuffle.  The block index runs like the copy
@@ -292,18 +317,26 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
   float c2v[kGvDepth][2];
   auto fetch = [&](int slot) {
     const bool live = fetched < items;
-    const bool row_ok = live && static_cast<int64_t>(t0 + f_tile) * kGvRows + frow < N;
-    const int blk = f_chunk * kGvUnitBlocks + fblk;
+    // fp32 scales: t(127) = 1, "c2" is the block's absmax and mu = 0, so the
+    // decode below returns the absmax itself.
+    if (live && t0 + f_tile != ragged_tile && f_chunk < full_chunks) {
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const bool v = row_ok && blk + 2 * e < nbk;
-      const int64_t gb = v ? fgb + 2 * e : 0;
-      // fp32 scales: t(127) = 1, "c2" is the block's absmax and mu = 0, so
-      // the decode below returns the absmax itself.
-      const int q = kScales32 ? 127 : p.qscale[gb];
-      const float c2 = __ldg(p.c2 + (kScales32 ? gb : gb >> 8));
-      qv[slot][e] = v ? q : 0;
-      c2v[slot][e] = v ? c2 : 0.0f;
+      for (int e = 0; e < 2; ++e) {
+        qv[slot][e] = kScales32 ? 127 : p.qscale[fgb + 2 * e];
+        c2v[slot][e] = __ldg(p.c2 + (kScales32 ? fgb + 2 * e : (fgb + 2 * e) >> 8));
+      }
+    } else {
+      const bool row_ok = live && static_cast<int64_t>(t0 + f_tile) * kGvRows + frow < N;
+      const int blk = f_chunk * kGvUnitBlocks + fblk;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool v = row_ok && blk + 2 * e < nbk;
+        const int64_t gb = v ? fgb + 2 * e : 0;
+        const int q = kScales32 ? 127 : p.qscale[gb];
+        const float c2 = __ldg(p.c2 + (kScales32 ? gb : gb >> 8));
+        qv[slot][e] = v ? q : 0;
+        c2v[slot][e] = v ? c2 : 0.0f;
+      }
     }
     if (live) {
       if (++f_tile == ntile) {
@@ -328,16 +361,20 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
   GvCursor cc{0, t0};
   bool first_reduce = true;
   int item = 0;
-  auto run_pass = [&](auto np_const) {
-    constexpr int NP = decltype(np_const)::value;
+  // One pass: np consecutive tiles of chunk cc.c, then one cross-warp
+  // reduction.  The tile loop is not unrolled (one tile body of code keeps the
+  // instruction cache warm); each tile's fp32 partial goes to its slot of the
+  // reduction buffer as soon as the tile is done.
+  const uint32_t red_lane = smem_u32(red) + static_cast<uint32_t>(warp * kGvRedWarpBytes + lane * 16);
+  auto run_pass = [&](int np) {
     const int c = cc.c, tile0 = cc.tile;
-    float acc[NP][NT][4];
-#pragma unroll
-    for (int j = 0; j < NP; ++j) {
+#pragma unroll 1
+    for (int j = 0; j < np; ++j) {
+      float acc[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[j][nt][e] = 0.0f;
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
       const float a_lo = __fadd_rn(__fmul_rn(s_qdiv[qv[0][0] + 128], c2v[0][0]), mu);
       const float a_hi = __fadd_rn(__fmul_rn(s_qdiv[qv[0][1] + 128], c2v[0][1]), mu);
 #pragma unroll
@@ -348,11 +385,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
       fetch(1);
       cp_async_wait<kGvDepth - 1>();  // this item (this lane's pieces)
       __syncwarp();                   // ... and the other lanes' pieces
-      const uint8_t* sl = ring + (item & (kGvDepth - 1)) * kGvSliceBytes + g * kGvSlicePitch + 8 * t;
+      const uint32_t sl = ring_frag + (item & (kGvDepth - 1)) * kGvSliceBytes;
 #pragma unroll
       for (int b = 0; b < kGvWarpBlocks; ++b) {
-        const uint2 wa = *reinterpret_cast<const uint2*>(sl + b * 32);
-        const uint2 wb = *reinterpret_cast<const uint2*>(sl + 8 * kGvSlicePitch + b * 32);
+        const uint2 wa = ld_shared_v2(sl + b * 32);
+        const uint2 wb = ld_shared_v2(sl + 8 * kGvSlicePitch + b * 32);
         float d[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -385,12 +422,18 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
         const float s_g8 = __shfl_sync(0xffffffffu, sv, g + 8 + 16 * (b & 1));
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          acc[j][nt][0] = fmaf(s_g, d[nt][0], acc[j][nt][0]);
-          acc[j][nt][1] = fmaf(s_g, d[nt][1], acc[j][nt][1]);
-          acc[j][nt][2] = fmaf(s_g8, d[nt][2], acc[j][nt][2]);
-          acc[j][nt][3] = fmaf(s_g8, d[nt][3], acc[j][nt][3]);
+          acc[nt][0] = fmaf(s_g, d[nt][0], acc[nt][0]);
+          acc[nt][1] = fmaf(s_g, d[nt][1], acc[nt][1]);
+          acc[nt][2] = fmaf(s_g8, d[nt][2], acc[nt][2]);
+          acc[nt][3] = fmaf(s_g8, d[nt][3], acc[nt][3]);
         }
       }
+      // This tile's partial: slot [tile j][token tile][lane][4] of the warp's buffer.
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(red_lane + (j * NT + nt) * 512),
+                     "f"(acc[nt][0]), "f"(acc[nt][1]), "f"(acc[nt][2]), "f"(acc[nt][3])
+                     : "memory");
       __syncwarp();  // the slot is read; refill it
       issue_next();
       ++item;
@@ -398,13 +441,6 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
 
     // Cross-warp reduction: thread tau sums float tau of the 16 warps'
     // partials ([tile][token tile][lane][4]).
-#pragma unroll
-    for (int j = 0; j < NP; ++j)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        *reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(red) + warp * kGvRedWarpBytes +
-                                   ((j * NT + nt) * 32 + lane) * 16) =
-            make_float4(acc[j][nt][0], acc[j][nt][1], acc[j][nt][2], acc[j][nt][3]);
     __syncthreads();
     if (first_reduce) {  // U partials come from the preceding kernel
       pdl_wait_prior();
@@ -416,7 +452,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
       }
       first_reduce = false;
     }
-    if (tid < NP * NT * 128) {
+    if (tid < np * NT * 128) {
       float y = 0.0f;
 #pragma unroll
       for (int w = 0; w < kGvWarps; ++w) y += red[w * (kGvRedWarpBytes / 4) + tid];
@@ -439,7 +475,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
     }
     __syncthreads();  // the reduction buffer is free again
 #pragma unroll 1
-    for (int j = 0; j < NP; ++j) cc.next(t0, t1);
+    for (int j = 0; j < np; ++j) cc.next(t0, t1);
   };
 
   for (int i0 = 0; i0 < items;) {
@@ -455,15 +491,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
         }
       x_chunk = cc.c;
     }
-    if (np == P) {
-      run_pass(std::integral_constant<int, P>{});
-    } else if constexpr (P == 4) {
-      if (np == 3) run_pass(std::integral_constant<int, 3>{});
-      else if (np == 2) run_pass(std::integral_constant<int, 2>{});
-      else run_pass(std::integral_constant<int, 1>{});
-    } else {
-      run_pass(std::integral_constant<int, 1>{});
-    }
+    run_pass(np);
     i0 += np;
   }
   cp_async_wait<0>();
