@@ -673,7 +673,7 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
       e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
       if (e != cudaSuccess) return from_cuda(e);
     }
-    Timed tm(kFamGemv, s, gemv_launches(K));
+    Timed tm(kFamGemv, s, gemv_launches(K, static_cast<int>(M)));
     return from_cuda(launch_gemv(gp, s));
   }
   // Tensor-core path: dense bf16 weight, U = X A^T, padded B, GEMM with the rank-r step.

@@ -6,28 +6,30 @@
 //
 // The packed weight (0.5 B per weight) is the only large operand, so the path
 // is HBM-bound: it streams the codes once and never writes a dequantized
-// copy.  Three kernels:
+// copy.  Up to three kernels:
 //
-//   xa_part_kernel   U partials: each CTA reduces X A^T over 1024 of K with
+//   xa_part_kernel   U partials, each CTA reduces X A^T over 1024 of K with
 //                    warp MMAs ([P][16][64] fp32); it releases the next
-//                    kernel at once (programmatic dependent launch).
+//                    kernel at once (programmatic dependent launch).  Not
+//                    launched for 9..16 tokens and K <= 4096: the GEMV then
+//                    computes U itself from the X fragments it holds.
 //   gemv_kernel      persistent, one CTA per SM, which owns a contiguous
-//                    range of 8-row tiles.  Each of its 16 warps owns one
+//                    range of 16-row tiles.  Each of its 16 warps owns one
 //                    quarter-kilo slice of K (4 blocks of 64; X held in
 //                    registers as MMA fragments) and walks every tile of the
 //                    CTA: a private ring of 16-byte cp.async copies keeps its
-//                    next 4 tile slices in flight (rows padded in shared
+//                    next 2 tile slices in flight (rows padded in shared
 //                    memory so the fragment loads never conflict), nibble
 //                    pairs are decoded through a byte -> bf16x2 table,
 //                    m16n8k16 MMAs accumulate each block and the decoded
 //                    block scale is applied to the block's fp32 partial.
-//                    Partials of 4 tiles stay in registers; then one
-//                    cross-warp reduction (two CTA barriers) sums the 16
-//                    slices, adds the rank-r term s U B^T (U from the
-//                    partials of the first kernel, the CTA's B rows copied
-//                    once) and stores Y as bf16.  No barrier sits inside a
-//                    tile, so each warp overlaps the latency of one tile's
-//                    loads, lookups and MMAs with the next.
+//                    Each tile's partial goes to the reduction buffer; after
+//                    2 (M > 8) or 4 tiles one cross-warp reduction (two CTA
+//                    barriers) sums the 16 slices, adds the rank-r term
+//                    s U B^T (the CTA's B rows copied once) and stores Y as
+//                    bf16.  No barrier sits inside a tile, so each warp
+//                    overlaps the latency of one tile's loads, lookups and
+//                    MMAs with the next.
 //   gemv_finalize    only when K > 4096: sums the per-chunk fp32 partials and
 //                    adds the rank-r term.
 //
@@ -442,9 +444,14 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
     // Cross-warp reduction: thread tau sums float tau of the 16 warps'
     // partials ([tile][token tile][lane][4]).
     __syncthreads();
-    if (first_reduce) {  // U partials come from the preceding kernel
+    if (first_reduce) {
+      // U from the preceding kernel (programmatic launch): its partials must
+      // be complete before they are read here (K <= 4096) or before this
+      // grid ends (K > 4096: the finalize kernel reads them).  When this
+      // kernel computed U itself no kernel precedes by programmatic launch
+      // and the wait returns at once.
       pdl_wait_prior();
-      if (single) {
+      if (single && !kM16) {
         // The B rows were this thread's oldest copy group, complete since its
         // first item's wait; the barrier above published every thread's.
         gather_u(p, s_u, tid, kGvThreads);
@@ -478,6 +485,52 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
     for (int j = 0; j < np; ++j) cc.next(t0, t1);
   };
 
+  // U = X A^T when K fits one chunk: warp w multiplies its K slice of X (the
+  // fragments in registers, as the MMA's 16-row operand: tokens g, g + 8) by
+  // the same slice of A (8 columns of U per MMA); the 16 warps' partials are
+  // summed through the reduction buffer, up to four 8-column groups per
+  // round, into U in shared memory.  The first CTA also writes U_out.
+  auto compute_u = [&]() {
+    const int n_jt = (p.r + 7) / 8;
+#pragma unroll 1
+    for (int jt0 = 0; jt0 < n_jt; jt0 += 4) {
+      const int njt = n_jt - jt0 < 4 ? n_jt - jt0 : 4;
+#pragma unroll 1
+      for (int jj = 0; jj < njt; ++jj) {
+        const int j = 8 * (jt0 + jj) + g;
+        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int b = 0; b < kGvWarpBlocks; ++b) {
+          const int64_t blk = kGvWarpBlocks * warp + b;
+          uint32_t aw[8];
+          load16(p.A, K, j, blk * kBlock + 16 * t, blk < nbk && j < p.r, aw);
+#pragma unroll
+          for (int s4 = 0; s4 < 4; ++s4) {
+            const uint32_t af[4] = {xf[0][b][2 * s4], NT > 1 ? xf[NT - 1][b][2 * s4] : 0u, xf[0][b][2 * s4 + 1],
+                                    NT > 1 ? xf[NT - 1][b][2 * s4 + 1] : 0u};
+            const uint32_t bf[2] = {aw[2 * s4], aw[2 * s4 + 1]};
+            mma_16816(d, af, bf);
+          }
+        }
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(red_lane + jj * 512), "f"(d[0]), "f"(d[1]),
+                     "f"(d[2]), "f"(d[3])
+                     : "memory");
+      }
+      __syncthreads();
+      if (tid < njt * 128) {
+        float u = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kGvWarps; ++w) u += red[w * (kGvRedWarpBytes / 4) + tid];
+        const int comp = tid & 3, ls = (tid >> 2) & 31, jj = tid >> 7;
+        const int tok = (ls >> 2) + 8 * (comp >> 1);
+        const int j = 8 * (jt0 + jj) + 2 * (ls & 3) + (comp & 1);
+        s_u[tok * kRankPad + j] = u;
+        if (blockIdx.x == 0 && p.U_out != nullptr && tok < p.M && j < p.r) p.U_out[tok * p.r + j] = u;
+      }
+      __syncthreads();
+    }
+  };
+
   for (int i0 = 0; i0 < items;) {
     const int np = (t1 - cc.tile) < P ? (t1 - cc.tile) : P;
     if (cc.c != x_chunk) {
@@ -490,6 +543,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
           load16(p.X, K, tok, (blkw + b) * kBlock + 16 * t, blkw + b < nbk && tok < p.M, xf[nt][b]);
         }
       x_chunk = cc.c;
+      if (kM16 && single) compute_u();
     }
     run_pass(np);
     i0 += np;
@@ -530,7 +584,7 @@ __global__ void __launch_bounds__(256) gemv_finalize_kernel(const __grid_constan
 int gemv_upart_count(int64_t K) { return static_cast<int>((K / kBlock + kXaWarps - 1) / kXaWarps); }
 int gemv_chunks(int64_t K) { return static_cast<int>((K / kBlock + kGvUnitBlocks - 1) / kGvUnitBlocks); }
 
-int gemv_launches(int64_t K) { return gemv_chunks(K) > 1 ? 3 : 2; }
+int gemv_launches(int64_t K, int M) { return gemv_chunks(K) > 1 ? 3 : (M > 8 ? 1 : 2); }
 
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   static bool configured = false;
@@ -550,10 +604,17 @@ cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
 
-  xa_part_kernel<<<p.n_upart, kXaWarps * 32, kXaWarps * kGemvMaxM * kRankPad * 4, stream>>>(p.X, p.A, p.M, p.K, p.r,
-                                                                                          p.upart);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  // M > 8 and K <= 4096: the GEMV computes U itself (its first reduction
+  // comes after two tiles, too early to hide a separate kernel); otherwise U
+  // partials come from the first kernel, which releases the GEMV at once
+  // (programmatic launch) and finishes while the GEMV streams its tiles.
+  const bool fused_u = gemv_chunks(p.K) == 1 && p.M > 8;
+  if (!fused_u) {
+    xa_part_kernel<<<p.n_upart, kXaWarps * 32, kXaWarps * kGemvMaxM * kRankPad * 4, stream>>>(p.X, p.A, p.M, p.K,
+                                                                                            p.r, p.upart);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
 
   const int64_t tiles = (p.N + kGvRows - 1) / kGvRows;
   cudaLaunchConfig_t cfg = {};
@@ -565,7 +626,7 @@ cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = fused_u ? 0 : 1;
   if (p.scale_format == kScalesFp32)
     e = p.M > 8 ? cudaLaunchKernelEx(&cfg, gemv_kernel<true, true>, p)
                 : cudaLaunchKernelEx(&cfg, gemv_kernel<false, true>, p);

@@ -131,7 +131,7 @@ struct GemvParams {
 
 int gemv_upart_count(int64_t K);
 int gemv_chunks(int64_t K);
-int gemv_launches(int64_t K);
+int gemv_launches(int64_t K, int M);
 // Y[m][n] = sum_k X[m][k] W[n][k] + s * sum_j (X A^T)[m][j] B[n][j].
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream);
 
