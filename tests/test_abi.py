@@ -102,3 +102,41 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         binding.lib()
+
+
+def _enum_values(name):
+    text = open(os.path.join(ROOT, "include", "qlora_nf4.h")).read()
+    body = re.search(r"typedef enum " + name + r"\s*\{(.*?)\}", text, flags=re.S).group(1)
+    return {k: int(v) for k, v in re.findall(r"(QLORA_[A-Z0-9_]+)\s*=\s*(\d+)", body)}
+
+
+def test_format_constants_match_the_header():
+    assert _enum_values("qlora_codebook") == {"QLORA_CODEBOOK_NF4": binding.CODEBOOK_NF4,
+                                              "QLORA_CODEBOOK_FP4": binding.CODEBOOK_FP4}
+    assert _enum_values("qlora_scale_format") == {"QLORA_SCALES_DQ_INT8": binding.SCALES_DQ_INT8,
+                                                  "QLORA_SCALES_DQ_FP8": binding.SCALES_DQ_FP8,
+                                                  "QLORA_SCALES_FP32": binding.SCALES_FP32}
+    assert _enum_values("qlora_input_dtype") == {"QLORA_INPUT_FP32": binding.INPUT_FP32,
+                                                 "QLORA_INPUT_BF16": binding.INPUT_BF16,
+                                                 "QLORA_INPUT_FP16": binding.INPUT_FP16}
+
+
+def test_weight_descriptor_layout_matches_the_header():
+    """The ctypes descriptor has the header's fields in the header's order."""
+    text = open(os.path.join(ROOT, "include", "qlora_nf4.h")).read()
+    body = re.search(r"typedef struct qlora_nf4_weight\s*\{(.*?)\}", text, flags=re.S).group(1)
+    fields = re.findall(r"\*?\s*([a-z_0-9]+);", body)
+    assert fields == [f for f, _ in binding.QloraNf4WeightC._fields_]
+    assert ctypes.sizeof(binding.QloraNf4WeightC) == 64
+
+
+def test_format_arguments_rejected_on_the_host(lib):
+    """Invalid codebook / scale format / missing absmax are refused before any
+    device work (the checks run on the host): status 1 = QLORA_ERR_INVALID_ARG."""
+    st = binding.QloraNf4WeightC(8, 128, 16, 16, 16, 16, 2, 0, None)
+    out = ctypes.c_void_p(16)
+    assert lib.qlora_nf4_dequantize(ctypes.byref(st), out, 0, 0, None) == 1
+    st = binding.QloraNf4WeightC(8, 128, 16, 16, 16, 16, 0, 3, None)
+    assert lib.qlora_nf4_dequantize(ctypes.byref(st), out, 0, 0, None) == 1
+    st = binding.QloraNf4WeightC(8, 128, 16, None, None, None, 0, binding.SCALES_FP32, None)
+    assert lib.qlora_nf4_dequantize(ctypes.byref(st), out, 0, 0, None) == 1
