@@ -14,7 +14,7 @@
 //                   absmax by three xor-shuffles, IEEE fp32 division by the
 //                   absmax (by 1 for an all-zero block; a reciprocal multiply
 //                   with an exact-division fallback next to a threshold),
-//                   nearest level from a 129-cell decision table (one 16-byte
+//                   nearest level from a 130-cell decision table (one 16-byte
 //                   lookup per weight), eight codes packed into one 32-bit
 //                   word (even element in the low nibble).
 //  chunk_sums       one warp per chunk: the fp64 sum of its 256 block scales;
