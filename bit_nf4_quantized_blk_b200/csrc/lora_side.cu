@@ -46,6 +46,18 @@ struct PipeBarriers {
   int abort_flag;
 };
 
+// Cross-proxy fence for this CTA's shared memory: orders the executing
+// thread's earlier accesses through the generic proxy (ldmatrix, ld.shared)
+// against its later accesses through the async proxy (TMA writes), and the
+// reverse.  The PTX memory model orders accesses to the same bytes made
+// through different proxies only across such a fence; the mbarrier
+// release/acquire of a stage orders the generic proxy alone.  The stages here
+// are read by ldmatrix and refilled by TMA, so every reading thread runs it
+// after its last read of a stage and before the stage is released.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -57,8 +69,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // ---------------------------------------------------------------------------
 // Grid (ceil(M/64), splits).  One thread of warp 0 streams the CTA's tiles of
 // In (64 rows x 64 columns, TMA, 128-byte swizzle) and of Wt (r16 rows of
-// A, or 64 rows x r16 columns of the padded B) through an 8-deep ring; warps
-// 1-4 each own 16 rows and run the warp MMAs.  skinny_finalize_kernel adds
+// A, or 64 rows x r16 columns of the padded B) through a kStages-deep ring;
+// warps 1-4 each own 16 rows and run the warp MMAs.  skinny_finalize_kernel adds
 // the splits in order and writes the outputs.
 template <bool kRowLayout, int NT>
 __global__ void __launch_bounds__(kThreads) skinny_kernel(const __grid_constant__ CUtensorMap tmIn,
@@ -145,6 +157,7 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const __grid_constant_
         mma_bf16_16816(acc[nt + 1], afr, b1);
       }
     }
+    fence_proxy_async_shared();  // this warp's ldmatrix reads of stage s before its TMA refill
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->empty[s]);
   }
@@ -276,7 +289,7 @@ cudaError_t launch_split_hilo(const float* src, int64_t M, int r, uint16_t* hi, 
 // ---------------------------------------------------------------------------
 // Grid (ceil(C/64), splits).  Warp 0 streams tiles of In (64 tokens x 64
 // columns, 128-byte swizzle) and the matching 64 x r16 tiles of the hi / lo
-// split of S through an 8-deep TMA ring; warps 1-4 each own 16 columns:
+// split of S through a kStages-deep TMA ring; warps 1-4 each own 16 columns:
 // A = In^T by transposed 8x8 loads, B = hi and lo.
 template <int NT>
 __global__ void __launch_bounds__(kThreads) colsum_kernel(const __grid_constant__ CUtensorMap tmIn,
@@ -362,6 +375,7 @@ __global__ void __launch_bounds__(kThreads) colsum_kernel(const __grid_constant_
         mma_bf16_16816(acc[nt + 1], afr, l1);
       }
     }
+    fence_proxy_async_shared();  // this warp's ldmatrix reads of stage s before its TMA refill
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->empty[s]);
   }
