@@ -539,15 +539,14 @@ __global__ void __launch_bounds__(192, 1)
 
 namespace {
 
-// Pair clusters that can be resident at once (0: the pair kernel cannot run).
+// One device's answer for max_pair_clusters.
 template <bool kBMN>
-int max_pair_clusters() {
-  static int cached = -1;
-  if (cached >= 0) return cached;
-  cached = 0;
+int query_pair_clusters() {
   if (cudaFuncSetAttribute(gemm_tn2_kernel<kBMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES) !=
-      cudaSuccess)
-    return cached;
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2);
   cfg.blockDim = dim3(192);
@@ -564,8 +563,16 @@ int max_pair_clusters() {
     cudaGetLastError();
     n = 0;
   }
-  cached = n;
-  return cached;
+  return n;
+}
+
+// Pair clusters that can be resident at once on the current device (0: the
+// pair kernel cannot run there).  Sets the kernel's shared-memory limit on
+// the device as it first asks.
+template <bool kBMN>
+int max_pair_clusters(int dev) {
+  static DeviceValue cached;
+  return cached.get(dev, [] { return query_pair_clusters<kBMN>(); });
 }
 
 template <bool kBMN>
@@ -603,15 +610,18 @@ cudaError_t launch_pair(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
 }  // namespace
 
 cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_tn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  const int clusters = a.b_mn_major ? max_pair_clusters<true>() : max_pair_clusters<false>();
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static DeviceOnce configured;
+  e = configured.run(dev, [] {
+    cudaError_t r = cudaFuncSetAttribute(gemm_tn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(gemm_tn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    return r;
+  });
+  if (e != cudaSuccess) return e;
+  const int clusters = a.b_mn_major ? max_pair_clusters<true>(dev) : max_pair_clusters<false>(dev);
   const bool pair = clusters > 0;
   // B (and B2) boxes: the pair kernel loads 128 rows of N per CTA.
   const uint32_t bn_box = pair ? static_cast<uint32_t>(BNH) : static_cast<uint32_t>(BN);

@@ -587,20 +587,20 @@ int gemv_chunks(int64_t K) { return static_cast<int>((K / kBlock + kGvUnitBlocks
 int gemv_launches(int64_t K, int M) { return gemv_chunks(K) > 1 ? 3 : (M > 8 ? 1 : 2); }
 
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaSuccess;
-    for (auto fn : {gemv_kernel<true, false>, gemv_kernel<false, false>, gemv_kernel<true, true>,
-                    gemv_kernel<false, true>})
-      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(xa_part_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kXaWarps * kGemvMaxM * kRankPad * 4);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static DeviceOnce configured;
+  e = configured.run(dev, [] {
+    cudaError_t r = cudaSuccess;
+    for (auto fn : {gemv_kernel<true, false>, gemv_kernel<false, false>, gemv_kernel<true, true>,
+                    gemv_kernel<false, true>})
+      if (r == cudaSuccess) r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes);
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(xa_part_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kXaWarps * kGemvMaxM * kRankPad * 4);
+    return r;
+  });
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
 

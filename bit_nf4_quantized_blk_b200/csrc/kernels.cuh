@@ -3,6 +3,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "device_once.h"
 
 namespace qnf4 {
 

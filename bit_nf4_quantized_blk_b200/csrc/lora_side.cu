@@ -237,13 +237,14 @@ cudaError_t launch_skinny_nt(const CUtensorMap& tin, const CUtensorMap& tw, int6
                              float* part, int* status, cudaStream_t stream) {
   constexpr int kStage = kInTile + 128 * NT * 8;
   constexpr int smem = 1024 + kStages * kStage + static_cast<int>(sizeof(PipeBarriers));
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(skinny_kernel<kRowLayout, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static DeviceOnce configured;
+  e = configured.run(dev, [] {
+    return cudaFuncSetAttribute(skinny_kernel<kRowLayout, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>((M + kTileRows - 1) / kTileRows), static_cast<unsigned>(splits));
   skinny_kernel<kRowLayout, NT><<<grid, kThreads, smem, stream>>>(tin, tw, M, C, splits, part, status);
   return cudaGetLastError();
@@ -427,12 +428,14 @@ cudaError_t launch_colsum_nt(const CUtensorMap& tin, const CUtensorMap& thi, con
                              int64_t C, int splits, float* part, int* status, cudaStream_t stream) {
   constexpr int kStage = kInTile + 2 * 128 * NT * 8;
   constexpr int smem = 1024 + kStages * kStage + static_cast<int>(sizeof(PipeBarriers));
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(colsum_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static DeviceOnce configured;
+  e = configured.run(dev, [] {
+    return cudaFuncSetAttribute(colsum_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>((C + kTileCols - 1) / kTileCols), static_cast<unsigned>(splits));
   colsum_kernel<NT><<<grid, kThreads, smem, stream>>>(tin, thi, tlo, M, C, splits, part, status);
   return cudaGetLastError();

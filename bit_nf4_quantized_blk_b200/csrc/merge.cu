@@ -216,22 +216,20 @@ template <int kSteps, bool kFp32, bool kPair32>
 cudaError_t launch_merge_kernel(const WeightView& w, const uint16_t* A, const uint16_t* B, int r, float scale,
                                 void* out, cudaStream_t stream) {
   // Resident CTAs on the device, queried once per device and instantiation.
-  constexpr int kMaxDevices = 64;
-  static int resident[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int ctas = dev < kMaxDevices ? resident[dev] : 0;
-  if (ctas == 0) {
+  static DeviceValue resident;
+  const int ctas = resident.get(dev, [dev, &e] {
     int sms = 0, per_sm = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, merge_kernel<kSteps, kFp32, kPair32>,
-                                                        kMergeThreads, 0);
-    if (e != cudaSuccess) return e;
-    ctas = sms * (per_sm > 0 ? per_sm : 1);
-    if (dev < kMaxDevices) resident[dev] = ctas;
-  }
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, merge_kernel<kSteps, kFp32, kPair32>, kMergeThreads,
+                                                        0);
+    if (e != cudaSuccess) return -1;
+    return sms * (per_sm > 0 ? per_sm : 1);
+  });
+  if (ctas < 0) return e;
   const int64_t gx = (w.cols / kBlock + kMergeWarps - 1) / kMergeWarps;
   const int64_t n_tiles = (w.rows + 15) / 16;
   int64_t gy = (static_cast<int64_t>(ctas) + gx - 1) / gx;

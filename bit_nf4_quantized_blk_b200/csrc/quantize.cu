@@ -450,13 +450,15 @@ namespace {
 
 template <int kIn, bool kFp4, bool kScales32>
 cudaError_t launch_codes(const QuantBatchParams& p, unsigned grid, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(quantize_codes_kernel<kIn, kFp4, kScales32>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static DeviceOnce configured;
+  e = configured.run(dev, [] {
+    return cudaFuncSetAttribute(quantize_codes_kernel<kIn, kFp4, kScales32>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   quantize_codes_kernel<kIn, kFp4, kScales32><<<grid, kQThreads, kQuantSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }
