@@ -54,7 +54,7 @@ def _stale(obj: str, deps) -> bool:
 
 def build(verbose: bool = False, ptxas_info: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
-    headers = [os.path.join(CSRC, h) for h in os.listdir(CSRC) if h.endswith(".cuh")]
+    headers = [os.path.join(CSRC, h) for h in os.listdir(CSRC) if h.endswith((".cuh", ".h"))]
     headers.append(os.path.join(HERE, "..", "include", "qlora_nf4.h"))
     objs = []
     for src in SOURCES:

