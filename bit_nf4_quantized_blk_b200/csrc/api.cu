@@ -395,12 +395,22 @@ WeightView view_of(const qlora_nf4_weight* w) {
   return WeightView{w->packed, w->qscale, w->c2, w->mu, w->rows, w->cols, w->codebook, w->scale_format, w->absmax};
 }
 
+// Shapes the linear paths take: M >= 1 tokens, N (rows) a multiple of 8, K
+// (cols) a multiple of 64, rank 1..64; and sizes within the kernels' 32-bit
+// indices and TMA coordinates: M * 64 < 2^31, N and K < 2^31, N * K <= 2^40.
+qlora_status check_linear_shape(int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (M < 1 || N < 1 || N % 8 != 0 || K < kBlock || K % kBlock != 0 || r < 1 || r > kMaxRank)
+    return QLORA_ERR_INVALID_ARG;
+  if (M > (int64_t{1} << 31) / kRankPad || N > INT32_MAX || K > INT32_MAX || N > (int64_t{1} << 40) / K)
+    return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
 qlora_status check_linear_args(const qlora_nf4_weight* w, int64_t M, int32_t r, size_t ws_bytes, const void* ws) {
   qlora_status st = check_weight(w);
   if (st != QLORA_OK) return st;
-  if (M < 1 || r < 1 || r > kMaxRank) return QLORA_ERR_INVALID_ARG;
-  if (w->rows % 8 != 0) return QLORA_ERR_INVALID_ARG;
-  if (M > (int64_t{1} << 31) / kRankPad) return QLORA_ERR_UNSUPPORTED;
+  st = check_linear_shape(M, w->rows, w->cols, r);
+  if (st != QLORA_OK) return st;
   if (ws == nullptr || !aligned(ws, 256)) return ws == nullptr ? QLORA_ERR_WORKSPACE : QLORA_ERR_ALIGNMENT;
   if (ws_bytes < linear_ws_layout(M, w->rows, w->cols).total) return QLORA_ERR_WORKSPACE;
   return QLORA_OK;
@@ -605,7 +615,7 @@ extern "C" qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A
 }
 
 extern "C" size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r) {
-  if (M < 1 || N < 1 || K < kBlock || K % kBlock != 0 || r < 1 || r > kMaxRank) return 0;
+  if (check_linear_shape(M, N, K, r) != QLORA_OK) return 0;
   return linear_ws_layout(M, N, K).total;
 }
 

@@ -276,7 +276,10 @@ qlora_status qlora_workspace_status(void *ws, size_t ws_bytes, void *stream);
 /*
  * Workspace bytes for qlora_linear_fwd / qlora_linear_bwd at tokens M,
  * weight [N, K] and rank r (the larger of the two needs; one workspace may
- * serve both).  Returns 0 for invalid sizes.
+ * serve both).  Returns 0 for sizes the linear calls refuse: M < 1, N not a
+ * positive multiple of 8, K not a positive multiple of 64, r outside 1..64,
+ * or beyond the limits M <= 2^25, N and K < 2^31, N * K <= 2^40 (for
+ * which the calls return QLORA_ERR_UNSUPPORTED).
  */
 size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
 

@@ -75,6 +75,24 @@ def test_linear_ws_bytes(lib):
     assert binding.qlora_linear_ws_bytes(0, 1024, 1024, 8) == 0
     assert binding.qlora_linear_ws_bytes(16, 1024, 1000, 8) == 0
     assert binding.qlora_linear_ws_bytes(16, 1024, 1024, 65) == 0
+    assert binding.qlora_linear_ws_bytes(16, 1020, 1024, 8) == 0  # N not a multiple of 8
+    assert binding.qlora_linear_ws_bytes(2**25, 8, 64, 8) > 0  # the largest M the calls take
+    assert binding.qlora_linear_ws_bytes(2**25 + 1, 8, 64, 8) == 0
+    assert binding.qlora_linear_ws_bytes(16, 2**33, 64, 8) == 0  # N beyond 32-bit indices
+    assert binding.qlora_linear_ws_bytes(16, 8, 2**31, 8) == 0  # K likewise
+
+
+def test_linear_size_limits_refused_on_the_host(lib):
+    """A weight whose row count passes the storage checks but exceeds the
+    linear kernels' 32-bit indices is refused (7 = QLORA_ERR_UNSUPPORTED)
+    before the workspace or the device is looked at."""
+    W = binding.QloraNf4WeightC(2**33, 64, 16, 16, 16, 16)
+    assert lib.qlora_linear_fwd(ctypes.byref(W), 16, 4, 16, 16, 8, 1.0, 16, None, 256, 1 << 30, None) == 7
+    assert lib.qlora_linear_bwd(ctypes.byref(W), 16, 16, 4, 16, 16, 8, 1.0, None, 16, 0, None, None, 256,
+                                1 << 30, None) == 7
+    W8 = binding.QloraNf4WeightC(8, 64, 16, 16, 16, 16)
+    assert lib.qlora_linear_fwd(ctypes.byref(W8), 16, 2**25 + 1, 16, 16, 8, 1.0, 16, None, 256, 1 << 30,
+                                None) == 7
 
 
 def test_argument_checks_run_before_any_launch(lib):
