@@ -124,8 +124,50 @@ def lib() -> ctypes.CDLL:
     return L
 
 
-def _ptr(t) -> int | None:
-    return None if t is None else t.data_ptr()
+# dtypes accepted for "bf16" buffers: bf16 data or its 16-bit patterns.
+_BF16_BITS = (torch.bfloat16, torch.int16, torch.uint16)
+_F32 = (torch.float32,)
+_OUT_DTYPES = {0: _BF16_BITS, 1: _F32}  # out_dtype 0 = bf16, 1 = fp32
+
+
+def _dev(t, name: str, dtypes=None, need: int | None = None) -> int:
+    """Device pointer of tensor argument ``name`` after the checks a raw
+    pointer cannot carry: a torch.Tensor, contiguous, of one of ``dtypes``,
+    with at least ``need`` elements, on the current CUDA device (the device
+    the library launches on).  What the library checks itself (alignment,
+    weight shapes, ranks, enum values) is left to it."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {', '.join(str(d) for d in dtypes)}")
+    if need is not None and t.numel() < need:
+        raise ValueError(f"{name}: {t.numel()} elements, needs at least {need}")
+    _check_placement(t, name)
+    return t.data_ptr()
+
+
+def _check_placement(t: torch.Tensor, name: str) -> None:
+    """The tensor lives on the current CUDA device (the one the library launches on)."""
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor, got one on {t.device}")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name}: on {t.device}, but the library runs on the current device cuda:{cur}")
+
+
+def _dev_opt(t, name: str, dtypes=None, need: int | None = None) -> int | None:
+    return None if t is None else _dev(t, name, dtypes, need)
+
+
+def _ws(ws, name: str = "ws") -> tuple[int, int]:
+    """(pointer, size in bytes) of a workspace tensor of any dtype."""
+    return _dev(ws, name), ws.numel() * ws.element_size()
+
+
+def _rank_ok(r: int) -> bool:
+    return 1 <= r <= 64
 
 
 def _stream(stream) -> int | None:
@@ -172,9 +214,39 @@ class NF4Weight:
             scale_format,
         )
 
+    @property
+    def numel(self) -> int | None:
+        """rows * cols, or None when the shape is one the library refuses."""
+        ok = self.rows >= 1 and self.cols >= 64 and self.cols % 64 == 0
+        return self.rows * self.cols if ok else None
+
     def c_struct(self) -> QloraNf4WeightC:
-        return QloraNf4WeightC(self.rows, self.cols, self.packed.data_ptr(), _ptr(self.qscale), _ptr(self.c2),
-                               _ptr(self.mu), self.codebook, self.scale_format, _ptr(self.absmax))
+        n = self.numel
+        blocks = None if n is None else n // 64
+        chunks = None if n is None else (blocks + 255) // 256
+        return QloraNf4WeightC(
+            self.rows,
+            self.cols,
+            _dev(self.packed, "packed", (torch.uint8,), None if n is None else n // 2),
+            _dev_opt(self.qscale, "qscale", (torch.int8, torch.uint8), blocks),
+            _dev_opt(self.c2, "c2", _F32, chunks),
+            _dev_opt(self.mu, "mu", _F32, None if n is None else 1),
+            self.codebook,
+            self.scale_format,
+            _dev_opt(self.absmax, "absmax", _F32, blocks),
+        )
+
+
+def _weight_array(ws):
+    arr = (QloraNf4WeightC * len(ws))()
+    for i, w in enumerate(ws):
+        arr[i] = w.c_struct()
+    return arr
+
+
+def _same_length(a, b, what: str) -> None:
+    if len(a) != len(b):
+        raise ValueError(f"{what}: {len(a)} inputs for {len(b)} outputs")
 
 
 def qlora_status_string(status: int) -> str:
@@ -190,35 +262,41 @@ def qlora_nf4_sizes(rows: int, cols: int) -> dict:
 
 def qlora_nf4_quantize(W: torch.Tensor, out: NF4Weight, ws: torch.Tensor, d_status=None, stream=None) -> None:
     st = out.c_struct()
-    _check("qlora_nf4_quantize", lib().qlora_nf4_quantize(W.data_ptr(), ctypes.byref(st), ws.data_ptr(),
-                                                          ws.numel() * ws.element_size(), _ptr(d_status),
-                                                          _stream(stream)))
+    wp = _dev(W, "W", _F32, out.numel)
+    wsp, wsb = _ws(ws)
+    dsp = _dev_opt(d_status, "d_status", (torch.int32,), 1)
+    _check("qlora_nf4_quantize", lib().qlora_nf4_quantize(wp, ctypes.byref(st), wsp, wsb, dsp, _stream(stream)))
+
+
+def _input_code(W: torch.Tensor, name: str) -> int:
+    if not isinstance(W, torch.Tensor) or W.dtype not in _INPUT_OF_DTYPE:
+        raise TypeError(f"{name}: expected an fp32, bf16 or fp16 torch.Tensor")
+    return _INPUT_OF_DTYPE[W.dtype]
 
 
 def qlora_nf4_quantize_ex(W: torch.Tensor, out: NF4Weight, ws: torch.Tensor, d_status=None, stream=None) -> None:
     """Quantize an fp32, bf16 or fp16 tensor (the input dtype follows W.dtype)."""
+    code = _input_code(W, "W")
     st = out.c_struct()
+    wp = _dev(W, "W", None, out.numel)
+    wsp, wsb = _ws(ws)
+    dsp = _dev_opt(d_status, "d_status", (torch.int32,), 1)
     _check("qlora_nf4_quantize_ex",
-           lib().qlora_nf4_quantize_ex(W.data_ptr(), _INPUT_OF_DTYPE[W.dtype], ctypes.byref(st), ws.data_ptr(),
-                                       ws.numel() * ws.element_size(), _ptr(d_status), _stream(stream)))
+           lib().qlora_nf4_quantize_ex(wp, code, ctypes.byref(st), wsp, wsb, dsp, _stream(stream)))
 
 
 def qlora_nf4_quantize_batched_ex(Ws, outs, ws: torch.Tensor, d_status=None, stream=None) -> None:
-    dtypes = {w.dtype for w in Ws}
-    if len(dtypes) != 1:
+    _same_length(Ws, outs, "qlora_nf4_quantize_batched_ex")
+    codes = {_input_code(w, f"Ws[{i}]") for i, w in enumerate(Ws)}
+    if len(codes) > 1:
         raise ValueError("one input dtype per call")
     arr = _weight_array(outs)
-    ptrs = (ctypes.c_void_p * len(Ws))(*[w.data_ptr() for w in Ws])
+    ptrs = (ctypes.c_void_p * len(Ws))(*[_dev(w, f"Ws[{i}]", None, o.numel) for i, (w, o) in enumerate(zip(Ws, outs))])
+    wsp, wsb = _ws(ws)
+    dsp = _dev_opt(d_status, "d_status", (torch.int32,), 1)
+    code = codes.pop() if codes else INPUT_FP32
     _check("qlora_nf4_quantize_batched_ex",
-           lib().qlora_nf4_quantize_batched_ex(ptrs, _INPUT_OF_DTYPE[dtypes.pop()], arr, len(outs), ws.data_ptr(),
-                                               ws.numel() * ws.element_size(), _ptr(d_status), _stream(stream)))
-
-
-def _weight_array(ws):
-    arr = (QloraNf4WeightC * len(ws))()
-    for i, w in enumerate(ws):
-        arr[i] = w.c_struct()
-    return arr
+           lib().qlora_nf4_quantize_batched_ex(ptrs, code, arr, len(outs), wsp, wsb, dsp, _stream(stream)))
 
 
 def qlora_nf4_quantize_batched_ws_bytes(outs) -> int:
@@ -227,67 +305,106 @@ def qlora_nf4_quantize_batched_ws_bytes(outs) -> int:
 
 
 def qlora_nf4_quantize_batched(Ws, outs, ws: torch.Tensor, d_status=None, stream=None) -> None:
+    _same_length(Ws, outs, "qlora_nf4_quantize_batched")
     arr = _weight_array(outs)
-    ptrs = (ctypes.c_void_p * len(Ws))(*[w.data_ptr() for w in Ws])
+    ptrs = (ctypes.c_void_p * len(Ws))(*[_dev(w, f"Ws[{i}]", _F32, o.numel) for i, (w, o) in enumerate(zip(Ws, outs))])
+    wsp, wsb = _ws(ws)
+    dsp = _dev_opt(d_status, "d_status", (torch.int32,), 1)
     _check("qlora_nf4_quantize_batched",
-           lib().qlora_nf4_quantize_batched(ptrs, arr, len(outs), ws.data_ptr(), ws.numel() * ws.element_size(),
-                                            _ptr(d_status), _stream(stream)))
+           lib().qlora_nf4_quantize_batched(ptrs, arr, len(outs), wsp, wsb, dsp, _stream(stream)))
 
 
 def qlora_nf4_quantize_noalloc(W: torch.Tensor, out: NF4Weight, d_status=None, stream=None) -> None:
     """Quantize without a workspace (library-internal scratch; tensors up to 2^26 weights)."""
     st = out.c_struct()
-    _check("qlora_nf4_quantize_noalloc",
-           lib().qlora_nf4_quantize_noalloc(W.data_ptr(), ctypes.byref(st), _ptr(d_status), _stream(stream)))
+    wp = _dev(W, "W", _F32, out.numel)
+    dsp = _dev_opt(d_status, "d_status", (torch.int32,), 1)
+    _check("qlora_nf4_quantize_noalloc", lib().qlora_nf4_quantize_noalloc(wp, ctypes.byref(st), dsp, _stream(stream)))
 
 
 def qlora_nf4_dequantize(w: NF4Weight, out: torch.Tensor, out_dtype: int = 0, transpose: int = 0, stream=None) -> None:
     st = w.c_struct()
-    _check("qlora_nf4_dequantize",
-           lib().qlora_nf4_dequantize(ctypes.byref(st), out.data_ptr(), out_dtype, transpose, _stream(stream)))
+    op = _dev(out, "out", _OUT_DTYPES.get(out_dtype), w.numel)
+    _check("qlora_nf4_dequantize", lib().qlora_nf4_dequantize(ctypes.byref(st), op, out_dtype, transpose,
+                                                              _stream(stream)))
 
 
 def qlora_nf4_dequantize_batched(weights, outs, out_dtype: int = 0, stream=None) -> None:
+    _same_length(weights, outs, "qlora_nf4_dequantize_batched")
     arr = _weight_array(weights)
-    ptrs = (ctypes.c_void_p * len(outs))(*[o.data_ptr() for o in outs])
+    dt = _OUT_DTYPES.get(out_dtype)
+    ptrs = (ctypes.c_void_p * len(outs))(*[_dev(o, f"outs[{i}]", dt, w.numel)
+                                           for i, (w, o) in enumerate(zip(weights, outs))])
     _check("qlora_nf4_dequantize_batched",
            lib().qlora_nf4_dequantize_batched(arr, ptrs, len(weights), out_dtype, _stream(stream)))
 
 
 def qlora_merge(w: NF4Weight, A, B, r: int, scale: float, out, out_dtype: int = 0, stream=None) -> None:
     st = w.c_struct()
-    _check("qlora_merge",
-           lib().qlora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(scale), out.data_ptr(),
-                             out_dtype, _stream(stream)))
+    sized = w.numel is not None and _rank_ok(r)
+    ap = _dev(A, "A", _BF16_BITS, r * w.cols if sized else None)
+    bp = _dev(B, "B", _BF16_BITS, w.rows * r if sized else None)
+    op = _dev(out, "out", _OUT_DTYPES.get(out_dtype), w.numel)
+    _check("qlora_merge", lib().qlora_merge(ctypes.byref(st), ap, bp, r, float(scale), op, out_dtype, _stream(stream)))
 
 
 def qlora_workspace_reset(ws: torch.Tensor, stream=None) -> None:
-    _check("qlora_workspace_reset", lib().qlora_workspace_reset(ws.data_ptr(), ws.numel(), _stream(stream)))
+    wsp, wsb = _ws(ws)
+    _check("qlora_workspace_reset", lib().qlora_workspace_reset(wsp, wsb, _stream(stream)))
 
 
 def qlora_workspace_status(ws: torch.Tensor, stream=None) -> int:
-    return int(lib().qlora_workspace_status(ws.data_ptr(), ws.numel(), _stream(stream)))
+    wsp, wsb = _ws(ws)
+    return int(lib().qlora_workspace_status(wsp, wsb, _stream(stream)))
 
 
 def qlora_linear_ws_bytes(M: int, N: int, K: int, r: int) -> int:
     return int(lib().qlora_linear_ws_bytes(M, N, K, r))
 
 
+def _tokens(X, name: str, w: NF4Weight) -> int:
+    """M of a [M, K] activation, checking its second dimension against the weight's K."""
+    if not isinstance(X, torch.Tensor) or X.dim() != 2:
+        raise ValueError(f"{name}: expected a 2-D [M, K] tensor")
+    if w.numel is not None and X.shape[1] != w.cols:
+        raise ValueError(f"{name}: {X.shape[1]} columns, the weight has K = {w.cols}")
+    return X.shape[0]
+
+
 def qlora_linear_fwd(w: NF4Weight, X, A, B, r: int, scale: float, Y, U_out, ws, stream=None) -> None:
     st = w.c_struct()
+    M = _tokens(X, "X", w)
+    sized = w.numel is not None and _rank_ok(r)
+    N, K = w.rows, w.cols
+    xp = _dev(X, "X", _BF16_BITS)
+    ap = _dev(A, "A", _BF16_BITS, r * K if sized else None)
+    bp = _dev(B, "B", _BF16_BITS, N * r if sized else None)
+    yp = _dev(Y, "Y", _BF16_BITS, M * N if w.numel is not None else None)
+    up = _dev_opt(U_out, "U_out", _F32, M * r if sized else None)
+    wsp, wsb = _ws(ws)
     _check("qlora_linear_fwd",
-           lib().qlora_linear_fwd(ctypes.byref(st), X.data_ptr(), X.shape[0], A.data_ptr(), B.data_ptr(), r,
-                                  float(scale), Y.data_ptr(), _ptr(U_out), ws.data_ptr(), ws.numel(),
-                                  _stream(stream)))
+           lib().qlora_linear_fwd(ctypes.byref(st), xp, M, ap, bp, r, float(scale), yp, up, wsp, wsb, _stream(stream)))
 
 
 def qlora_linear_bwd(w: NF4Weight, X, dY, A, B, r: int, scale: float, dX, accumulate: int, dA, dB, ws,
                      U=None, stream=None) -> None:
     st = w.c_struct()
+    M = _tokens(X, "X", w)
+    sized = w.numel is not None and _rank_ok(r)
+    N, K = w.rows, w.cols
+    known = w.numel is not None
+    xp = _dev(X, "X", _BF16_BITS)
+    gp = _dev(dY, "dY", _BF16_BITS, M * N if known else None)
+    ap = _dev(A, "A", _BF16_BITS, r * K if sized else None)
+    bp = _dev(B, "B", _BF16_BITS, N * r if sized else None)
+    up = _dev_opt(U, "U", _F32, M * r if sized else None)
+    dxp = _dev_opt(dX, "dX", _BF16_BITS, M * K if known else None)
+    dap = _dev_opt(dA, "dA", _F32, r * K if sized else None)
+    dbp = _dev_opt(dB, "dB", _F32, N * r if sized else None)
+    wsp, wsb = _ws(ws)
     _check("qlora_linear_bwd",
-           lib().qlora_linear_bwd(ctypes.byref(st), X.data_ptr(), dY.data_ptr(), X.shape[0], A.data_ptr(),
-                                  B.data_ptr(), r, float(scale), _ptr(U), _ptr(dX), int(accumulate), _ptr(dA),
-                                  _ptr(dB), ws.data_ptr(), ws.numel(), _stream(stream)))
+           lib().qlora_linear_bwd(ctypes.byref(st), xp, gp, M, ap, bp, r, float(scale), up, dxp, int(accumulate), dap,
+                                  dbp, wsp, wsb, _stream(stream)))
 
 
 def qlora_timing_enable(enable: bool) -> None:
