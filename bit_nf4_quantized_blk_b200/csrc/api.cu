@@ -8,6 +8,7 @@
 // integration" (section "Exact CPU teaching quantizer and adapter gradient
 // path") with the same fp32 rule the definition uses.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -194,8 +195,10 @@ const Nf4DecisionTable* decision_table(int codebook) {
 enum Family { kFamQuant, kFamDequant, kFamGemv, kFamSide, kFamGemm, kFamMerge, kFamCount };
 const char* const kFamNames[kFamCount] = {"quantize", "dequant", "gemv", "side", "gemm", "merge"};
 
+// Shared by every host thread: `mu` guards the event pool and the records.
 struct TimingState {
-  bool enabled = false;
+  std::mutex mu;
+  std::atomic<bool> enabled{false};
   std::vector<cudaEvent_t> pool;
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending[kFamCount];
   double ms[kFamCount] = {};
@@ -207,8 +210,9 @@ TimingState& timing() {
   return t;
 }
 
-cudaEvent_t take_event() {
-  TimingState& T = timing();
+// An event from the pool, or a new one (nullptr if none can be created).
+// The caller holds T.mu.
+cudaEvent_t take_event_locked(TimingState& T) {
   if (!T.pool.empty()) {
     cudaEvent_t e = T.pool.back();
     T.pool.pop_back();
@@ -219,22 +223,32 @@ cudaEvent_t take_event() {
   return e;
 }
 
-// Brackets the kernels enqueued during its lifetime with two events.
+// Brackets the kernels enqueued during its lifetime with two events.  An
+// event that cannot be taken or recorded drops the record, never the launch.
 class Timed {
  public:
   Timed(Family fam, cudaStream_t s, int kernels = 1) : fam_(fam), s_(s), kernels_(kernels) {
-    if (timing().enabled) {
-      start_ = take_event();
-      if (start_ != nullptr) cudaEventRecord(start_, s_);
+    TimingState& T = timing();
+    if (!T.enabled.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lock(T.mu);
+    start_ = take_event_locked(T);
+    if (start_ != nullptr && cudaEventRecord(start_, s_) != cudaSuccess) {
+      T.pool.push_back(start_);
+      start_ = nullptr;
     }
   }
   ~Timed() {
     if (start_ == nullptr) return;
-    cudaEvent_t stop = take_event();
-    if (stop == nullptr) return;
-    cudaEventRecord(stop, s_);
-    timing().pending[fam_].push_back({start_, stop});
-    timing().launches[fam_] += kernels_;
+    TimingState& T = timing();
+    std::lock_guard<std::mutex> lock(T.mu);
+    cudaEvent_t stop = take_event_locked(T);
+    if (stop == nullptr || cudaEventRecord(stop, s_) != cudaSuccess) {
+      T.pool.push_back(start_);
+      if (stop != nullptr) T.pool.push_back(stop);
+      return;
+    }
+    T.pending[fam_].push_back({start_, stop});
+    T.launches[fam_] += kernels_;
   }
   Timed(const Timed&) = delete;
   Timed& operator=(const Timed&) = delete;
@@ -821,6 +835,7 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
 
 extern "C" qlora_status qlora_timing_enable(int32_t enable) {
   TimingState& T = timing();
+  std::lock_guard<std::mutex> lock(T.mu);
   if (enable) {
     for (int f = 0; f < kFamCount; ++f) {
       for (auto& pr : T.pending[f]) {
@@ -832,7 +847,7 @@ extern "C" qlora_status qlora_timing_enable(int32_t enable) {
       T.launches[f] = 0;
     }
   }
-  T.enabled = enable != 0;
+  T.enabled.store(enable != 0, std::memory_order_relaxed);
   return QLORA_OK;
 }
 
@@ -843,19 +858,25 @@ extern "C" qlora_status qlora_timing_read(const char* family, double* total_ms, 
     if (std::strcmp(family, kFamNames[i]) == 0) f = i;
   if (f < 0) return QLORA_ERR_INVALID_ARG;
   TimingState& T = timing();
+  std::lock_guard<std::mutex> lock(T.mu);
+  // Every pending pair is consumed, so a failed pair is neither counted nor
+  // read again; the first failure is returned after the others are summed.
+  cudaError_t first_error = cudaSuccess;
   for (auto& pr : T.pending[f]) {
     float ms = 0.0f;
     cudaError_t e = cudaEventSynchronize(pr.second);
     if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pr.first, pr.second);
-    if (e != cudaSuccess) return from_cuda(e);
-    T.ms[f] += ms;
+    if (e == cudaSuccess)
+      T.ms[f] += ms;
+    else if (first_error == cudaSuccess)
+      first_error = e;
     T.pool.push_back(pr.first);
     T.pool.push_back(pr.second);
   }
   T.pending[f].clear();
   if (total_ms) *total_ms = T.ms[f];
   if (launches) *launches = T.launches[f];
-  return QLORA_OK;
+  return from_cuda(first_error);
 }
 
 // ===========================================================================

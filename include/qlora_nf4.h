@@ -327,8 +327,11 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
  *   qlora_timing_read   : waits for the recorded events of `family` and returns
  *                         the summed device time in milliseconds and the number
  *                         of launches since enabling; INVALID_ARG for an unknown
- *                         family name.
- * Not thread-safe with concurrent enqueueing from several host threads.
+ *                         family name; CUDA if an event could not be read (the
+ *                         other records are still summed and every record read
+ *                         is consumed).
+ * Host threads may enqueue concurrently while timing is enabled.  The events
+ * belong to the device current at their creation: time one device per process.
  */
 qlora_status qlora_timing_enable(int32_t enable);
 qlora_status qlora_timing_read(const char *family, double *total_ms, int64_t *launches);
