@@ -395,6 +395,105 @@ def bench_merge(reps=10):
 # CPU oracle baseline
 # ---------------------------------------------------------------------------
 
+def bench_stack(steps=2, warmup=1, layers=32, M=M_TOKENS, device="cuda"):
+    """The 32-layer chained stack of the 7B layer's projections at 8192 tokens
+    (r = 16, alpha = 32, weights with 0.1% x10 outliers), both phases:
+
+    * quantize: one batched quantize + DQ call over all 224 fp32 weights
+      (6.98 G values), inputs resident in HBM, 4.5159 algorithmic B/weight;
+    * fwd+bwd: per layer q = Q(h), k = K(h), v = V(h), a = O(q), g = G(a),
+      u = U(a), h' = D(g + u), then the backward through the same graph
+      (dh = dX_q + dX_k + dX_v and da = dX_g + dX_u through the accumulate
+      flag; k, v and the top take seeded upstream gradients), 32 x 7.211
+      TFLOP per pass.  g + u is one torch add (model plumbing, not the method).
+    """
+    r, s = R, 32.0 / R
+    Q, K_, V, O, G, U, D = range(7)
+    projs = workloads.LAYER7B
+    Ws, outs, adapters = [], [], []
+    for layer in range(layers):
+        As, Bs = [], []
+        for t in range(7):
+            W, A, B = workloads.stack_projection(layer, t, device=device)
+            Ws.append(W)
+            As.append(A)
+            Bs.append(B)
+            outs.append(binding.NF4Weight.empty(projs[t].n, projs[t].k, device=device))
+        adapters.append((As, Bs))
+    del W
+    qws = torch.empty(binding.qlora_nf4_quantize_batched_ws_bytes(outs), dtype=torch.uint8, device=device)
+    dstat = torch.zeros(1, dtype=torch.int32, device=device)
+    n_weights = sum(p.n * p.k for p in projs) * layers
+    q_ms = timed(lambda: binding.qlora_nf4_quantize_batched(Ws, outs, qws, d_status=dstat), steps, warmup, 1)
+    assert dstat.item() == 0, "quantize reported non-finite input"
+    q_bytes = n_weights * (4 + 0.5 + 1 / 64) + 4 * sum(o.c2.numel() + 1 for o in outs)
+    del Ws
+    if device == "cuda":
+        torch.cuda.empty_cache()
+
+    ws = torch.empty(max(binding.qlora_linear_ws_bytes(M, p.n, p.k, r) for p in projs), dtype=torch.uint8,
+                     device=device)
+    binding.qlora_workspace_reset(ws)
+    bf = lambda n: torch.empty((M, n), dtype=torch.bfloat16, device=device)  # noqa: E731
+    f32 = lambda: torch.empty((M, r), dtype=torch.float32, device=device)  # noqa: E731
+    h0 = workloads.stack_input(M, device=device)
+    top = workloads.stack_leaf_grad(layers - 1, "top", M, device=device)
+    leaf = {(layer, n): workloads.stack_leaf_grad(layer, n, M, device=device)
+            for layer in range(layers) for n in ("k", "v")}
+    act = [dict(q=bf(4096), k=bf(1024), v=bf(1024), a=bf(4096), g=bf(14336), u=bf(14336), gu=bf(14336),
+                out=bf(4096), U=[f32() for _ in range(7)]) for _ in range(layers)]
+    grads = [(torch.empty((r, p.k), dtype=torch.float32, device=device),
+              torch.empty((p.n, r), dtype=torch.float32, device=device)) for p in projs]
+    dgu, da, dq = bf(14336), bf(4096), bf(4096)
+    dh_bufs = [bf(4096), bf(4096)]
+
+    def fwd(layer, t, x, y):
+        A, B = adapters[layer][0][t], adapters[layer][1][t]
+        binding.qlora_linear_fwd(outs[layer * 7 + t], x, A, B, r, s, y, act[layer]["U"][t], ws)
+
+    def bwd(layer, t, x, dy, dx, accumulate):
+        A, B = adapters[layer][0][t], adapters[layer][1][t]
+        dA, dB = grads[t]
+        binding.qlora_linear_bwd(outs[layer * 7 + t], x, dy, A, B, r, s, dx, accumulate, dA, dB, ws,
+                                 U=act[layer]["U"][t])
+
+    def step():
+        h = h0
+        for layer in range(layers):
+            a_ = act[layer]
+            fwd(layer, Q, h, a_["q"])
+            fwd(layer, K_, h, a_["k"])
+            fwd(layer, V, h, a_["v"])
+            fwd(layer, O, a_["q"], a_["a"])
+            fwd(layer, G, a_["a"], a_["g"])
+            fwd(layer, U, a_["a"], a_["u"])
+            torch.add(a_["g"], a_["u"], out=a_["gu"])
+            fwd(layer, D, a_["gu"], a_["out"])
+            h = a_["out"]
+        dh = top
+        for layer in reversed(range(layers)):
+            a_ = act[layer]
+            x_in = h0 if layer == 0 else act[layer - 1]["out"]
+            bwd(layer, D, a_["gu"], dh, dgu, 0)
+            bwd(layer, G, a_["a"], dgu, da, 0)
+            bwd(layer, U, a_["a"], dgu, da, 1)
+            bwd(layer, O, a_["q"], da, dq, 0)
+            dh_prev = dh_bufs[layer % 2]
+            bwd(layer, Q, x_in, dq, dh_prev, 0)
+            bwd(layer, K_, x_in, leaf[(layer, "k")], dh_prev, 1)
+            bwd(layer, V, x_in, leaf[(layer, "v")], dh_prev, 1)
+            dh = dh_prev
+
+    f_ms = timed(step, steps, warmup, 1)
+    assert binding.qlora_workspace_status(ws) == 0, "device status"
+    flops = step_flops(M) * layers
+    return {
+        "quantize": {"weights": n_weights, "ms": q_ms, "GB/s": q_bytes / q_ms / 1e6, "bytes_per_weight": 4.5159},
+        "fwd_bwd": {"flops": flops, "ms": f_ms, "TFLOP/s": flops / (f_ms / 1e3) / 1e12},
+        "steps": steps, "warmup": warmup,
+    }
+
+
 def oracle_sample_step(cases_cpu, row_div: int, tokens: int):
     """Run the oracle on a bounded sample of the layer step and extrapolate.
 
@@ -573,6 +672,11 @@ def run_ours(args, rank, world, local_rank):
             v["frac_hbm"] = v["GB/s"] / hbm
         extras["hbm_peak_gbs"] = hbm
         line["secondary"] = extras
+    if rank == 0 and args.stack:
+        line.setdefault("secondary", {})["stack_32x7_8192tok"] = bench_stack()
+        st = line["secondary"]["stack_32x7_8192tok"]
+        st["quantize"]["frac_hbm"] = st["quantize"]["GB/s"] / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        st["fwd_bwd"]["frac_bf16_sustained"] = st["fwd_bwd"]["TFLOP/s"] / peak
     if rank == 0 and world == 1 and not args.no_cpu:
         cases = cpu_cases(device, 256)
         v, t = oracle_sample_step(cases, 32, 256)
@@ -592,6 +696,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--stack", action="store_true",
+                    help="also time the 32-layer chained stack (quantize, fwd+bwd; about 35 GB on the device)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
