@@ -171,10 +171,43 @@ class LayerStep:
         for c, o, dX, dA, dB, U in reversed(list(zip(self.cases, self.outs, self.dX, self.dA, self.dB, self.U))):
             binding.qlora_linear_bwd(o, c.X, c.dY, c.A, c.B, c.r, c.s, dX, 0, dA, dB, self.lws, U=U)
 
+    def run_two_streams(self):
+        """run() with the projections' calls alternating over two streams, one
+        workspace per stream, so that one projection's HBM-bound kernels can
+        run beside another's GEMM.  A backward waits for its own forward (its
+        saved U); the step ends when both streams have finished.  The outputs
+        are bit-identical to run()'s."""
+        if getattr(self, "_streams", None) is None:
+            self._ws2 = torch.empty_like(self.lws)
+            binding.qlora_workspace_reset(self._ws2)
+            self._streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+        main = torch.cuda.current_stream()
+        wss, streams = [self.lws, self._ws2], self._streams
+        binding.qlora_nf4_quantize_batched([c.W for c in self.cases], self.outs, self.qws, d_status=self.dstat)
+        for st in streams:
+            st.wait_stream(main)
+        fwd_done = []
+        for i, (c, o, Y, U) in enumerate(zip(self.cases, self.outs, self.Y, self.U)):
+            with torch.cuda.stream(streams[i % 2]):
+                binding.qlora_linear_fwd(o, c.X, c.A, c.B, c.r, c.s, Y, U, wss[i % 2])
+                ev = torch.cuda.Event()
+                ev.record(streams[i % 2])
+                fwd_done.append(ev)
+        for j, i in enumerate(reversed(range(len(self.cases)))):
+            c, o = self.cases[i], self.outs[i]
+            with torch.cuda.stream(streams[j % 2]):
+                streams[j % 2].wait_event(fwd_done[i])
+                binding.qlora_linear_bwd(o, c.X, c.dY, c.A, c.B, c.r, c.s, self.dX[i], 0, self.dA[i], self.dB[i],
+                                         wss[j % 2], U=self.U[i])
+        for st in streams:
+            main.wait_stream(st)
+
     def check_status(self):
         assert self.dstat.item() == 0, "quantize reported non-finite input"
-        st = binding.qlora_workspace_status(self.lws)
-        assert st == 0, f"device status {st}"
+        for ws in (self.lws, getattr(self, "_ws2", None)):
+            if ws is not None:
+                st = binding.qlora_workspace_status(ws)
+                assert st == 0, f"device status {st}"
 
     # end-to-end: host buffers in, host buffers out
     def host_buffers(self):
@@ -619,7 +652,7 @@ def run_ours(args, rank, world, local_rank):
     binding.qlora_timing_enable(True)
     clock.start()
     window = []
-    ms = timed(step.run, args.steps, args.warmup, world, window)
+    ms = timed(step.run if args.streams == 1 else step.run_two_streams, args.steps, args.warmup, world, window)
     clocks = clock.stop(window)
     fam = {f: binding.qlora_timing_read(f) for f in ("quantize", "dequant", "gemv", "side", "gemm")}
     binding.qlora_timing_enable(False)
@@ -645,7 +678,8 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD,
                    "flops_per_step_per_gpu": flops, "l2": "inputs larger than L2 (GBs per step)",
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"replicas x{world}",
+                   **({"streams": "projections alternate over 2 streams"} if args.streams == 2 else {})},
         "roofline": {"bound": "tensor", "kernel": "gemm_tn2_kernel (tcgen05 pair-CTA 256x256 tile)",
                      "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tflops / peak,
                      "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": gemm_traffic_per_launch(),
@@ -696,6 +730,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--streams", type=int, choices=[1, 2], default=1,
+                    help="2: the timed step alternates the projections' calls over two streams")
     ap.add_argument("--stack", action="store_true",
                     help="also time the 32-layer chained stack (quantize, fwd+bwd; about 35 GB on the device)")
     args = ap.parse_args()
