@@ -103,3 +103,14 @@ def test_fill_kernels_between_calls_change_nothing(step):
     for trial in range(2):
         assert _differing(ref, _serial_with_fills(step, fill)) == [], f"trial {trial}"
     del fill
+
+
+def test_bench_two_stream_step_matches_serial(step):
+    """bench.py --streams 2 times LayerStep.run_two_streams: the same outputs
+    bit for bit as the serial step, on both workspaces' status words."""
+    ref = _serial(step)
+    for trial in range(3):
+        step.run_two_streams()
+        torch.cuda.synchronize()
+        assert _differing(ref, _outputs(step)) == [], f"trial {trial}"
+    step.check_status()
