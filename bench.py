@@ -560,6 +560,52 @@ def oracle_sample_step(cases_cpu, row_div: int, tokens: int):
     return step_flops() / total / 1e12, total
 
 
+def oracle_secondary(device, row_div=16):
+    """The oracle on bounded samples of the secondary rows, times scaled to
+    the full work (rank 0, N = 1, beside the GPU's own rows):
+
+    * quantize + DQ and dequantize (bf16) of the first N/row_div rows of each
+      of the six tensors of the first OPT-1.3B layer, as weights/s and GB/s at
+      4.5159 and 2.5159 algorithmic bytes per weight;
+    * the decode-shaped forward on the 14336 x 4096 gate at M = 16: fp32
+      decode of the first N/row_div rows plus the fp64 forward of those rows
+      (the sample's quantization is not timed), as microseconds per full call.
+    """
+    from oracle import lora, nf4
+
+    t_q = t_d = 0.0
+    n = 0
+    for layer, t, p in workloads.opt13b_weight_shapes():
+        if layer != 0:
+            continue
+        rows = max(8, p.n // row_div)
+        W = workloads.opt13b_weight(layer, t, device=device)[:rows].cpu().numpy()
+        t0 = time.perf_counter()
+        st = nf4.quantize_weight(W)
+        t1 = time.perf_counter()
+        nf4.dequantize_weight(st, "bf16")
+        t2 = time.perf_counter()
+        t_q += t1 - t0
+        t_d += t2 - t1
+        n += rows * p.k
+    case = workloads.gemv_case(16, device=device)
+    rows = max(8, case.proj.n // row_div)
+    st = nf4.quantize_weight(case.W[:rows].cpu().numpy())
+    f64 = lambda t: t.float().cpu().numpy().astype(np.float64)  # noqa: E731
+    X, A, B = f64(case.X), f64(case.A), f64(case.B[:rows])
+    t0 = time.perf_counter()
+    Wh = nf4.dequantize_weight(st, "fp32").astype(np.float64)
+    lora.lora_forward(X, Wh, A, B, case.s)
+    t_gemv = (time.perf_counter() - t0) * (case.proj.n / rows)
+    return {
+        "quantize": {"weights_per_s": n / t_q, "GB/s": n * 4.5159 / t_q / 1e9},
+        "dequant_bf16": {"weights_per_s": n / t_d, "GB/s": n * 2.5159 / t_d / 1e9},
+        "gemv_gate_14336x4096_M16": {"us_per_call": t_gemv * 1e6},
+        "sample": (f"first 1/{row_div} of the rows of the first OPT-1.3B layer's six tensors ({n} weights); "
+                   f"first 1/{row_div} of the gate's rows at M = 16; times scaled to full calls"),
+    }
+
+
 class CpuCase(dict):
     """Host copies of one projection's inputs (first `tokens` token rows only)."""
 
@@ -717,7 +763,8 @@ def run_ours(args, rank, world, local_rank):
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
                                 "sample": "oracle (numpy; fp64 LoRA) on 1/32 of each weight's rows and 256 of 8192 "
                                           "tokens per projection, times scaled to the full step",
-                                "extrapolated_step_s": t}
+                                "extrapolated_step_s": t,
+                                "secondary": oracle_secondary(device)}
     if rank == 0:
         print(json.dumps(line))
 
