@@ -621,6 +621,20 @@ def cpu_cases(device, tokens):
     return [CpuCase(workloads.layer7b_case(t, m=M_TOKENS, device=device), tokens) for t in range(7)]
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's processor string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
 def cores_used():
     try:
         return len(os.sched_getaffinity(0))
@@ -653,7 +667,8 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_flops() / (value * 1e12) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "flops_per_step_per_gpu": step_flops(), "parallelism": "replicas x1"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model(), "nproc": os.cpu_count()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": wall,
     }))
@@ -761,6 +776,7 @@ def run_ours(args, rank, world, local_rank):
         cases = cpu_cases(device, 256)
         v, t = oracle_sample_step(cases, 32, 256)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+                                "cpu_model": cpu_model(), "nproc": os.cpu_count(),
                                 "sample": "oracle (numpy; fp64 LoRA) on 1/32 of each weight's rows and 256 of 8192 "
                                           "tokens per projection, times scaled to the full step",
                                 "extrapolated_step_s": t,

@@ -12,3 +12,8 @@ def test_oracle_secondary_small_sample():
         v = res[key][field]
         assert v > 0 and math.isfinite(v), key
     assert "1/256" in res["sample"]
+
+
+def test_cpu_model_is_named():
+    assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
+    assert bench.cores_used() >= 1
