@@ -45,6 +45,10 @@
  *     Calls on different streams with different workspaces may overlap; the
  *     results do not depend on the overlap (every kernel sums in a fixed
  *     order), bit for bit.
+ *   - Every call launches on the calling thread's current device; all its
+ *     pointers must be that device's memory.  One process may use several
+ *     devices (kernel attributes are set per device) and several host
+ *     threads.
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
