@@ -199,3 +199,21 @@ def test_format_arguments_are_checked():
     Wh = torch.zeros(8 * 128 + 8, dtype=torch.bfloat16, device="cuda")[4:4 + 8 * 128].view(8, 128)  # 8-byte offset
     with pytest.raises(binding.QloraError, match="ALIGNMENT"):
         binding.qlora_nf4_quantize_ex(Wh, binding.NF4Weight.empty(8, 128), ws)
+
+
+@pytest.mark.parametrize("codebook,fmt", FORMATS)
+def test_zero_second_level_scale(codebook, fmt):
+    """c2 = 0 in every chunk: an all-zero weight, and a weight whose blocks all
+    share one absmax (every block scale equals the mean).  The scale codes are
+    0, the decoded scale is the mean, and the state and the fp32 dequantized
+    weight are bit-exact with the oracle's."""
+    zero = np.zeros((8, 1024), np.float32)
+    same = np.tile(np.linspace(-0.5, 0.5, 64, dtype=np.float32), (8, 16))
+    for W, what in ((zero, "all zero"), (same, "one absmax")):
+        st = nf4.quantize_weight(W, codebook=codebook, scale_format=fmt)
+        out = gpu_quantize(torch.from_numpy(W), CB[codebook], SF[fmt])
+        assert_state_equal(out, st, f"{what} {codebook}/{fmt}")
+        d32 = torch.empty(W.shape, dtype=torch.float32, device="cuda")
+        binding.qlora_nf4_dequantize(out, d32, 1)
+        torch.cuda.synchronize()
+        assert np.array_equal(f32_bits(d32.cpu().numpy()), f32_bits(nf4.dequantize_weight(st, "fp32"))), what
