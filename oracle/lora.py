@@ -35,7 +35,12 @@ def _f64(a) -> np.ndarray:
 
 
 def lora_forward(X, W_hat, A, B, s: float):
-    """``(Y, U)`` with ``U = X A^T`` and ``Y = X W_hat^T + s U B^T``."""
+    """``(Y, U)`` with ``U = X A^T`` and ``Y = X W_hat^T + s U B^T``.
+
+    "FT-02: QLoRA -- Fine-Tuning with Quantization", section "4. The LoRA
+    mechanics the API wraps" (``LoRALinear.forward``); "QLoRA: NF4 storage,
+    gradients and local integration", ``FrozenNF4LoRA.forward``.
+    """
     X, W_hat, A, B = _f64(X), _f64(W_hat), _f64(A), _f64(B)
     U = X @ A.T
     Y = X @ W_hat.T + F64(s) * (U @ B.T)
@@ -43,7 +48,12 @@ def lora_forward(X, W_hat, A, B, s: float):
 
 
 def lora_backward(X, dY, W_hat, A, B, s: float):
-    """``(dX, dA, dB, V)`` for the upstream gradient ``dY`` of ``Y``."""
+    """``(dX, dA, dB, V)`` for the upstream gradient ``dY`` of ``Y``.
+
+    The gradient formulas of "QLoRA: NF4 storage, gradients and local
+    integration", the paragraph after the teaching program (section "Exact
+    CPU teaching quantizer and adapter gradient path"), with ``V = dY B``.
+    """
     X, dY, W_hat, A, B = _f64(X), _f64(dY), _f64(W_hat), _f64(A), _f64(B)
     s = F64(s)
     U = X @ A.T
@@ -55,19 +65,22 @@ def lora_backward(X, dY, W_hat, A, B, s: float):
 
 
 def lora_forward_rows(rows, X, W_hat, A, B, s: float) -> np.ndarray:
-    """Rows ``rows`` of ``Y`` only (each output row depends on its own input row)."""
+    """Rows ``rows`` of ``Y`` only (each output row depends on its own input
+    row): :func:`lora_forward` on those rows, the same passage."""
     Y, _ = lora_forward(_f64(X)[rows], W_hat, A, B, s)
     return Y
 
 
 def lora_backward_rows(rows, dY, W_hat, A, B, s: float) -> np.ndarray:
-    """Rows ``rows`` of ``dX`` only: ``dX[m] = dY[m] W_hat + s (dY[m] B) A``."""
+    """Rows ``rows`` of ``dX`` only: ``dX[m] = dY[m] W_hat + s (dY[m] B) A``
+    (the ``dX`` formula of :func:`lora_backward`, row by row)."""
     dYr, W_hat, A, B = _f64(dY)[rows], _f64(W_hat), _f64(A), _f64(B)
     return dYr @ W_hat + F64(s) * ((dYr @ B) @ A)
 
 
 def lora_adapter_grads(X, dY, A, B, s: float):
-    """``(dA, dB)`` alone: they need no ``W_hat``."""
+    """``(dA, dB)`` alone: they need no ``W_hat`` (the ``dA`` and ``dB``
+    formulas of :func:`lora_backward`, the same passage)."""
     X, dY, A, B = _f64(X), _f64(dY), _f64(A), _f64(B)
     s = F64(s)
     dA = s * ((dY @ B).T @ X)

@@ -147,6 +147,8 @@ def nearest_level(x: np.ndarray, levels: np.ndarray = NF4_LEVELS) -> np.ndarray:
     fp32, ties going to the lowest index (numpy ``argmin`` returns the first
     minimum), exactly as the teaching quantizer's ``argmin`` over the level
     axis.  ``levels`` is the codebook in code order (NF4 by default).
+    Source: "QLoRA: NF4 storage, gradients and local integration", section
+    "Exact CPU teaching quantizer and adapter gradient path" (``quantize_nf4``).
     """
     x = np.asarray(x, dtype=F32).ravel()
     levels = np.asarray(levels, dtype=F32)
@@ -162,7 +164,8 @@ def pack_nibbles(codes: np.ndarray, pad_code: int = ZERO_CODE) -> np.ndarray:
     """Step Q4: two 4-bit codes per byte, element ``2i`` in the low nibble.
 
     An odd number of codes is padded with the zero level's code (7 for NF4),
-    as the teaching quantizer does.
+    as the teaching quantizer does.  Source: the same section as
+    :func:`nearest_level` (the packing of ``quantize_nf4``).
     """
     c = np.asarray(codes, dtype=np.uint8).ravel()
     if c.size % 2:
@@ -197,7 +200,11 @@ def quantize_nf4(w: np.ndarray, block: int = BLOCK, codebook: str = "nf4"):
     Q1 ``a_b = max |w|`` per block.  Q2 ``x = fp32(w / a_b)``, dividing by 1
     for an all-zero block (the zero-block convention), so that block's codes
     are all the zero level's code and its stored scale is 0.  Q3 nearest
-    level of ``codebook`` ("nf4" or "fp4").  Q4 packing.
+    level of ``codebook`` ("nf4" or "fp4").  Q4 packing.  Source: "QLoRA: NF4
+    storage, gradients and local integration", sections "Exact CPU teaching
+    quantizer and adapter gradient path" and "NF4: nonuniform reconstruction
+    levels" (block of 64); the FP4 levels of "FT-02: QLoRA -- Fine-Tuning
+    with Quantization", "Exercise 3: NF4 vs FP4 at equal memory".
     """
     assert_ieee_subnormals()
     w = np.asarray(w)
@@ -231,7 +238,11 @@ def mean_offset(absmax: np.ndarray, dq_block: int = DQ_BLOCK) -> np.float32:
     """Step D1: ``mu = fp32(S / nb)``, the per-tensor mean of the block scales.
 
     ``S`` is summed in fp64: first the 256 scales of each chunk left to right
-    (``P_j``), then the chunk sums left to right in chunk order.
+    (``P_j``), then the chunk sums left to right in chunk order.  Source:
+    "QLoRA: NF4 storage, gradients and local integration", section "Double
+    quantization: correct the scale arithmetic" (the stored offset); the
+    summation order is this repository's reading of an order the page leaves
+    open.
     """
     a = np.asarray(absmax, dtype=F32).ravel()
     nb = a.size
@@ -251,7 +262,9 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
     8 E + 48 + rint(|x| / 2^(E-3)) with E = max(floor(log2 |x|), -6): a
     rounding up to the next power of two carries into the exponent field by
     itself.  Magnitudes past 448 saturate to 0x7E.  The sign bit is the
-    input's (-0 gives 0x80).
+    input's (-0 gives 0x80).  Source: the FP8 scale codes of "FT-02: QLoRA --
+    Fine-Tuning with Quantization", section "2c. Double quantization", read
+    as the E4M3 format from its definition.
     """
     x = np.asarray(x, dtype=F32)
     if not np.isfinite(x).all():
@@ -267,7 +280,7 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
 
 def e4m3_decode(codes: np.ndarray) -> np.ndarray:
     """E4M3 codes -> fp32 values (exact): (8 + m) 2^(e-10) for e >= 1,
-    m 2^-9 for e = 0; NaN for magnitude 0x7F."""
+    m 2^-9 for e = 0; NaN for magnitude 0x7F.  Source: as :func:`e4m3_encode`."""
     c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
     e, m = (c >> 3) & 0xF, c & 0x7
     mag = np.where(e == 0, np.ldexp(m.astype(np.float64), -9),
@@ -283,6 +296,10 @@ def double_quantize(absmax: np.ndarray, dq_block: int = DQ_BLOCK, scale_format: 
     partial, last) chunk ``j``.  D4, "dq_int8": ``q_b = rint(fp32(fp32(d_b /
     c2_j) * 127))`` with ties to even (int8); "dq_fp8": ``q_b =
     E4M3(fp32(d_b / c2_j))`` (uint8 codes).  ``q_b = 0`` where ``c2_j == 0``.
+    Source: "QLoRA: NF4 storage, gradients and local integration", section
+    "Double quantization: correct the scale arithmetic"; "QLoRA Deep Dive:
+    4-bit NormalFloat & Double Quantization Internals", section "2. Squeezing
+    More Memory: Double Quantization (DQ)".
     """
     if scale_format not in ("dq_int8", "dq_fp8"):
         raise ValueError(scale_format)
@@ -309,7 +326,9 @@ def double_quantize(absmax: np.ndarray, dq_block: int = DQ_BLOCK, scale_format: 
 def decode_scales(q: np.ndarray, c2: np.ndarray, mu, dq_block: int = DQ_BLOCK,
                   scale_format: str = "dq_int8") -> np.ndarray:
     """Step R1: ``a'_b = fp32(fp32(t_b * c2_j) + mu)`` with ``t_b = fp32(q_b /
-    127)`` ("dq_int8") or the E4M3 value of ``q_b`` ("dq_fp8")."""
+    127)`` ("dq_int8") or the E4M3 value of ``q_b`` ("dq_fp8").  Source: the
+    inverse of :func:`double_quantize`, same passages; "QLoRA Deep Dive ...",
+    section "The Quantization Process in QLoRA" (decode before use)."""
     c = np.repeat(np.asarray(c2, dtype=F32), dq_block)[: np.asarray(q).size]
     if scale_format == "dq_int8":
         q = np.asarray(q, dtype=np.int8).ravel()
@@ -336,7 +355,9 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 
 def dequantize_codes(codes: np.ndarray, scales: np.ndarray, block: int = BLOCK,
                      levels: np.ndarray = NF4_LEVELS) -> np.ndarray:
-    """Step R2 in fp32: ``w_hat = fp32(L[code] * a'_b)`` for every code."""
+    """Step R2 in fp32: ``w_hat = fp32(L[code] * a'_b)`` for every code.
+    Source: "QLoRA: NF4 storage, gradients and local integration",
+    ``dequantize_nf4`` of the teaching program."""
     codes = np.asarray(codes, dtype=np.uint8).ravel()
     per = np.repeat(np.asarray(scales, dtype=F32), block)[: codes.size]
     return (np.asarray(levels, dtype=F32)[codes] * per).astype(F32)
@@ -364,7 +385,9 @@ def widen_16bit(bits: np.ndarray, dtype: str) -> np.ndarray:
     """16-bit weights (bit patterns, uint16) -> the fp32 values they denote.
 
     "bf16": the bits are the top half of an fp32; "fp16": IEEE half.  Both
-    widenings are exact.
+    widenings are exact.  Source: "FT-02: QLoRA -- Fine-Tuning with
+    Quantization", section "3. BitsAndBytesConfig in practice" (16-bit
+    checkpoints converted at load).
     """
     b = np.asarray(bits, dtype=np.uint16)
     if dtype == "bf16":
@@ -375,7 +398,8 @@ def widen_16bit(bits: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def quantize_weight(w: np.ndarray, codebook: str = "nf4", scale_format: str = "dq_int8") -> NF4DQState:
-    """Steps Q0-Q4 then D1-D4 (none for fp32 scales) on one fp32 tensor."""
+    """Steps Q0-Q4 then D1-D4 (none for fp32 scales) on one fp32 tensor:
+    :func:`quantize_nf4` then :func:`double_quantize`, with their sources."""
     w = np.asarray(w)
     if scale_format not in SCALE_FORMATS:
         raise ValueError(scale_format)
