@@ -146,3 +146,15 @@ def test_opt_in_flags(dry, capsys):
     assert "frac_hbm" in st["quantize"] and "frac_bf16_sustained" in st["fwd_bwd"]
     assert "cpu_baseline" not in d
     assert dry["step"].two_stream_runs == 3 + 5 and dry["step"].runs == 1
+
+
+def test_gemm_traffic_follows_the_source_digest(monkeypatch, tmp_path):
+    """roofline.traffic comes from the committed capture only while the GEMM's
+    sources hash to the digest recorded beside it; otherwise it is null."""
+    assert isinstance(bench.gemm_traffic_per_launch(), int)  # the committed summary matches the tree
+    stale = tmp_path / "summary.md"
+    stale.write_text("traffic_bytes_per_launch: 123\nsource_digest: 0000000000000000\n")
+    monkeypatch.setattr(bench, "GEMM_TRAFFIC_PROFILE", str(stale))
+    assert bench.gemm_traffic_per_launch() is None
+    monkeypatch.setattr(bench, "GEMM_TRAFFIC_PROFILE", str(tmp_path / "missing.md"))
+    assert bench.gemm_traffic_per_launch() is None
