@@ -485,3 +485,35 @@ def test_exact_ties_go_to_the_lower_level():
         assert nf4.nearest_level(np.array([m32]))[0] == j - 1
         assert nf4.nearest_level(np.array([np.nextafter(m32, F32(2))]))[0] == j
     assert found >= 1
+
+
+def _dq_tie_scales():
+    """One chunk of 256 block scales 256 +- d for d = 127 and every
+    half-integer k + 1/2 (k = 0 .. 126): the mean is exactly 256, every
+    deviation d_b = a_b - mu is exact, c2 = 127, and d / c2 * 127 gives back
+    d exactly in fp32 for all of them (checked here), so each half-integer
+    deviation lands exactly on a rounding tie of step D4."""
+    d = np.array([127.0] + [k + 0.5 for k in range(127)], F32)
+    a = np.empty(256, F32)
+    a[0::2] = F32(256.0) + d
+    a[1::2] = F32(256.0) - d
+    for v in d[1:]:
+        for sv in (v, -v):
+            assert F32(F32(F32(sv) / F32(127.0)) * F32(127.0)) == F32(sv)  # an exact tie reaches D4
+    return a, d
+
+
+def test_dq_rounding_ties_go_to_even():
+    """Step D4 rounds to nearest with ties to even: a deviation of exactly
+    k + 1/2 code steps gives the even one of k and k + 1 (0.5 -> 0, 1.5 -> 2,
+    2.5 -> 2, and the same magnitudes with the sign for negative deviations).
+    Rounding half away from zero, or truncation, fails here."""
+    a, d = _dq_tie_scales()
+    q, c2, mu = nf4.double_quantize(a)
+    assert mu == F32(256.0) and c2[0] == F32(127.0)
+    assert q[0] == 127 and q[1] == -127
+    for i, k in enumerate(range(127), start=1):
+        want = k if k % 2 == 0 else k + 1  # the even neighbour of k + 1/2
+        assert q[2 * i] == want, (k, q[2 * i])
+        assert q[2 * i + 1] == -want, (k, q[2 * i + 1])
+    assert [int(v) for v in q[2:8]] == [0, 0, 2, -2, 2, -2]  # 0.5, 1.5, 2.5 and their negatives
