@@ -105,6 +105,19 @@ class ClockSampler:
         except ValueError:
             return None
 
+    @staticmethod
+    def around(device_index, fn):
+        """(fn(), clocks sampled while it ran); clocks is None when
+        `device_index` is None or nvidia-smi is unavailable."""
+        if device_index is None:
+            return fn(), None
+        c = ClockSampler(device_index)
+        c.start()
+        t0 = time.time()
+        out = fn()
+        t1 = time.time()
+        return out, c.stop([t0, t1])
+
     def stop(self, window=None):
         if self.proc is None:
             return None
@@ -339,36 +352,79 @@ def timed(fn, steps, warmup, world, window=None):
 # Secondary measurements (rank 0): quantize / dequant / GEMV / merge rows
 # ---------------------------------------------------------------------------
 
+def timed_reps(fn, reps, warmup, before=None):
+    """Per-call device times (ms) of `reps` calls after `warmup` untimed ones,
+    every call bracketed by its own pair of events on the current stream;
+    `before` (untimed) runs ahead of each call.  All calls are enqueued before
+    the host waits, so host launch latency stays outside the intervals."""
+    for _ in range(warmup):
+        if before is not None:
+            before(0)
+        fn()
+    torch.cuda.synchronize()
+    evs = []
+    for i in range(reps):
+        if before is not None:
+            before(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def rep_stats(ms_list):
+    return {"ms": statistics.median(ms_list), "ms_min": min(ms_list), "reps": len(ms_list)}
+
 def l2_flush_buffer():
     size = 2 * torch.cuda.get_device_properties(0).L2_cache_size
     return torch.empty(max(size, 256 << 20) // 4, dtype=torch.float32, device="cuda")
 
 
-def bench_quantize_dequant(reps=5):
+def bench_quantize_dequant(reps=20, clock=None):
+    """Config 2: quantize + DQ, then bf16 dequantize, of the 168 OPT-1.3B-shaped
+    tensors (one batched call each), `reps` timed calls of each (median and
+    minimum), with the SM clocks sampled over each row's calls."""
     items = workloads.opt13b_weight_shapes()
     Ws = [workloads.opt13b_weight(layer, t, device="cuda") for layer, t, _ in items]
     outs = [binding.NF4Weight.empty(p.n, p.k) for _, _, p in items]
     ws = torch.empty(binding.qlora_nf4_quantize_batched_ws_bytes(outs), dtype=torch.uint8, device="cuda")
     dstat = torch.zeros(1, dtype=torch.int32, device="cuda")
     n = sum(p.n * p.k for _, _, p in items)
-    q_ms = timed(lambda: binding.qlora_nf4_quantize_batched(Ws, outs, ws, d_status=dstat), reps, 2, 1)
+    res = {}
+    q_clock = ClockSampler.around(clock, lambda: timed_reps(
+        lambda: binding.qlora_nf4_quantize_batched(Ws, outs, ws, d_status=dstat), reps, 3))
     assert dstat.item() == 0
     ys = [torch.empty((p.n, p.k), dtype=torch.bfloat16, device="cuda") for _, _, p in items]
-    d_ms = timed(lambda: binding.qlora_nf4_dequantize_batched(outs, ys, 0), reps, 2, 1)
+    d_clock = ClockSampler.around(clock, lambda: timed_reps(
+        lambda: binding.qlora_nf4_dequantize_batched(outs, ys, 0), reps, 3))
     q_bytes = n * (4 + 0.5 + 1 / 64) + 4 * sum(o.c2.numel() + 1 for o in outs)
     d_bytes = n * (0.5 + 1 / 64 + 2) + 4 * sum(o.c2.numel() + 1 for o in outs)
     del Ws, ys
-    return {
-        "quantize": {"weights": n, "ms": q_ms, "GB/s": q_bytes / q_ms / 1e6, "bytes_per_weight": 4.5159},
-        "dequant_bf16": {"weights": n, "ms": d_ms, "GB/s": d_bytes / d_ms / 1e6, "bytes_per_weight": 2.5159},
-    }
+    for name, (ms_list, clocks), nbytes, bpw in (("quantize", q_clock, q_bytes, 4.5159),
+                                                   ("dequant_bf16", d_clock, d_bytes, 2.5159)):
+        st = rep_stats(ms_list)
+        res[name] = {"weights": n, **st, "GB/s": nbytes / st["ms"] / 1e6, "GB/s_best": nbytes / st["ms_min"] / 1e6,
+                     "bytes_per_weight": bpw, "clocks": clocks}
+    return res
 
 
-def bench_gemv(reps=50):
+def bench_gemv(reps=100, copies=8):
+    """Config 3: the decode-shaped forward on the 14336 x 4096 gate at M = 1,
+    4, 16.  `copies` quantized copies of the gate (8 x 31 MB, more than the
+    L2) are used in turn, so every call reads its weight from HBM with no
+    flush kernel in between; the old figure with a 2 x L2 write flush before
+    every call (whose dirty lines the GEMV then has to write back) is kept
+    beside it for comparison."""
     case = workloads.gemv_case(16, device="cuda")
-    out = binding.NF4Weight.empty(14336, 4096)
     qws = torch.empty(binding.qlora_nf4_sizes(14336, 4096)["ws_bytes"], dtype=torch.uint8, device="cuda")
-    binding.qlora_nf4_quantize(case.W, out, qws)
+    outs = []
+    for _ in range(copies):
+        o = binding.NF4Weight.empty(14336, 4096)
+        binding.qlora_nf4_quantize(case.W, o, qws)
+        outs.append(o)
     flush = l2_flush_buffer()
     res = {}
     for M in (1, 4, 16):
@@ -376,26 +432,25 @@ def bench_gemv(reps=50):
         Y = torch.empty((M, 14336), dtype=torch.bfloat16, device="cuda")
         ws = torch.empty(binding.qlora_linear_ws_bytes(M, 14336, 4096, 16), dtype=torch.uint8, device="cuda")
         binding.qlora_workspace_reset(ws)
-        fwd = lambda: binding.qlora_linear_fwd(out, X, case.A, case.B, 16, case.s, Y, None, ws)  # noqa: E731
-        for _ in range(3):
-            fwd()
-        # Enqueue every repetition before waiting: the L2 flush between calls
-        # keeps the GPU busy while the host enqueues the next call, so no
-        # host launch latency lands inside the timed interval.
-        evs = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fwd()
-            b.record()
-            evs.append((a, b))
-        torch.cuda.synchronize()
-        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
-        nbytes = (out.packed.numel() + out.qscale.numel() + 4 * out.c2.numel() + 4 + 2 * (case.A.numel() + case.B.numel())
+        cur = [0]
+
+        def fwd():
+            binding.qlora_linear_fwd(outs[cur[0] % copies], X, case.A, case.B, 16, case.s, Y, None, ws)
+            cur[0] += 1
+
+        rot = rep_stats(timed_reps(fwd, reps, 3))
+        cur[0] = 0
+        fl = rep_stats(timed_reps(lambda: binding.qlora_linear_fwd(outs[0], X, case.A, case.B, 16, case.s, Y, None, ws),
+                                  reps // 2, 3, before=lambda i: flush.zero_()))
+        o = outs[0]
+        nbytes = (o.packed.numel() + o.qscale.numel() + 4 * o.c2.numel() + 4 + 2 * (case.A.numel() + case.B.numel())
                   + 2 * M * (4096 + 14336))
-        res[f"M={M}"] = {"us": ms * 1e3, "GB/s": nbytes / ms / 1e6, "bytes": nbytes}
+        res[f"M={M}"] = {"us": rot["ms"] * 1e3, "us_min": rot["ms_min"] * 1e3, "GB/s": nbytes / rot["ms"] / 1e6,
+                         "bytes": nbytes, "reps": rot["reps"],
+                         "write_flush": {"us": fl["ms"] * 1e3, "GB/s": nbytes / fl["ms"] / 1e6}}
         assert binding.qlora_workspace_status(ws) == 0
+    res["method"] = (f"{copies} quantized copies of the gate used in turn (no flush kernel); write_flush: a 2 x L2 "
+                     "write before every call")
     return res
 
 
@@ -675,7 +730,7 @@ def run_reference(args, rank, world):
 
 
 GEMM_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "gemm_tn_layer_step_traffic.md")
-GEMM_SOURCES = ("csrc/gemm_tc.cu", "csrc/common.cuh")  # the GEMM kernels and the device helpers they use
+GEMM_SOURCES = ("csrc/gemm_nf4.cu", "csrc/gemm_common.cuh", "csrc/common.cuh")  # the GEMM and its device helpers
 
 
 def gemm_traffic_per_launch():
@@ -709,7 +764,8 @@ def run_ours(args, rank, world, local_rank):
     step.check_status()
 
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    clock = ClockSampler(int(vis.split(",")[local_rank]) if vis and vis.split(",")[0].isdigit() else local_rank)
+    smi_index = int(vis.split(",")[local_rank]) if vis and vis.split(",")[0].isdigit() else local_rank
+    clock = ClockSampler(smi_index)
     binding.qlora_timing_enable(True)
     clock.start()
     window = []
@@ -723,7 +779,16 @@ def run_ours(args, rank, world, local_rank):
     gemm_ms, gemm_n = fam["gemm"]
     gemm_ms_per_step = gemm_ms / steps_recorded
     gemm_tflops = gemm_flops_per_step() / (gemm_ms_per_step / 1e3) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # The timed region is a fraction of a second at full clock: the burst
+    # cuBLAS figure is the comparable peak.  The clock-normalised fraction
+    # divides by the peak scaled to the median SM clock sampled in the timed
+    # region (the burst figure taken as a 1965 MHz one unless the peaks file
+    # records its clock).
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_mhz = next((float(v) for k, v in peaks.items() if "bf16" in k and "mhz" in k and "sustained" not in k
+                     and isinstance(v, (int, float))), 1965.0)
+    frac_clock = (gemm_tflops / (peak * clocks["sm_mhz"] / peak_mhz)
+                  if clocks and clocks.get("sm_mhz") else None)
 
     flops = step_flops()
     value = job_throughput(flops, world, ms) / 1e12
@@ -741,11 +806,16 @@ def run_ours(args, rank, world, local_rank):
                    "flops_per_step_per_gpu": flops, "l2": "inputs larger than L2 (GBs per step)",
                    "parallelism": f"replicas x{world}",
                    **({"streams": "projections alternate over 2 streams"} if args.streams == 2 else {})},
-        "roofline": {"bound": "tensor", "kernel": "gemm_tn2_kernel (tcgen05 pair-CTA 256x256 tile)",
+        "roofline": {"bound": "tensor",
+                     "kernel": "gemm_nf4_kernel (tcgen05 pair-CTA 256x256 tile, 4-bit weight decoded into shared memory)",
                      "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tflops / peak,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": gemm_traffic_per_launch(),
+                     "peak_source": f"{peak_src} bf16_tflops (burst; the timed region is "
+                                    f"{args.steps * ms / 1e3:.2f} s at the sampled clock)",
+                     "frac_clock_normalized": frac_clock, "peak_clock_mhz": peak_mhz,
+                     "traffic": gemm_traffic_per_launch(),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
-                     "share_of_step": gemm_ms_per_step / ms},
+                     "share_of_step": gemm_ms_per_step / ms,
+                     "gemm_ms_per_step": gemm_ms_per_step, "gemm_flops_per_step": gemm_flops_per_step()},
         "gpu_launches": int(round(launches_total / steps_recorded * args.steps)),
         "kernel_ms_per_step": {f: v[0] / steps_recorded for f, v in fam.items()},
         "clocks": clocks,
@@ -757,21 +827,27 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and not args.no_extras:
         del step
         torch.cuda.empty_cache()
-        extras = bench_quantize_dequant()
+        extras = bench_quantize_dequant(clock=smi_index)
         extras["gemv_gate_14336x4096"] = bench_gemv()
         extras["merge_layer7b_r16"] = bench_merge()
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         for k in ("quantize", "dequant_bf16", "merge_layer7b_r16"):
             extras[k]["frac_hbm"] = extras[k]["GB/s"] / hbm
         for k, v in extras["gemv_gate_14336x4096"].items():
-            v["frac_hbm"] = v["GB/s"] / hbm
+            if isinstance(v, dict):
+                v["frac_hbm"] = v["GB/s"] / hbm
+                v["write_flush"]["frac_hbm"] = v["write_flush"]["GB/s"] / hbm
         extras["hbm_peak_gbs"] = hbm
         line["secondary"] = extras
-    if rank == 0 and args.stack:
-        line.setdefault("secondary", {})["stack_32x7_8192tok"] = bench_stack()
-        st = line["secondary"]["stack_32x7_8192tok"]
+    if rank == 0 and not args.no_stack:
+        torch.cuda.empty_cache()
+        st, st_clocks = ClockSampler.around(smi_index, bench_stack)
+        line.setdefault("secondary", {})["stack_32x7_8192tok"] = st
+        st["clocks"] = st_clocks
         st["quantize"]["frac_hbm"] = st["quantize"]["GB/s"] / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        st["fwd_bwd"]["frac_bf16_sustained"] = st["fwd_bwd"]["TFLOP/s"] / peak
+        st["fwd_bwd"]["frac_bf16_burst"] = st["fwd_bwd"]["TFLOP/s"] / peak
+        st["fwd_bwd"]["frac_bf16_sustained"] = st["fwd_bwd"]["TFLOP/s"] / peaks.get(
+            "bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     if rank == 0 and world == 1 and not args.no_cpu:
         cases = cpu_cases(device, 256)
         v, t = oracle_sample_step(cases, 32, 256)
@@ -795,8 +871,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--streams", type=int, choices=[1, 2], default=1,
                     help="2: the timed step alternates the projections' calls over two streams")
-    ap.add_argument("--stack", action="store_true",
-                    help="also time the 32-layer chained stack (quantize, fwd+bwd; about 35 GB on the device)")
+    ap.add_argument("--no-stack", action="store_true",
+                    help="skip the 32-layer chained stack (quantize, fwd+bwd; about 35 GB on the device), "
+                         "which the default run times on rank 0")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

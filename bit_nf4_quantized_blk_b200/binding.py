@@ -45,7 +45,10 @@ EXPORTED = [
     "qlora_workspace_reset",
     "qlora_workspace_status",
     "qlora_linear_ws_bytes",
+    "qlora_linear_set_weight_path",
+    "qlora_linear_weight_path",
     "qlora_linear_fwd",
+    "qlora_linear_fwd_stall_diagnostic",
     "qlora_linear_bwd",
     "qlora_timing_enable",
     "qlora_timing_read",
@@ -62,6 +65,7 @@ class QloraError(RuntimeError):
 CODEBOOK_NF4, CODEBOOK_FP4 = 0, 1
 SCALES_DQ_INT8, SCALES_DQ_FP8, SCALES_FP32 = 0, 1, 2
 INPUT_FP32, INPUT_BF16, INPUT_FP16 = 0, 1, 2
+WEIGHT_PATH_FUSED, WEIGHT_PATH_DENSE = 0, 1  # qlora_weight_path
 _INPUT_OF_DTYPE = {torch.float32: INPUT_FP32, torch.bfloat16: INPUT_BF16, torch.float16: INPUT_FP16}
 
 
@@ -111,7 +115,10 @@ def lib() -> ctypes.CDLL:
         "qlora_workspace_reset": (i32, [P, sz, P]),
         "qlora_workspace_status": (i32, [P, sz, P]),
         "qlora_linear_ws_bytes": (sz, [i64, i64, i64, i32]),
+        "qlora_linear_set_weight_path": (i32, [i32]),
+        "qlora_linear_weight_path": (i32, []),
         "qlora_linear_fwd": (i32, [W, P, i64, P, P, i32, f32, P, P, P, sz, P]),
+        "qlora_linear_fwd_stall_diagnostic": (i32, [W, P, i64, P, P, i32, f32, P, P, sz, i32, P]),
         "qlora_linear_bwd": (i32, [W, P, P, i64, P, P, i32, f32, P, P, i32, P, P, P, sz, P]),
         "qlora_timing_enable": (i32, [i32]),
         "qlora_timing_read": (i32, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]),
@@ -362,6 +369,32 @@ def qlora_linear_ws_bytes(M: int, N: int, K: int, r: int) -> int:
     return int(lib().qlora_linear_ws_bytes(M, N, K, r))
 
 
+def qlora_linear_set_weight_path(path: int) -> None:
+    _check("qlora_linear_set_weight_path", lib().qlora_linear_set_weight_path(int(path)))
+
+
+def qlora_linear_weight_path() -> int:
+    return int(lib().qlora_linear_weight_path())
+
+
+class weight_path:
+    """Context manager: run the enclosed linear calls on `path`
+    (WEIGHT_PATH_FUSED or WEIGHT_PATH_DENSE), restoring the previous path."""
+
+    def __init__(self, path: int):
+        self.path = path
+        self.prev = None
+
+    def __enter__(self):
+        self.prev = qlora_linear_weight_path()
+        qlora_linear_set_weight_path(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        qlora_linear_set_weight_path(self.prev)
+        return False
+
+
 def _tokens(X, name: str, w: NF4Weight) -> int:
     """M of a [M, K] activation, checking its second dimension against the weight's K."""
     if not isinstance(X, torch.Tensor) or X.dim() != 2:
@@ -384,6 +417,24 @@ def qlora_linear_fwd(w: NF4Weight, X, A, B, r: int, scale: float, Y, U_out, ws, 
     wsp, wsb = _ws(ws)
     _check("qlora_linear_fwd",
            lib().qlora_linear_fwd(ctypes.byref(st), xp, M, ap, bp, r, float(scale), yp, up, wsp, wsb, _stream(stream)))
+
+
+def qlora_linear_fwd_stall_diagnostic(w: NF4Weight, X, A, B, r: int, scale: float, Y, ws, wait_limit_us: int,
+                                      stream=None) -> None:
+    """Diagnostic: the tensor-core forward with its GEMM made to time out
+    (see the header); read the outcome with qlora_workspace_status."""
+    st = w.c_struct()
+    M = _tokens(X, "X", w)
+    sized = w.numel is not None and _rank_ok(r)
+    N, K = w.rows, w.cols
+    xp = _dev(X, "X", _BF16_BITS)
+    ap = _dev(A, "A", _BF16_BITS, r * K if sized else None)
+    bp = _dev(B, "B", _BF16_BITS, N * r if sized else None)
+    yp = _dev(Y, "Y", _BF16_BITS, M * N if w.numel is not None else None)
+    wsp, wsb = _ws(ws)
+    _check("qlora_linear_fwd_stall_diagnostic",
+           lib().qlora_linear_fwd_stall_diagnostic(ctypes.byref(st), xp, M, ap, bp, r, float(scale), yp, wsp, wsb,
+                                                   int(wait_limit_us), _stream(stream)))
 
 
 def qlora_linear_bwd(w: NF4Weight, X, dY, A, B, r: int, scale: float, dX, accumulate: int, dA, dB, ws,

@@ -345,10 +345,10 @@ int64_t max_group_chunks(const qlora_nf4_weight* outs, int32_t count) {
 
 // Linear workspace layout.
 struct LinearWs {
-  size_t wbf, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, gu, gy, total;
+  size_t wbf, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, vdbpart, gu, gy, total;
 };
 
-LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
+LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, bool dense) {
   LinearWs l;
   size_t off = kWsHeader;
   auto take = [&](size_t bytes) {
@@ -357,7 +357,9 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
     return at;
   };
   const size_t mr = static_cast<size_t>(M) * kRankPad;
-  l.wbf = take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
+  // The dense bf16 copy of the weight exists only on the dense-weight path
+  // (the backward's GEMM runs at every M).
+  l.wbf = take(dense ? static_cast<size_t>(N) * static_cast<size_t>(K) * 2 : 0);
   l.us = take(mr * 2);
   l.uhi = take(mr * 2);
   l.ulo = take(mr * 2);
@@ -369,6 +371,7 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K) {
   l.part = take(p1 > p2 ? p1 : p2);
   const size_t s1 = skinny_partial_bytes(M, N), s2 = skinny_partial_bytes(M, K);
   l.skpart = take(s1 > s2 ? s1 : s2);
+  l.vdbpart = take(M > kGemvMaxM ? vdb_partial_bytes(M, N) : 0);
   // Decode path (M <= 16): U partials and, for K > 4096, per-chunk fp32 outputs.
   const bool decode = M <= kGemvMaxM;
   l.gu = take(decode ? static_cast<size_t>(gemv_upart_count(K)) * kGemvMaxM * kRankPad * 4 : 0);
@@ -420,15 +423,44 @@ qlora_status check_linear_shape(int64_t M, int64_t N, int64_t K, int32_t r) {
   return QLORA_OK;
 }
 
-qlora_status check_linear_args(const qlora_nf4_weight* w, int64_t M, int32_t r, size_t ws_bytes, const void* ws) {
+// Weight path of the tensor-core linear calls (process-wide, read once per call).
+std::atomic<int> g_weight_path{QLORA_WEIGHT_PATH_FUSED};
+
+bool dense_weight_path() { return g_weight_path.load(std::memory_order_relaxed) == QLORA_WEIGHT_PATH_DENSE; }
+
+qlora_status check_linear_args(const qlora_nf4_weight* w, int64_t M, int32_t r, size_t ws_bytes, const void* ws,
+                               bool dense) {
   qlora_status st = check_weight(w);
   if (st != QLORA_OK) return st;
   st = check_linear_shape(M, w->rows, w->cols, r);
   if (st != QLORA_OK) return st;
   if (ws == nullptr || !aligned(ws, 256)) return ws == nullptr ? QLORA_ERR_WORKSPACE : QLORA_ERR_ALIGNMENT;
-  if (ws_bytes < linear_ws_layout(M, w->rows, w->cols).total) return QLORA_ERR_WORKSPACE;
+  if (ws_bytes < linear_ws_layout(M, w->rows, w->cols, dense).total) return QLORA_ERR_WORKSPACE;
   return QLORA_OK;
 }
+
+// The 4-bit weight decoded inside the tensor-core GEMM.
+cudaError_t launch_linear_gemm_nf4(const qlora_nf4_weight* w, const uint16_t* A, int64_t M, const uint16_t* A2,
+                                   const uint16_t* B2, int r, int64_t ldb2, uint16_t* D, int accumulate, int* status,
+                                   bool backward, cudaStream_t s, uint64_t wait_limit_ns = 0, int debug_stall = 0) {
+  Nf4GemmArgs g{};
+  g.w = view_of(w);
+  g.A = A;
+  g.A2 = A2;
+  g.B2 = B2;
+  g.M = M;
+  g.r = r;
+  g.ldb2 = ldb2;
+  g.D = D;
+  g.accumulate = accumulate;
+  g.status = status;
+  g.backward = backward ? 1 : 0;
+  g.wait_limit_ns = wait_limit_ns;
+  g.debug_stall = debug_stall;
+  return launch_gemm_nf4(g, s);
+}
+
+qlora_status gemm_status(cudaError_t e) { return e == cudaErrorNotSupported ? QLORA_ERR_UNSUPPORTED : from_cuda(e); }
 
 }  // namespace
 
@@ -630,8 +662,16 @@ extern "C" qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A
 
 extern "C" size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r) {
   if (check_linear_shape(M, N, K, r) != QLORA_OK) return 0;
-  return linear_ws_layout(M, N, K).total;
+  return linear_ws_layout(M, N, K, dense_weight_path()).total;
 }
+
+extern "C" qlora_status qlora_linear_set_weight_path(int32_t path) {
+  if (path != QLORA_WEIGHT_PATH_FUSED && path != QLORA_WEIGHT_PATH_DENSE) return QLORA_ERR_INVALID_ARG;
+  g_weight_path.store(path, std::memory_order_relaxed);
+  return QLORA_OK;
+}
+
+extern "C" int32_t qlora_linear_weight_path(void) { return g_weight_path.load(std::memory_order_relaxed); }
 
 extern "C" qlora_status qlora_workspace_reset(void* ws, size_t ws_bytes, void* stream) {
   if (ws == nullptr || ws_bytes < kWsHeader) return QLORA_ERR_WORKSPACE;
@@ -650,10 +690,19 @@ extern "C" qlora_status qlora_workspace_status(void* ws, size_t ws_bytes, void* 
   return static_cast<qlora_status>(h);
 }
 
-extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
-                                         const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* U_out,
-                                         void* ws, size_t ws_bytes, void* stream) {
-  qlora_status st = check_linear_args(w, M, r, ws_bytes, ws);
+namespace {
+
+// Diagnostic settings of the fused GEMM (all zero in product calls).
+struct GemmDiagnostics {
+  uint64_t wait_limit_ns;
+  int debug_stall;
+};
+
+qlora_status linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B,
+                        int32_t r, float scale, uint16_t* Y, float* U_out, void* ws, size_t ws_bytes, void* stream,
+                        const GemmDiagnostics& diag) {
+  const bool dense = dense_weight_path() && !diag.debug_stall;
+  qlora_status st = check_linear_args(w, M, r, ws_bytes, ws, dense);
   if (st != QLORA_OK) return st;
   if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) || (U_out && !aligned(U_out, 4)))
@@ -663,7 +712,7 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
   if (st != QLORA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t N = w->rows, K = w->cols;
-  const LinearWs lay = linear_ws_layout(M, N, K);
+  const LinearWs lay = linear_ws_layout(M, N, K, dense);
   int* status = at<int>(ws, 0);
   cudaError_t e;
   if (M <= kGemvMaxM) {
@@ -700,14 +749,16 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
     Timed tm(kFamGemv, s, gemv_launches(K, static_cast<int>(M)));
     return from_cuda(launch_gemv(gp, s));
   }
-  // Tensor-core path: dense bf16 weight, U = X A^T, padded B, GEMM with the rank-r step.
-  DequantBatchParams p;
-  dequant_one(p, w, at<uint16_t>(ws, lay.wbf));
-  {
+  // Tensor-core path: U = X A^T, padded B if needed, GEMM with the rank-r
+  // step; the GEMM decodes the 4-bit weight itself, or, on the dense-weight
+  // path, reads a bf16 copy dequantized first into the workspace.
+  if (dense) {
+    DequantBatchParams p;
+    dequant_one(p, w, at<uint16_t>(ws, lay.wbf));
     Timed tm(kFamDequant, s);
     e = launch_dequant_batch(p, 0, s);
+    if (e != cudaSuccess) return from_cuda(e);
   }
-  if (e != cudaSuccess) return from_cuda(e);
   SkinnyOut so{};
   so.o32 = U_out;
   so.o32_ld = r;
@@ -722,12 +773,19 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
     if (e == cudaSuccess && !b_direct) e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
   }
   if (e != cudaSuccess) return from_cuda(e);
+  const uint16_t* B2 = b_direct ? B : at<uint16_t>(ws, lay.bpad);
+  const int64_t ldb2 = b_direct ? r : kRankPad;
+  if (!dense) {
+    Timed tm(kFamGemm, s);
+    return gemm_status(launch_linear_gemm_nf4(w, X, M, at<uint16_t>(ws, lay.us), B2, r, ldb2, Y, 0, status, false, s,
+                                              diag.wait_limit_ns, diag.debug_stall));
+  }
   GemmArgs g{};
   g.A = X;
   g.B = at<uint16_t>(ws, lay.wbf);
   g.A2 = at<uint16_t>(ws, lay.us);
-  g.B2 = b_direct ? B : at<uint16_t>(ws, lay.bpad);
-  g.ldb2 = b_direct ? r : kRankPad;
+  g.B2 = B2;
+  g.ldb2 = ldb2;
   g.M = M;
   g.N = N;
   g.K = K;
@@ -739,11 +797,29 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16
   return from_cuda(launch_gemm_tn(g, s));
 }
 
+}  // namespace
+
+extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
+                                         const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* U_out,
+                                         void* ws, size_t ws_bytes, void* stream) {
+  return linear_fwd(w, X, M, A, B, r, scale, Y, U_out, ws, ws_bytes, stream, GemmDiagnostics{0, 0});
+}
+
+extern "C" qlora_status qlora_linear_fwd_stall_diagnostic(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
+                                                          const uint16_t* A, const uint16_t* B, int32_t r,
+                                                          float scale, uint16_t* Y, void* ws, size_t ws_bytes,
+                                                          int32_t wait_limit_us, void* stream) {
+  if (M <= kGemvMaxM || wait_limit_us < 1 || wait_limit_us > 1000000) return QLORA_ERR_INVALID_ARG;
+  return linear_fwd(w, X, M, A, B, r, scale, Y, nullptr, ws, ws_bytes, stream,
+                    GemmDiagnostics{static_cast<uint64_t>(wait_limit_us) * 1000ull, 1});
+}
+
 extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,
                                          const uint16_t* A, const uint16_t* B, int32_t r, float scale, const float* U,
                                          uint16_t* dX, int32_t accumulate, float* dA, float* dB, void* ws,
                                          size_t ws_bytes, void* stream) {
-  qlora_status st = check_linear_args(w, M, r, ws_bytes, ws);
+  const bool dense = dense_weight_path();
+  qlora_status st = check_linear_args(w, M, r, ws_bytes, ws, dense);
   if (st != QLORA_OK) return st;
   if (!X || !dY || !A || !B) return QLORA_ERR_INVALID_ARG;
   if (accumulate != 0 && accumulate != 1) return QLORA_ERR_INVALID_ARG;
@@ -755,47 +831,69 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
   if (st != QLORA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t N = w->rows, K = w->cols;
-  const LinearWs lay = linear_ws_layout(M, N, K);
+  const LinearWs lay = linear_ws_layout(M, N, K, dense);
   int* status = at<int>(ws, 0);
   cudaError_t e;
 
-  // V = dY B (bf16 s*V for the dX rank step; hi/lo split for dA).
-  SkinnyOut vo{};
-  vo.os = at<uint16_t>(ws, lay.vs);
-  vo.ohi = at<uint16_t>(ws, lay.vhi);
-  vo.olo = at<uint16_t>(ws, lay.vlo);
-  vo.scale = scale;
   const bool b_direct = (r % 8) == 0 && aligned(B, 16);
-  {
-    Timed tm(kFamSide, s, b_direct ? 2 : 3);
-    if (!b_direct) e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
-    if (b_direct)
-      e = launch_skinny(dY, M, N, B, false, r, r, at<float>(ws, lay.skpart), vo, status, s);
-    else if (e == cudaSuccess)
-      e = launch_skinny(dY, M, N, at<uint16_t>(ws, lay.bpad), false, r, kRankPad, at<float>(ws, lay.skpart), vo,
-                        status, s);
-  }
-  if (e != cudaSuccess) return from_cuda(e);
-
-  if (dB != nullptr) {  // dB = s dY^T U with U = X A^T (saved by the forward, or recomputed)
-    {
-      Timed tm(kFamSide, s, U != nullptr ? 3 : 4);
-      if (U != nullptr) {
-        e = launch_split_hilo(U, M, r, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), s);
-      } else {
-        SkinnyOut uo{};
-        uo.ohi = at<uint16_t>(ws, lay.uhi);
-        uo.olo = at<uint16_t>(ws, lay.ulo);
-        uo.scale = 1.0f;
-        e = launch_skinny(X, M, K, A, true, r, 0, at<float>(ws, lay.skpart), uo, status, s);
-      }
-      if (e == cudaSuccess)
-        e = launch_colsum(dY, M, N, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), r, scale,
-                          at<float>(ws, lay.part), dB, false, status, s);
-    }
+  // B [N, r] feeds the rank-r kernels directly when its rows are 16-byte
+  // multiples, else through a zero-padded copy [N, 64].
+  if (!b_direct) {
+    Timed tm(kFamSide, s);
+    e = launch_pad_rank(B, false, N, r, at<uint16_t>(ws, lay.bpad), s);
     if (e != cudaSuccess) return from_cuda(e);
   }
-  if (dX != nullptr) {  // dX = dY W_hat + s V A, reading W_hat [N, K] and A [r, K] as MN-major operands
+  const uint16_t* Bk = b_direct ? B : at<uint16_t>(ws, lay.bpad);
+  const int64_t ldbk = b_direct ? r : kRankPad;
+  // U = X A^T as a bf16 hi/lo pair (from the saved fp32 U, or recomputed).
+  auto u_hilo = [&]() -> cudaError_t {
+    if (U != nullptr) {
+      Timed tm(kFamSide, s);
+      return launch_split_hilo(U, M, r, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), s);
+    }
+    SkinnyOut uo{};
+    uo.ohi = at<uint16_t>(ws, lay.uhi);
+    uo.olo = at<uint16_t>(ws, lay.ulo);
+    uo.scale = 1.0f;
+    Timed tm(kFamSide, s, 2);
+    return launch_skinny(X, M, K, A, true, r, 0, at<float>(ws, lay.skpart), uo, status, s);
+  };
+  if (dB != nullptr && r <= kVdbMaxRank && M > kGemvMaxM) {
+    // V = dY B (s*V for the dX rank step, hi/lo for dA) and dB = s dY^T U in one pass over dY.
+    e = u_hilo();
+    if (e != cudaSuccess) return from_cuda(e);
+    Timed tm(kFamSide, s, 2);
+    e = launch_vdb(dY, M, N, Bk, ldbk, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), r, scale,
+                   at<float>(ws, lay.vdbpart), at<uint16_t>(ws, lay.vs), at<uint16_t>(ws, lay.vhi),
+                   at<uint16_t>(ws, lay.vlo), dB, status, s);
+    if (e != cudaSuccess) return from_cuda(e);
+  } else {
+    // V = dY B (bf16 s*V for the dX rank step; hi/lo split for dA).
+    SkinnyOut vo{};
+    vo.os = at<uint16_t>(ws, lay.vs);
+    vo.ohi = at<uint16_t>(ws, lay.vhi);
+    vo.olo = at<uint16_t>(ws, lay.vlo);
+    vo.scale = scale;
+    {
+      Timed tm(kFamSide, s, 2);
+      e = launch_skinny(dY, M, N, Bk, false, r, ldbk, at<float>(ws, lay.skpart), vo, status, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+    if (dB != nullptr) {  // dB = s dY^T U
+      e = u_hilo();
+      if (e != cudaSuccess) return from_cuda(e);
+      Timed tm(kFamSide, s, 2);
+      e = launch_colsum(dY, M, N, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), r, scale,
+                        at<float>(ws, lay.part), dB, false, status, s);
+      if (e != cudaSuccess) return from_cuda(e);
+    }
+  }
+  if (dX != nullptr && !dense) {  // dX = dY W_hat + s V A, W_hat decoded in the GEMM, A [r, K] MN-major
+    Timed tm(kFamGemm, s);
+    e = launch_linear_gemm_nf4(w, dY, M, at<uint16_t>(ws, lay.vs), A, r, 0, dX, accumulate, status, true, s);
+    if (e != cudaSuccess) return gemm_status(e);
+  }
+  if (dX != nullptr && dense) {  // dense-weight path: W_hat [N, K] and A [r, K] read as MN-major operands
     DequantBatchParams p;
     dequant_one(p, w, at<uint16_t>(ws, lay.wbf));
     {

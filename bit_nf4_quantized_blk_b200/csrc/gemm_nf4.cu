@@ -1,0 +1,585 @@
+// Training-shaped GEMM of the QLoRA linear with the 4-bit weight decoded
+// inside the kernel (sm_100a, tcgen05 pair-CTA MMAs).
+//
+//   forward         Y  [M][N_w] = X  [M][K_w] W_hat^T + (s U) B^T
+//   backward-input  dX [M][K_w] = dY [M][N_w] W_hat   + (s V) A
+//
+// "QLoRA Deep Dive: 4-bit NormalFloat & Double Quantization Internals",
+// section "The Quantization Process in QLoRA": a block's 4-bit codes and its
+// constant are loaded, multiplied back and used directly in the computation;
+// "FT-02: QLoRA -- Fine-Tuning with Quantization", section "Reading the
+// result: the three lines that decide memory": the frozen weight stays in 4
+// bits and is dequantized on the fly in every forward (and backward) pass.
+// The gradient formulas are those of "QLoRA: NF4 storage, gradients and local
+// integration", section "Exact CPU teaching quantizer and adapter gradient
+// path".
+//
+// The dense bf16 weight never exists in HBM: each stage of the weight operand
+// is decoded from its packed codes and block-scale codes straight into the
+// 128-byte-swizzled shared-memory layout the tensor core reads.  One stage
+// covers 64 values of the reduction, and in both directions one 128-byte row
+// of the stage tile is exactly one quantization block (64 consecutive values
+// of one weight row), so a decoding thread owns one block per stage:
+//   forward  (B operand K-major):  tile row = weight row n, the 64 values of
+//            block (n, k0 / 64);
+//   backward (B operand MN-major): tile row = reduction index n, 64 output
+//            columns k0..k0+63 of weight row n = block (n, k0 / 64).
+// Decoded values are bf16(fp32(L[code] * a)) with the block scale
+// a = fp32(fp32(t * c2) + mu) (t = fp32(q / 127) for int8 codes, the E4M3
+// value for FP8 codes) or the stored fp32 absmax -- the same bits the dense
+// dequantize entry point writes.  The thread first forms the block's 16
+// possible bf16 values (16 multiplies, 8 conversions), splits them into a
+// low-byte and a high-byte table of four registers each, and then looks up
+// four codes at a time with byte permutes whose selectors are the packed
+// nibbles themselves (bit 3 of a code picks the upper half of the table).
+//
+// Pair-CTA layout (cluster of 2, 256 x 256 output tile per pair):
+//   warp 0      TMA producer of this CTA's 128 rows of A (X or dY) per stage,
+//               and of the rank step's tiles; the even CTA arms the stage's
+//               copy barrier (fullA) with both CTAs' bytes
+//   warp 1      TMEM allocation (both CTAs); in the even CTA, MMA issue:
+//               tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16
+//   warps 2-5   epilogue of this CTA's 128 accumulator rows
+//   warps 6-13  weight decoders: two groups of four warps take alternate
+//               stages; each thread decodes one block per stage of its group,
+//               keeps the codes of its next two stages in flight in
+//               registers, fences its shared-memory writes for the async
+//               proxy and its warp arrives on the even CTA's decoded-stage
+//               barrier (fullB).
+// The MMA issuer waits on both barriers of a stage.  Keeping the copies on a
+// barrier of their own lets a teardown wait for exactly the copies in
+// flight: the even producer waits for the last stages' copies of both CTAs
+// and then signals the odd CTA (`drained`), which waits for that before its
+// shared memory can go.
+// The rank-r LoRA term is one more pipeline step of ceil(r/16) MMAs into the
+// same accumulator, its operands loaded by TMA.  No TMA load uses cluster
+// multicast; the MMA's tcgen05.commit is delivered to both CTAs of the pair
+// (an mbarrier arrive, not a load).  Every barrier wait is bounded in time
+// (common.cuh).
+#include "common.cuh"
+#include "gemm_common.cuh"
+#include "kernels.cuh"
+
+namespace qnf4 {
+
+namespace {
+
+constexpr int BM = 128;          // rows of A per CTA (256 per pair)
+constexpr int BN = 256;          // output columns per pair tile
+constexpr int BNH = BN / 2;      // B rows (forward) / output columns (backward) per CTA
+constexpr int BK = 64;           // reduction values per stage (one quantization block)
+constexpr int STAGES = 6;
+constexpr int A_TILE = BM * BK * 2;    // 16 KB
+constexpr int B_TILE = BNH * BK * 2;   // 16 KB
+constexpr int TMEM_COLS = 512;         // two 128 x 256 fp32 accumulators per CTA
+constexpr int kDecodeGroups = 2;
+constexpr int kFirstDecodeWarp = 6;
+constexpr int kThreads = 32 * (kFirstDecodeWarp + 4 * kDecodeGroups);
+constexpr int kDecodedArrivals = 2 * 4;    // the four decode warps of each CTA that handle a stage
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_TILE + B_TILE) + 512;
+constexpr size_t kL2PanelBudget = size_t(48) << 20;
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Four bf16 values from four 4-bit codes: `m` holds the codes' low three bits
+// in its four low nibbles (the permute selectors), `h` their bit 3 (0 / 1 per
+// nibble).  lo*/hi* are the low and high bytes of the 16-entry value table.
+__device__ __forceinline__ void lookup4(uint32_t m, uint32_t h, uint32_t lo0, uint32_t lo1, uint32_t lo2, uint32_t lo3,
+                                        uint32_t hi0, uint32_t hi1, uint32_t hi2, uint32_t hi3, uint32_t& out01,
+                                        uint32_t& out23) {
+  const uint32_t upper = prmt(0x0000FF00u, 0u, h);  // byte i = 0xFF where code i >= 8
+  const uint32_t lo = (prmt(lo0, lo1, m) & ~upper) | (prmt(lo2, lo3, m) & upper);
+  const uint32_t hi = (prmt(hi0, hi1, m) & ~upper) | (prmt(hi2, hi3, m) & upper);
+  out01 = prmt(lo, hi, 0x5140u);  // value 0 in the low half, value 1 in the high half
+  out23 = prmt(lo, hi, 0x7362u);
+}
+
+// Decode one quantization block (64 codes in w, element 2i in the low nibble
+// of byte i) with scale `a` into a 128-byte row of a 128B-swizzled tile at
+// shared address `row`: 16-byte chunk j (values 8j..8j+7) goes to chunk
+// position j ^ sw.
+__device__ __forceinline__ void decode_block_to_smem(uint32_t row, uint32_t sw, const uint32_t (&w)[8], float a,
+                                                     const float (&L)[16]) {
+  uint32_t P[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) P[i] = pack_bf16x2(__fmul_rn(L[2 * i], a), __fmul_rn(L[2 * i + 1], a));
+  // P[i] bytes: (lo 2i, hi 2i, lo 2i+1, hi 2i+1)
+  const uint32_t lo0 = prmt(P[0], P[1], 0x6420u), lo1 = prmt(P[2], P[3], 0x6420u);
+  const uint32_t lo2 = prmt(P[4], P[5], 0x6420u), lo3 = prmt(P[6], P[7], 0x6420u);
+  const uint32_t hi0 = prmt(P[0], P[1], 0x7531u), hi1 = prmt(P[2], P[3], 0x7531u);
+  const uint32_t hi2 = prmt(P[4], P[5], 0x7531u), hi3 = prmt(P[6], P[7], 0x7531u);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t m = w[j] & 0x77777777u;
+    const uint32_t h = (w[j] >> 3) & 0x11111111u;
+    uint32_t o0, o1, o2, o3;
+    lookup4(m, h, lo0, lo1, lo2, lo3, hi0, hi1, hi2, hi3, o0, o1);
+    lookup4(m >> 16, h >> 16, lo0, lo1, lo2, lo3, hi0, hi1, hi2, hi3, o2, o3);
+    st_shared_v4(row + ((static_cast<uint32_t>(j) ^ sw) << 4), o0, o1, o2, o3);
+  }
+}
+
+// The packed codes, scale code and second-level scale of one block, in flight.
+struct BlockLoad {
+  uint32_t w[8];
+  float x;   // c2 of the block's chunk, or the fp32 absmax
+  int q;     // int8 / E4M3 scale code (bit pattern)
+};
+
+__device__ __forceinline__ void load_block(BlockLoad& b, const Nf4GemmParams& p, int64_t blk) {
+  if (blk < 0) return;
+  const uint4* src = reinterpret_cast<const uint4*>(p.packed + blk * 32);
+  const uint4 u0 = ld_stream_u4(src), u1 = ld_stream_u4(src + 1);
+  b.w[0] = u0.x; b.w[1] = u0.y; b.w[2] = u0.z; b.w[3] = u0.w;
+  b.w[4] = u1.x; b.w[5] = u1.y; b.w[6] = u1.z; b.w[7] = u1.w;
+  if (p.scale_format == kScalesFp32) {
+    b.x = __ldg(p.absmax + blk);
+    b.q = 0;
+  } else {
+    b.q = __ldg(p.qscale + blk);
+    b.x = __ldg(p.c2 + (blk >> 8));
+  }
+}
+
+}  // namespace
+
+template <bool kBwd>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_nf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ Nf4GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_TILE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_TILE);  // fullA: TMA bytes (even CTA)
+  uint64_t* decoded = full + STAGES;      // fullB: decode warps of both CTAs (even CTA)
+  uint64_t* empty = decoded + STAGES;
+  uint64_t* acc_full = empty + STAGES;    // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2], even CTA
+  uint64_t* drain = acc_empty + 2;
+  uint64_t* drained = drain + 1;          // odd CTA: every copy of the pair has landed
+  uint64_t* never = drained + 1;          // diagnostic: a barrier nothing arrives at
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t rank = cluster_ctarank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = p.M, N = p.N, num_k = p.num_k, r_steps = p.r_steps;
+  const int m_tiles = (M + 2 * BM - 1) / (2 * BM), n_tiles = (N + BN - 1) / BN;
+  const int total_tiles = m_tiles * n_tiles;
+  const int pair = static_cast<int>(cluster_id_x()), npairs = static_cast<int>(num_clusters_x());
+  const int k_iters = num_k + (r_steps > 0 ? 1 : 0);
+  int* status = p.status;
+  const uint64_t lim = p.wait_limit_ns;  // pipeline waits (teardown waits keep the full limit)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&decoded[s], kDecodedArrivals);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);  // 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(drain, 1);
+    mbar_init(drained, 1);
+    mbar_init(never, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      if (r_steps > 0) {
+        tma_prefetch_desc(&tmA2);
+        tma_prefetch_desc(&tmB2);
+      }
+      const uint32_t full0 = map_to_cta(&full[0], 0);
+      int it = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += npairs) {
+        int mb, nb;
+        pair_tile_coords(t, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
+        const int m0 = mb * 2 * BM + static_cast<int>(rank) * BM;
+        const int n0 = nb * BN + static_cast<int>(rank) * BNH;
+        for (int i = 0; i < k_iters; ++i, ++it) {
+          const int s = it % STAGES, u = it / STAGES;
+          if (it >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
+          if (i < num_k) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * A_TILE);
+            tma_load_2d_pair(sA + s * A_TILE, &tmA, fb, i * BK, m0);
+          } else if constexpr (!kBwd) {
+            // rank step: A2 = s U [M][64], B2 = LoRA B [N_w][r] (zero filled to 64)
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (A_TILE + B_TILE));
+            tma_load_2d_pair(sA + s * A_TILE, &tmA2, fb, 0, m0);
+            tma_load_2d_pair(sB + s * B_TILE, &tmB2, fb, 0, n0);
+          } else {
+            // rank step: A2 = s V [M][64], B2 = LoRA A [r][K_w] as MN-major boxes
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (A_TILE + (BNH / 64) * r_steps * 16 * 128));
+            tma_load_2d_pair(sA + s * A_TILE, &tmA2, fb, 0, m0);
+            for (int j = 0; j < BNH / 64; ++j)
+              tma_load_2d_pair(sB + s * B_TILE + j * 8192, &tmB2, fb, n0 + 64 * j, 0);
+          }
+        }
+      }
+      // Teardown: the copies into both CTAs' shared memory must have landed
+      // before either goes.  Every copy of a stage completes on the even
+      // CTA's copy barrier, so the even producer waits for the last stages
+      // it armed (both CTAs' bytes) and then tells the odd CTA, which waits
+      // for that word.  (Both producers wait on the same released stages, so
+      // they stop after the same number of issued stages.)
+      if (rank == 0) {
+        for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
+          mbar_wait_teardown(&full[i % STAGES], (i / STAGES) & 1, status);
+        mbar_arrive_cluster(map_to_cta(drained, 1));
+      } else {
+        mbar_wait_teardown(drained, 0, status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * BM, BN, kBwd);
+      int it = 0, tl = 0;
+      // Diagnostic launch: the issuer first waits on a barrier nothing
+      // arrives at, so its wait runs out and the whole pair takes the abort
+      // path (every other wait then ends on the abort flag or its own limit).
+      bool ok = !p.debug_stall || mbar_wait(never, 0, abort_flag, status, lim);
+      for (int t = pair; t < total_tiles && ok; t += npairs, ++tl) {
+        const int buf = tl & 1, use = tl >> 1;
+        if (use > 0 && !mbar_wait_cluster(&acc_empty[buf], (use - 1) & 1, abort_flag, status, lim)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN);
+        for (int i = 0; i < k_iters; ++i, ++it) {
+          const int s = it % STAGES, u = it / STAGES;
+          if (!mbar_wait_cluster(&full[s], u & 1, abort_flag, status, lim) ||
+              !mbar_wait_cluster(&decoded[s], u & 1, abort_flag, status, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nsteps = i < num_k ? BK / 16 : r_steps;
+          const uint64_t adesc = smem_desc_k128(smem_u32(sA + s * A_TILE));
+          const uint64_t bdesc = kBwd ? smem_desc_mn128(smem_u32(sB + s * B_TILE), 8192, 1024)
+                                      : smem_desc_k128(smem_u32(sB + s * B_TILE));
+          // One K = 16 step: A (K-major) +32 bytes inside the swizzle atom;
+          // B +32 bytes (K-major) or +2 atoms of 8 rows = 2048 bytes (MN-major).
+          const uint32_t bstep = kBwd ? (2048 >> 4) : 2;
+          for (int kk = 0; kk < nsteps; ++kk)
+            tc_mma_bf16_ss_pair(acc, adesc + 2 * kk, bdesc + bstep * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_commit_pair(&empty[s], 0x3);
+        }
+        if (ok) tc_commit_pair(&acc_full[buf], 0x3);
+      }
+      // Every MMA (which also reads the odd CTA's shared memory) must be
+      // complete before the pair's tensor memory and shared memory go.
+      tc_commit_pair(drain, 0x1);
+      mbar_wait_teardown(drain, 0, status);
+    }
+  } else if (warp < kFirstDecodeWarp) {
+    // Epilogue warps 2..5 own TMEM lane quadrants (warp % 4).
+    const int q = warp & 3;
+    const uint32_t acc_empty0 = map_to_cta(&acc_empty[0], 0);
+    int tl = 0;
+    for (int t = pair; t < total_tiles; t += npairs, ++tl) {
+      const int buf = tl & 1, use = tl >> 1;
+      const bool ok =
+          __all_sync(0xffffffffu, mbar_wait_cluster(&acc_full[buf], use & 1, abort_flag, status, lim) ? 1 : 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      int mb, nb;
+      pair_tile_coords(t, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
+      const int row = mb * 2 * BM + static_cast<int>(rank) * BM + q * 32 + lane;
+      const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(acc + c * 32, v);
+        tmem_wait_ld();
+        store_row32_bf16(v, p.D, row, nb * BN + c * 32, M, N, p.accumulate);
+      }
+      // Hand the accumulator buffer back to the even CTA's MMA thread.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * static_cast<uint32_t>(buf));
+    }
+  } else {
+    // Weight decoders.  Group g takes the pipeline iterations it with
+    // it % kDecodeGroups == g; thread `tid` writes one 128-byte row of the
+    // stage's B tile.
+    const int dw = warp - kFirstDecodeWarp;
+    const int grp = dw >> 2;
+    const int tid = ((dw & 3) << 5) | lane;
+    const uint32_t row_off = kBwd ? static_cast<uint32_t>((tid >> 6) * 8192 + (tid & 63) * 128)
+                                  : static_cast<uint32_t>(tid * 128);
+    const uint32_t sw = static_cast<uint32_t>(tid & 7);
+    float L[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) L[j] = codebook_level(p.codebook, j);
+    const bool fp32_scales = p.scale_format == kScalesFp32;
+    const float mu = fp32_scales ? 0.0f : __ldg(p.mu);
+    const int64_t kblocks = p.Kw / kBlock;
+    const uint32_t decoded0 = map_to_cta(&decoded[0], 0);
+    const uint32_t sB0 = smem_u32(sB);
+    const int my_tiles = pair < total_tiles ? (total_tiles - 1 - pair) / npairs + 1 : 0;
+    const int total_it = my_tiles * k_iters;
+
+    // The iterations of this group, in order: it = grp, grp + G, ...  Cursor
+    // (tl, i): tile tl of this pair, pipeline step i of that tile; the block
+    // index is recomputed from the tile's coordinates only when tl changes.
+    constexpr int G = kDecodeGroups;
+    struct Cursor {
+      int it, tl, i;
+      int64_t row_base;  // forward: first weight row of this CTA's half; backward: first output block
+    };
+    auto tile_base = [&](int tl) -> int64_t {
+      int mb, nb;
+      pair_tile_coords(pair + tl * npairs, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
+      return kBwd ? (static_cast<int64_t>(nb) * BN + static_cast<int64_t>(rank) * BNH) / kBlock
+                  : static_cast<int64_t>(nb) * BN + static_cast<int64_t>(rank) * BNH;
+    };
+    auto advance = [&](Cursor& c) {
+      c.it += G;
+      c.i += G;
+      if (c.i >= k_iters) {
+        while (c.i >= k_iters) {
+          c.i -= k_iters;
+          ++c.tl;
+        }
+        if (c.it < total_it) c.row_base = tile_base(c.tl);
+      }
+    };
+    // Block index this thread decodes at cursor c: >= 0 a block, -1 a row
+    // past the weight (written as zeros), -2 the rank step (nothing).
+    auto block_of = [&](const Cursor& c) -> int64_t {
+      if (c.i >= num_k) return -2;
+      if constexpr (!kBwd) {
+        const int64_t n = c.row_base + tid;
+        return n < p.Nw ? n * kblocks + c.i : -1;
+      } else {
+        const int64_t n = static_cast<int64_t>(c.i) * BK + (tid & 63);
+        const int64_t kb = c.row_base + (tid >> 6);
+        return (n < p.Nw && kb < kblocks) ? n * kblocks + kb : -1;
+      }
+    };
+
+    // One pipeline step of this group: prefetch the block of `ahead` (two
+    // steps later) into `nxt`, wait for the stage slot, decode `cur` into it,
+    // fence and signal.  The three register sets rotate by unrolling (no
+    // copies), so a load in flight is never waited on before its use.
+    bool ok = true;
+    auto step = [&](const Cursor& c, BlockLoad& cur, int64_t bc, const Cursor& ahead, BlockLoad& nxt,
+                    int64_t& bn) {
+      if (ahead.it < total_it) {
+        bn = block_of(ahead);
+        load_block(nxt, p, bn);
+      }
+      const int s = c.it % STAGES, u = c.it / STAGES;
+      if (c.it >= STAGES &&
+          __all_sync(0xffffffffu, mbar_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim) ? 1 : 0) == 0) {
+        ok = false;
+        return;
+      }
+      // Every stage gets this warp's arrival, the rank step too (its
+      // operands come by TMA), so the barrier's phases follow the slot's uses.
+      if (bc != -2) {
+        const uint32_t row = sB0 + static_cast<uint32_t>(s * B_TILE) + row_off;
+        if (bc >= 0) {
+          const float a = fp32_scales ? cur.x
+                                      : decode_scale_value(scale_code_value(p.scale_format, static_cast<int8_t>(cur.q)),
+                                                           cur.x, mu);
+          decode_block_to_smem(row, sw, cur.w, a, L);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) st_shared_v4(row + (static_cast<uint32_t>(j) << 4), 0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();  // these generic-proxy writes before the tensor core's reads
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(decoded0 + 8u * static_cast<uint32_t>(s));
+    };
+
+    if (grp < total_it) {
+      Cursor c0{grp, 0, grp, 0};
+      while (c0.i >= k_iters) {
+        c0.i -= k_iters;
+        ++c0.tl;
+      }
+      c0.row_base = tile_base(c0.tl);
+      Cursor c1 = c0;
+      advance(c1);
+      Cursor c2 = c1;
+      advance(c2);
+      BlockLoad b0, b1, b2;
+      int64_t k0 = block_of(c0), k1 = -2, k2 = -2;
+      load_block(b0, p, k0);
+      if (c1.it < total_it) {
+        k1 = block_of(c1);
+        load_block(b1, p, k1);
+      }
+      // c0 -> b0, c1 -> b1, c2 -> b2 (loaded by the first step)
+      while (true) {
+        step(c0, b0, k0, c2, b2, k2);
+        if (!ok || c1.it >= total_it) break;
+        advance(c0);
+        advance(c0);
+        advance(c0);  // c0 is now three steps ahead: the block after c2
+        step(c1, b1, k1, c0, b0, k0);
+        if (!ok || c2.it >= total_it) break;
+        advance(c1);
+        advance(c1);
+        advance(c1);
+        step(c2, b2, k2, c1, b1, k1);
+        if (!ok || c0.it >= total_it) break;
+        advance(c2);
+        advance(c2);
+        advance(c2);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the pair's MMAs are complete; no remote signal is in flight
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+namespace {
+
+template <bool kBwd>
+int query_nf4_clusters() {
+  if (cudaFuncSetAttribute(gemm_nf4_kernel<kBwd>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_nf4_kernel<kBwd>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  return n;
+}
+
+// Pair clusters of the decoding kernel that fit at once on the current device
+// (0: it cannot run there); sets the kernel's shared-memory limit on the
+// device as it first asks.
+template <bool kBwd>
+int nf4_pair_clusters(int dev) {
+  static DeviceValue cached;
+  return cached.get(dev, [] { return query_nf4_clusters<kBwd>(); });
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_nf4(const Nf4GemmArgs& a, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool bwd = a.backward != 0;
+  const int clusters = bwd ? nf4_pair_clusters<true>(dev) : nf4_pair_clusters<false>(dev);
+  if (clusters <= 0) return cudaErrorNotSupported;
+  const WeightView& w = a.w;
+  // GEMM view: D [M][N] = A [M][K] op(W_hat) + A2 B2
+  const int64_t N = bwd ? w.cols : w.rows;
+  const int64_t K = bwd ? w.rows : w.cols;
+  CUtensorMap tA, tA2, tB2;
+  if (!encode_tensor_map_2d(&tA, a.A, a.M, K, BM, BK)) return cudaErrorInvalidValue;
+  int r_steps = 0;
+  if (a.A2 != nullptr && a.r > 0) {
+    r_steps = (a.r + 15) / 16;
+    if (!encode_tensor_map_2d(&tA2, a.A2, a.M, kRankPad, BM, BK)) return cudaErrorInvalidValue;
+    if (bwd) {
+      // LoRA A [r][K_w]: boxes of 16 * r_steps rows x 64 columns (MN-major B2)
+      if (!encode_tensor_map_2d(&tB2, a.B2, a.r, N, static_cast<uint32_t>(16 * r_steps), 64))
+        return cudaErrorInvalidValue;
+    } else {
+      // LoRA B [N_w][ldb2] with r valid columns, zero filled to 64
+      if (!encode_tensor_map_2d(&tB2, a.B2, N, a.r, BNH, BK, true, a.ldb2)) return cudaErrorInvalidValue;
+    }
+  } else {
+    tA2 = tA;
+    tB2 = tA;
+  }
+  Nf4GemmParams p{};
+  p.packed = w.packed;
+  p.qscale = w.qscale;
+  p.c2 = w.c2;
+  p.mu = w.mu;
+  p.absmax = w.absmax;
+  p.codebook = w.codebook;
+  p.scale_format = w.scale_format;
+  p.Nw = w.rows;
+  p.Kw = w.cols;
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(N);
+  p.num_k = static_cast<int>((K + BK - 1) / BK);
+  p.r_steps = r_steps;
+  p.D = a.D;
+  p.accumulate = a.accumulate;
+  p.status = a.status;
+  p.wait_limit_ns = a.wait_limit_ns ? a.wait_limit_ns : kWaitLimitNs;
+  p.debug_stall = a.debug_stall;
+  const int64_t m_tiles = (a.M + 2 * BM - 1) / (2 * BM), n_tiles = (N + BN - 1) / BN;
+  const int64_t tiles = m_tiles * n_tiles;
+  const int pairs = static_cast<int>(tiles < clusters ? tiles : clusters);
+  // HBM bytes of one 256-wide panel: A (bf16 activations) 2 B per value;
+  // the weight 0.5 B of codes + 1/64 B of scale codes per value.
+  const double a_panel = 256.0 * static_cast<double>(K) * 2.0;
+  const double b_panel = 256.0 * static_cast<double>(K) * (0.5 + 1.0 / 64.0);
+  const RasterChoice rc = choose_raster(m_tiles, n_tiles, a_panel, b_panel, static_cast<double>(kL2PanelBudget));
+  p.group = rc.group;
+  p.along_n = rc.along_n;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (bwd) return cudaLaunchKernelEx(&cfg, gemm_nf4_kernel<true>, tA, tA2, tB2, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nf4_kernel<false>, tA, tA2, tB2, p);
+}
+
+}  // namespace qnf4

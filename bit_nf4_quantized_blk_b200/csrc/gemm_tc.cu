@@ -19,8 +19,17 @@
 //   warps 2-5   epilogue: tcgen05.ld 32 columns at a time -> bf16 -> global
 // Every barrier wait is bounded (see common.cuh); a timeout aborts the CTA,
 // which then waits (bounded) for its copies and MMAs in flight and frees its
-// tensor memory before returning.  No cluster multicast is used.
+// tensor memory before returning.  No TMA or bulk load uses cluster
+// multicast: every CTA loads its own tiles.  The pair kernel's
+// tcgen05.commit does carry .multicast::cluster, which is an mbarrier arrive
+// delivered to both CTAs of the pair on this GPU, not a load.
+//
+// These kernels read a dense bf16 weight (the dequantized copy).  The linear
+// calls use them for the dense-weight ablation arm and as the fallback where
+// pair clusters cannot be scheduled; the default path is gemm_nf4.cu, which
+// decodes the 4-bit weight inside the GEMM.
 #include "common.cuh"
+#include "gemm_common.cuh"
 #include "kernels.cuh"
 
 namespace qnf4 {
@@ -236,41 +245,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(acc + c * 32, v);
         tmem_wait_ld();
-        const int col = nb * BN + c * 32;
-        if (row >= M || col >= N) continue;
-        uint16_t* dst = D + static_cast<int64_t>(row) * N + col;
-        if (col + 32 <= N) {
-          uint32_t pk[16];
-          if (accumulate) {
-            const uint4* old = reinterpret_cast<const uint4*>(dst);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const uint4 o = old[q4];
-              const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int idx = q4 * 8 + e * 2;
-                pk[q4 * 4 + e] = pack_bf16x2(__uint_as_float(v[idx]) + bf16_bits_to_float(ow[e] & 0xFFFF),
-                                             __uint_as_float(v[idx + 1]) + bf16_bits_to_float(ow[e] >> 16));
-              }
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-          }
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (col + e < N) {
-              float val = __uint_as_float(v[e]);
-              if (accumulate) val += bf16_bits_to_float(dst[e]);
-              dst[e] = static_cast<uint16_t>(pack_bf16x2(val, 0.0f) & 0xFFFF);
-            }
-          }
-        }
+        store_row32_bf16(v, D, row, nb * BN + c * 32, M, N, accumulate);
       }
       // Hand the accumulator buffer back to the MMA warp.
       tc_fence_before();
@@ -311,20 +286,6 @@ constexpr int B_TILE2 = BNH * BK * 2;    // 16 KB
 constexpr size_t kL2PanelBudget = size_t(48) << 20;  // bytes of operand panels kept resident per group
 constexpr int SMEM2_BYTES = 1024 + STAGES2 * (A_TILE2 + B_TILE2) + 512;
 }  // namespace
-
-// Tile order of the pair kernel: groups of `group` consecutive tiles along M
-// (along_n = 0) or N (along_n = 1) sweep the other dimension, so the panels of
-// one group stay in L2 while the other operand streams past once per group.
-__device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles, int group, int along_n, int& mb,
-                                                 int& nb) {
-  const int g_tiles = along_n ? n_tiles : m_tiles, o_tiles = along_n ? m_tiles : n_tiles;
-  const int per_group = group * o_tiles;
-  const int gi = t / per_group, first = gi * group;
-  const int gsize = min(group, g_tiles - first), local = t - gi * per_group;
-  const int gpos = first + local % gsize, opos = local / gsize;
-  mb = along_n ? opos : gpos;
-  nb = along_n ? gpos : opos;
-}
 
 template <bool kBMN>
 __global__ void __launch_bounds__(192, 1)
@@ -488,41 +449,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(acc + c * 32, v);
         tmem_wait_ld();
-        const int col = nb * BN2 + c * 32;
-        if (row >= M || col >= N) continue;
-        uint16_t* dst = D + static_cast<int64_t>(row) * N + col;
-        if (col + 32 <= N) {
-          uint32_t pk[16];
-          if (accumulate) {
-            const uint4* old = reinterpret_cast<const uint4*>(dst);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const uint4 o = old[q4];
-              const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int idx = q4 * 8 + e * 2;
-                pk[q4 * 4 + e] = pack_bf16x2(__uint_as_float(v[idx]) + bf16_bits_to_float(ow[e] & 0xFFFF),
-                                             __uint_as_float(v[idx + 1]) + bf16_bits_to_float(ow[e] >> 16));
-              }
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-          }
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (col + e < N) {
-              float val = __uint_as_float(v[e]);
-              if (accumulate) val += bf16_bits_to_float(dst[e]);
-              dst[e] = static_cast<uint16_t>(pack_bf16x2(val, 0.0f) & 0xFFFF);
-            }
-          }
-        }
+        store_row32_bf16(v, D, row, nb * BN2 + c * 32, M, N, accumulate);
       }
       // Hand the accumulator buffer back to the even CTA's MMA thread.
       tc_fence_before();
@@ -583,16 +510,10 @@ cudaError_t launch_pair(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
   const int64_t m_tiles = (a.M + 2 * BM2 - 1) / (2 * BM2), n_tiles = (a.N + BN2 - 1) / BN2;
   const int64_t tiles = m_tiles * n_tiles;
   const int pairs = static_cast<int>(tiles < clusters ? tiles : clusters);
-  // A 256-wide panel of either operand holds 256 x K bf16.  Group as many
-  // panels as the L2 budget keeps resident, along the dimension that makes
-  // the other operand's re-reads fewest: traffic ~ own + other * ceil(own / group).
-  const size_t panel = size_t(256) * static_cast<size_t>(a.K) * 2;
-  const int64_t fit = static_cast<int64_t>(kL2PanelBudget / panel) > 1 ? static_cast<int64_t>(kL2PanelBudget / panel) : 1;
-  const int64_t gm = fit < m_tiles ? fit : m_tiles, gn = fit < n_tiles ? fit : n_tiles;
-  const int64_t traffic_m = m_tiles + n_tiles * ((m_tiles + gm - 1) / gm);
-  const int64_t traffic_n = n_tiles + m_tiles * ((n_tiles + gn - 1) / gn);
-  const int along_n = traffic_n < traffic_m ? 1 : 0;
-  const int group = static_cast<int>(along_n ? gn : gm);
+  // A 256-wide panel of either operand holds 256 x K bf16.
+  const double panel = 256.0 * static_cast<double>(a.K) * 2.0;
+  const RasterChoice rc = choose_raster(m_tiles, n_tiles, panel, panel, static_cast<double>(kL2PanelBudget));
+  const int group = rc.group, along_n = rc.along_n;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
   cfg.blockDim = dim3(192);

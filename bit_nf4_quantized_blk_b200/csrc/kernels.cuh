@@ -170,6 +170,18 @@ size_t colsum_partial_bytes(int64_t M, int64_t C);
 cudaError_t launch_colsum(const uint16_t* In, int64_t M, int64_t C, const uint16_t* hi, const uint16_t* lo, int r,
                           float scale, float* part, float* dst, bool dst_rc, int* status, cudaStream_t stream);
 
+// Both rank-r products of the backward from one pass over G = dY [M][N]:
+// V = G B written as vs = s*V (bf16 [M][64]) and its hi / lo split (vhi,
+// vlo, [M][64]); dB = scale * G^T (uhi + ulo) into dB [N][r] (may be null).
+// B is [N][ldb] bf16 with r valid columns (ldb * 2 bytes a multiple of 16).
+// `part` is scratch of vdb_partial_bytes(M, N).  Ranks 1..kVdbMaxRank (wider
+// ranks use launch_skinny + launch_colsum).
+constexpr int kVdbMaxRank = 16;
+size_t vdb_partial_bytes(int64_t M, int64_t N);
+cudaError_t launch_vdb(const uint16_t* G, int64_t M, int64_t N, const uint16_t* B, int64_t ldb, const uint16_t* uhi,
+                       const uint16_t* ulo, int r, float scale, float* part, uint16_t* vs, uint16_t* vhi,
+                       uint16_t* vlo, float* dB, int* status, cudaStream_t stream);
+
 // Copy a bf16 [rows][r] matrix into [rows][64] zero padded, optionally from
 // the transposed source [r][rows].
 cudaError_t launch_pad_rank(const uint16_t* src, bool src_transposed, int64_t rows, int r, uint16_t* dst,
@@ -192,6 +204,52 @@ struct GemmArgs {
   int64_t ldb, ldb2;   // row pitches (elements) of K-major B / B2 (0: dense)
 };
 cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// tcgen05 GEMM with the 4-bit weight decoded in the kernel (gemm_nf4.cu):
+//   forward   D [M][N_w] = A [M][K_w] W_hat^T + A2 [M][64] B2^T  (B2 = LoRA B [N_w][ldb2])
+//   backward  D [M][K_w] = A [M][N_w] W_hat   + A2 [M][64] B2    (B2 = LoRA A [r][K_w])
+// ---------------------------------------------------------------------------
+struct Nf4GemmArgs {
+  WeightView w;
+  const uint16_t* A;   // X (forward) or dY (backward), bf16 row-major
+  const uint16_t* A2;  // [M][64] bf16 s*U or s*V, zero padded beyond r; null: no rank step
+  const uint16_t* B2;  // see above
+  int64_t M;
+  int r;
+  int64_t ldb2;        // row pitch (elements) of the forward's B2
+  uint16_t* D;
+  int accumulate;      // D += ... instead of D = ...
+  int* status;
+  int backward;        // 0: forward, 1: backward-input
+  // Diagnostics (zero in every product call): a wait limit for the pipeline
+  // waits (0: the default one second) and debug_stall = 1 to hold the MMA
+  // issuer on a barrier nothing arrives at, so the abort path runs.
+  uint64_t wait_limit_ns;
+  int debug_stall;
+};
+
+// Kernel parameters (the launcher fills them from Nf4GemmArgs).
+struct Nf4GemmParams {
+  const uint8_t* packed;
+  const int8_t* qscale;
+  const float* c2;
+  const float* mu;
+  const float* absmax;
+  int codebook, scale_format;
+  int64_t Nw, Kw;      // weight [N_w][K_w]
+  int M, N, num_k, r_steps;
+  uint16_t* D;
+  int accumulate;
+  int* status;
+  int group, along_n;  // tile raster
+  uint64_t wait_limit_ns;
+  int debug_stall;
+};
+
+// Returns cudaErrorNotSupported when pair clusters of the kernel cannot be
+// scheduled on the current device (the caller then takes the dense path).
+cudaError_t launch_gemm_nf4(const Nf4GemmArgs& a, cudaStream_t stream);
 
 // Driver entry point used to encode TMA descriptors (resolved once).
 bool encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,

@@ -280,12 +280,39 @@ qlora_status qlora_workspace_status(void *ws, size_t ws_bytes, void *stream);
 /*
  * Workspace bytes for qlora_linear_fwd / qlora_linear_bwd at tokens M,
  * weight [N, K] and rank r (the larger of the two needs; one workspace may
- * serve both).  Returns 0 for sizes the linear calls refuse: M < 1, N not a
+ * serve both) under the weight path in force (qlora_linear_set_weight_path).
+ * Returns 0 for sizes the linear calls refuse: M < 1, N not a
  * positive multiple of 8, K not a positive multiple of 64, r outside 1..64,
  * or beyond the limits M <= 2^25, N and K < 2^31, N * K <= 2^40 (for
  * which the calls return QLORA_ERR_UNSUPPORTED).
  */
 size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
+
+/*
+ * Weight path of the tensor-core linear calls (M > 16).
+ *   QLORA_WEIGHT_PATH_FUSED (default): the GEMM decodes the packed 4-bit
+ *     weight and its block scales straight into its shared-memory operand
+ *     tiles ("QLoRA Deep Dive: 4-bit NormalFloat & Double Quantization
+ *     Internals", section "The Quantization Process in QLoRA": a block is
+ *     multiplied back by its constant and used in the computation; "FT-02:
+ *     QLoRA -- Fine-Tuning with Quantization", section "Reading the result:
+ *     the three lines that decide memory": the weight stays in 4 bits and is
+ *     dequantized on the fly).  No dense copy of the weight is written.
+ *   QLORA_WEIGHT_PATH_DENSE: the ablation arm.  Each tensor-core call first
+ *     dequantizes the whole weight to bf16 in the workspace (N * K * 2 more
+ *     workspace bytes) and then runs a GEMM that reads that copy.
+ * Both paths decode the same bf16 values and accumulate in the same order,
+ * so their outputs are bit-identical.  The setting is process-wide; each
+ * call reads it once.  qlora_linear_ws_bytes answers for the path in force
+ * when it is called: a call on the dense path with a workspace sized for the
+ * fused path returns QLORA_ERR_WORKSPACE.  A fused call on a device where
+ * its kernel cannot be scheduled returns QLORA_ERR_UNSUPPORTED.
+ *   qlora_linear_set_weight_path : INVALID_ARG for an unknown value.
+ *   qlora_linear_weight_path     : the path in force.
+ */
+typedef enum qlora_weight_path { QLORA_WEIGHT_PATH_FUSED = 0, QLORA_WEIGHT_PATH_DENSE = 1 } qlora_weight_path;
+qlora_status qlora_linear_set_weight_path(int32_t path);
+int32_t qlora_linear_weight_path(void);
 
 /*
  * LoRA linear forward:  Y = X W^T + scale * (X A^T) B^T.
@@ -301,6 +328,25 @@ size_t qlora_linear_ws_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
 qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t M, const uint16_t *A,
                               const uint16_t *B, int32_t r, float scale, uint16_t *Y, float *U_out, void *ws,
                               size_t ws_bytes, void *stream);
+
+/*
+ * Diagnostic of the bounded device waits (the pages have no counterpart: it
+ * checks this library's failure detection, not a step of the method).
+ * Runs the tensor-core forward of qlora_linear_fwd (M > 16, the fused weight
+ * path) with the GEMM's MMA issuer first waiting on a barrier that nothing
+ * arrives at, and every pipeline wait of the GEMM limited to wait_limit_us
+ * microseconds (1 .. 1,000,000).  That wait runs out; the GEMM records
+ * QLORA_ERR_TIMEOUT in the workspace status, every warp leaves its loop,
+ * the copies already issued are waited for, tensor memory is freed and the
+ * kernel returns, so the device and the stream stay usable.  Y is left
+ * unspecified.  Returns QLORA_OK once enqueued (INVALID_ARG for M <= 16 or a
+ * limit out of range); read the outcome with qlora_workspace_status.  The
+ * other arguments are those of qlora_linear_fwd (no U output).
+ */
+qlora_status qlora_linear_fwd_stall_diagnostic(const qlora_nf4_weight *w, const uint16_t *X, int64_t M,
+                                               const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                                               uint16_t *Y, void *ws, size_t ws_bytes, int32_t wait_limit_us,
+                                               void *stream);
 
 /*
  * LoRA linear backward for upstream gradient dY of Y.

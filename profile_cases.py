@@ -1,21 +1,26 @@
-"""Bounded single-kernel cases for profiler captures.
+"""Bounded single-kernel cases for profiler captures (a harness beside
+``bench.py``, not part of the library package).
 
-``python -m bit_nf4_quantized_blk_b200.profile_cases --case gemm --reps 3``
-sets up one realistic case (inputs larger than L2, a few hundred MB on the
+``python profile_cases.py --case gemm --reps 3`` sets up one realistic case (inputs larger than L2, a few hundred MB on the
 device at most), runs the library call ``reps`` times and exits; a profiler
 pointed at it with a kernel filter and a launch count captures the kernel of
 interest.  The cases use the 7B gate projection (14336 x 4096) at 8192
 tokens, the decode shape (16 tokens) for the GEMV, and the bf16 merged
-weight (r = 16) for the merge.
+weight (r = 16) for the merge.  ``--path dense`` runs the tensor-core calls on
+the dense-weight ablation path instead of the default fused one.
 """
 
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import torch
 
-from bit_nf4_quantized_blk_b200 import binding, workloads
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+from bit_nf4_quantized_blk_b200 import binding, workloads  # noqa: E402
 
 CASES = ("gemm", "gemm_bwd", "quantize", "dequant", "gemv", "side", "merge")
 
@@ -25,8 +30,11 @@ def main():
     ap.add_argument("--case", choices=CASES, required=True)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--tokens", type=int, default=8192)
+    ap.add_argument("--path", choices=("fused", "dense"), default="fused")
     args = ap.parse_args()
     torch.cuda.set_device(0)
+    binding.qlora_linear_set_weight_path(
+        binding.WEIGHT_PATH_DENSE if args.path == "dense" else binding.WEIGHT_PATH_FUSED)
     M = 16 if args.case in ("gemv", "merge") else args.tokens
     case = workloads.linear_case(workloads.GATE7B, M, 16, 32.0, 4, 0, 4, device="cuda", with_dy=args.case not in ("gemv", "merge"))
     out = binding.NF4Weight.empty(case.proj.n, case.proj.k)

@@ -70,8 +70,17 @@ def test_sizes(lib):
 
 
 def test_linear_ws_bytes(lib):
-    assert binding.qlora_linear_ws_bytes(16, 1024, 1024, 8) > 1024 * 1024 * 2
-    assert binding.qlora_linear_ws_bytes(8192, 14336, 4096, 16) > 14336 * 4096 * 2
+    assert binding.qlora_linear_weight_path() == binding.WEIGHT_PATH_FUSED  # the default
+    # the fused path holds no dense copy of the weight; the dense-weight
+    # ablation path adds one of N x K bf16 for the tensor-core calls (M > 16)
+    fused = binding.qlora_linear_ws_bytes(8192, 14336, 4096, 16)
+    assert 0 < fused < 14336 * 4096
+    with binding.weight_path(binding.WEIGHT_PATH_DENSE):
+        assert binding.qlora_linear_ws_bytes(8192, 14336, 4096, 16) >= fused + 14336 * 4096 * 2
+        decode_dense = binding.qlora_linear_ws_bytes(16, 1024, 1024, 8)
+    assert binding.qlora_linear_weight_path() == binding.WEIGHT_PATH_FUSED
+    # M <= 16: the forward is the GEMV, but the backward's GEMM still reads the copy on the dense path
+    assert decode_dense >= binding.qlora_linear_ws_bytes(16, 1024, 1024, 8) + 1024 * 1024 * 2
     assert binding.qlora_linear_ws_bytes(0, 1024, 1024, 8) == 0
     assert binding.qlora_linear_ws_bytes(16, 1024, 1000, 8) == 0
     assert binding.qlora_linear_ws_bytes(16, 1024, 1024, 65) == 0
@@ -80,6 +89,17 @@ def test_linear_ws_bytes(lib):
     assert binding.qlora_linear_ws_bytes(2**25 + 1, 8, 64, 8) == 0
     assert binding.qlora_linear_ws_bytes(16, 2**33, 64, 8) == 0  # N beyond 32-bit indices
     assert binding.qlora_linear_ws_bytes(16, 8, 2**31, 8) == 0  # K likewise
+
+
+def test_weight_path_selector(lib):
+    L = binding.lib()
+    assert L.qlora_linear_set_weight_path(2) == 1  # QLORA_ERR_INVALID_ARG
+    assert L.qlora_linear_set_weight_path(-1) == 1
+    assert L.qlora_linear_weight_path() == binding.WEIGHT_PATH_FUSED
+    assert L.qlora_linear_set_weight_path(binding.WEIGHT_PATH_DENSE) == 0
+    assert L.qlora_linear_weight_path() == binding.WEIGHT_PATH_DENSE
+    assert L.qlora_linear_set_weight_path(binding.WEIGHT_PATH_FUSED) == 0
+    assert L.qlora_linear_weight_path() == binding.WEIGHT_PATH_FUSED
 
 
 def test_linear_size_limits_refused_on_the_host(lib):

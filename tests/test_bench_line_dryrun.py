@@ -4,8 +4,9 @@ Every GPU-touching piece (the layer step, the timed loop, the library's
 timing records, the clock sampler and the secondary measurements) is a fake
 returning fixed numbers, so the test checks the line's assembly: every key
 of the measurement contract is present with the right type, the roofline and
-whole-job figures follow from the fakes' numbers, and the opt-in flags add
-their fields without changing the rest.
+whole-job figures follow from the fakes' numbers, the default run carries the
+32-layer stack row, and the flags add or drop their fields without changing
+the rest.
 """
 
 import argparse
@@ -52,6 +53,10 @@ class FakeClock:
     def stop(self, window):
         return {"sm_mhz": 1650.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 10}
 
+    @staticmethod
+    def around(device_index, fn):
+        return fn(), {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 4}
+
 
 @pytest.fixture
 def dry(monkeypatch):
@@ -85,9 +90,11 @@ def dry(monkeypatch):
     monkeypatch.setattr(binding, "qlora_timing_enable", lambda on: None)
     monkeypatch.setattr(binding, "qlora_timing_read", timing_read)
     monkeypatch.setattr(torch.cuda, "empty_cache", lambda: None)
-    monkeypatch.setattr(bench, "bench_quantize_dequant", lambda: {
+    monkeypatch.setattr(bench, "bench_quantize_dequant", lambda clock=None: {
         "quantize": {"ms": 1.0, "GB/s": 5000.0}, "dequant_bf16": {"ms": 1.0, "GB/s": 6000.0}})
-    monkeypatch.setattr(bench, "bench_gemv", lambda: {"M=1": {"us": 25.0, "GB/s": 1200.0}})
+    monkeypatch.setattr(bench, "bench_gemv", lambda: {"M=1": {"us": 25.0, "GB/s": 1200.0,
+                                                             "write_flush": {"us": 30.0, "GB/s": 1000.0}},
+                                                     "method": "rotation"})
     monkeypatch.setattr(bench, "bench_merge", lambda: {"ms": 0.2, "GB/s": 2700.0})
     monkeypatch.setattr(bench, "bench_stack", lambda: {"quantize": {"ms": 6.0, "GB/s": 5200.0},
                                                       "fwd_bwd": {"ms": 250.0, "TFLOP/s": 920.0}})
@@ -98,7 +105,7 @@ def dry(monkeypatch):
 
 
 def _args(**kw):
-    base = dict(gpus=1, steps=5, warmup=3, impl="ours", no_extras=False, no_cpu=False, streams=1, stack=False)
+    base = dict(gpus=1, steps=5, warmup=3, impl="ours", no_extras=False, no_cpu=False, streams=1, no_stack=False)
     base.update(kw)
     return argparse.Namespace(**base)
 
@@ -126,6 +133,8 @@ def test_default_line_has_every_contract_key(dry, capsys):
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(bench.gemm_flops_per_step() / (GEMM_MS_PER_STEP / 1e3) / 1e12)
     assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+    assert r["peak"] == bench.load_peaks()[0].get("bf16_tflops", bench.FALLBACK_PEAKS["bf16_tflops"])  # burst
+    assert r["frac_clock_normalized"] == pytest.approx(r["achieved"] / (r["peak"] * 1650.0 / r["peak_clock_mhz"]))
     cb = d["cpu_baseline"]
     for key in ("value", "unit", "cores", "kind", "sample", "cpu_model", "nproc", "secondary"):
         assert key in cb, key
@@ -135,15 +144,17 @@ def test_default_line_has_every_contract_key(dry, capsys):
         assert key in e, key
     assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert d["gpu_launches"] == (14 + 4 * 10) * 5
-    assert "secondary" in d and "stack_32x7_8192tok" not in d["secondary"]
+    st = d["secondary"]["stack_32x7_8192tok"]  # config 5 is part of the default run
+    assert "frac_hbm" in st["quantize"] and "frac_bf16_burst" in st["fwd_bwd"] and st["clocks"]["samples"] == 4
+    g = d["secondary"]["gemv_gate_14336x4096"]["M=1"]
+    assert "frac_hbm" in g and "frac_hbm" in g["write_flush"]
     assert dry["step"].runs == 1 + 3 + 5 and dry["step"].two_stream_runs == 0
 
 
-def test_opt_in_flags(dry, capsys):
-    d = _line(capsys, _args(streams=2, stack=True, no_cpu=True, no_extras=True))
+def test_flags(dry, capsys):
+    d = _line(capsys, _args(streams=2, no_stack=True, no_cpu=True, no_extras=True))
     assert d["config"]["streams"].startswith("projections alternate")
-    st = d["secondary"]["stack_32x7_8192tok"]
-    assert "frac_hbm" in st["quantize"] and "frac_bf16_sustained" in st["fwd_bwd"]
+    assert "stack_32x7_8192tok" not in d.get("secondary", {})
     assert "cpu_baseline" not in d
     assert dry["step"].two_stream_runs == 3 + 5 and dry["step"].runs == 1
 

@@ -155,3 +155,107 @@ def test_opt13b_shapes_full_batch():
         st = nf4.quantize_weight(Ws[i].cpu().numpy())
         want = nf4.dequantize_weight(st, "bf16")
         assert np.array_equal(ys[i].view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+def test_dq_rounding_ties_bit_exact():
+    """Block scales whose deviations land exactly on rounding ties of the
+    int8 scale codes (a chunk of 256 scales 256 +- d, d = 127 and every
+    k + 1/2): the kernel rounds them to even like the oracle (0.5 -> 0,
+    1.5 -> 2, 2.5 -> 2).  Each block's absmax is its first weight, with either
+    sign; the other weights are smaller random values."""
+    d = np.array([127.0] + [k + 0.5 for k in range(127)], np.float32)
+    a = np.empty(256, np.float32)
+    a[0::2] = np.float32(256.0) + d
+    a[1::2] = np.float32(256.0) - d
+    rng = np.random.default_rng(41)
+    W = (rng.uniform(-0.9, 0.9, (256, 64)) * a[:, None]).astype(np.float32)
+    W[:, 0] = a * np.where(np.arange(256) % 3 == 0, -1.0, 1.0).astype(np.float32)
+    st = nf4.quantize_weight(W)
+    assert st.mu == np.float32(256.0) and st.c2[0] == np.float32(127.0)
+    out = gpu_quantize(torch.from_numpy(W))
+    assert_state_equal(out, st, "DQ ties")
+    q = out.qscale.cpu().numpy()
+    assert [int(v) for v in q[2:8]] == [0, 0, 2, -2, 2, -2]
+
+
+def _adversarial_absmax(rng) -> np.ndarray:
+    """Block absmax values away from 1: log-uniform random ones over most of
+    the fp32 range, the fp32 neighbours of powers of two, values around both
+    ends of the kernel's reciprocal fast range (2^-121 and 2^119), subnormal
+    and tiny ones (the IEEE-division path), and the largest finite values."""
+    f = np.float32
+    vals = list((2.0 ** rng.uniform(-120.0, 118.0, 1500)).astype(f))
+    for e in rng.integers(-125, 127, 200):
+        p = f(2.0 ** int(e))
+        vals += [np.nextafter(p, f(0)), p, np.nextafter(p, f(np.inf)), f(p * f(1.0 + 3 * 2.0 ** -23))]
+    for edge in (f(2.0 ** -121), f(2.0 ** 119)):
+        x = edge
+        for _ in range(12):
+            x = np.nextafter(x, f(0))
+        for _ in range(25):
+            vals.append(x)
+            x = np.nextafter(x, f(np.inf))
+        vals += list((edge * (1.0 + rng.uniform(-0.01, 0.01, 40))).astype(f))
+    vals += [f(2.0 ** -130), f(2.0 ** -140), f(7 * 2.0 ** -149), f(3e38), np.finfo(f).max, f(2.0 ** -126)]
+    a = np.array(vals, dtype=f)
+    return a[(a > 0) & np.isfinite(a)]
+
+
+def _adversarial_weight(codebook: str, seed: int) -> np.ndarray:
+    """Blocks whose weights sit on the kernel's decision edges for their block
+    absmax a (one weight of magnitude a, random sign and position, per
+    block): fl32(T_j a) and its fp32 neighbours up to 3 ulps either side, and
+    fl32(T_j a (1 +- 2^-19)) +- 1 ulp, the edges of the band inside which the
+    kernel recodes from the IEEE quotient.  Blocks are padded with uniform
+    weights in (-a, a)."""
+    f = np.float32
+    rng = np.random.default_rng(seed)
+    T = nf4.decision_thresholds(codebook).astype(np.float64)
+    blocks = []
+    for a in _adversarial_absmax(rng):
+        cand = []
+        for t in T:
+            c = f(t * float(a))
+            lo = hi = c
+            cand.append(c)
+            for _ in range(3):
+                lo, hi = np.nextafter(lo, f(-np.inf)), np.nextafter(hi, f(np.inf))
+                cand += [lo, hi]
+            for rel in (1.0 - 2.0 ** -19, 1.0 + 2.0 ** -19):
+                e = f(t * float(a) * rel)
+                cand += [np.nextafter(e, f(-np.inf)), e, np.nextafter(e, f(np.inf))]
+        cand = np.array(cand, dtype=f)
+        cand = cand[np.abs(cand) <= a]
+        per = 63
+        nb = -(-cand.size // per)
+        pad = (rng.uniform(-1.0, 1.0, nb * per - cand.size) * float(a)).astype(f)
+        body = np.concatenate([cand, pad]).reshape(nb, per)
+        for row in body:
+            pos = int(rng.integers(0, 64))
+            sign = f(-1.0) if rng.integers(0, 2) else f(1.0)
+            blocks.append(np.insert(row, pos, sign * a))
+    W = np.stack(blocks).astype(f)
+    assert np.isfinite(W).all()
+    return W
+
+
+@pytest.mark.parametrize("codebook,scales", [("nf4", "dq_int8"), ("fp4", "dq_int8"), ("nf4", "fp32")])
+def test_decision_edges_at_block_scales_away_from_one(codebook, scales):
+    """Bit-exact codes (and the rest of the state) where the reciprocal fast
+    path is closest to being wrong: the block absmax is not a power of two
+    (or sits at the ends of the fast range) and the weights lie on and next
+    to every decision threshold and band edge."""
+    W = _adversarial_weight(codebook, 17 if codebook == "nf4" else 18)
+    # self-check of the construction: many weights normalise to within 2 ulps of a threshold
+    a = np.abs(W).max(axis=1, keepdims=True)
+    x = (W / a).astype(np.float32)
+    T = nf4.decision_thresholds(codebook)
+    near = np.zeros(x.shape, bool)
+    for t in T:
+        near |= np.abs(x.astype(np.float64) - float(t)) <= 2.0 * float(np.spacing(np.float32(abs(t))))
+    assert near.sum() > 100_000 if codebook == "nf4" else near.sum() > 50_000
+    cb = binding.CODEBOOK_NF4 if codebook == "nf4" else binding.CODEBOOK_FP4
+    sf = binding.SCALES_DQ_INT8 if scales == "dq_int8" else binding.SCALES_FP32
+    st = nf4.quantize_weight(W, codebook=codebook, scale_format=scales)
+    out = gpu_quantize(torch.from_numpy(W), cb, sf)
+    assert_state_equal(out, st, f"decision edges {codebook} {scales}")
