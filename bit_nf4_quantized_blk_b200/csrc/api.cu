@@ -345,7 +345,7 @@ int64_t max_group_chunks(const qlora_nf4_weight* outs, int32_t count) {
 
 // Linear workspace layout.
 struct LinearWs {
-  size_t wbf, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, vdbpart, gu, gy, total;
+  size_t wbf, scales, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, vdbpart, gu, gy, total;
 };
 
 LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, bool dense) {
@@ -360,6 +360,8 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, bool dense) {
   // The dense bf16 copy of the weight exists only on the dense-weight path
   // (the backward's GEMM runs at every M).
   l.wbf = take(dense ? static_cast<size_t>(N) * static_cast<size_t>(K) * 2 : 0);
+  // Decoded block scales for the fused GEMM's tile producer (1/16 B per weight).
+  l.scales = take(dense ? 0 : static_cast<size_t>(N) * static_cast<size_t>(block_scales_ld(K)) * sizeof(float));
   l.us = take(mr * 2);
   l.uhi = take(mr * 2);
   l.ulo = take(mr * 2);
@@ -440,11 +442,17 @@ qlora_status check_linear_args(const qlora_nf4_weight* w, int64_t M, int32_t r, 
 }
 
 // The 4-bit weight decoded inside the tensor-core GEMM.
-cudaError_t launch_linear_gemm_nf4(const qlora_nf4_weight* w, const uint16_t* A, int64_t M, const uint16_t* A2,
-                                   const uint16_t* B2, int r, int64_t ldb2, uint16_t* D, int accumulate, int* status,
-                                   bool backward, cudaStream_t s, uint64_t wait_limit_ns = 0, int debug_stall = 0) {
+// The 4-bit weight decoded inside the tensor-core GEMM; its decoded block
+// scales (`scales`, workspace) are written first by a small pre-pass.
+cudaError_t launch_linear_gemm_nf4(const qlora_nf4_weight* w, float* scales, const uint16_t* A, int64_t M,
+                                   const uint16_t* A2, const uint16_t* B2, int r, int64_t ldb2, uint16_t* D,
+                                   int accumulate, int* status, bool backward, cudaStream_t s,
+                                   uint64_t wait_limit_ns = 0, int debug_stall = 0) {
+  cudaError_t e = launch_block_scales(view_of(w), scales, s);
+  if (e != cudaSuccess) return e;
   Nf4GemmArgs g{};
   g.w = view_of(w);
+  g.scales = scales;
   g.A = A;
   g.A2 = A2;
   g.B2 = B2;
@@ -777,8 +785,8 @@ qlora_status linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
   const int64_t ldb2 = b_direct ? r : kRankPad;
   if (!dense) {
     Timed tm(kFamGemm, s);
-    return gemm_status(launch_linear_gemm_nf4(w, X, M, at<uint16_t>(ws, lay.us), B2, r, ldb2, Y, 0, status, false, s,
-                                              diag.wait_limit_ns, diag.debug_stall));
+    return gemm_status(launch_linear_gemm_nf4(w, at<float>(ws, lay.scales), X, M, at<uint16_t>(ws, lay.us), B2, r,
+                                              ldb2, Y, 0, status, false, s, diag.wait_limit_ns, diag.debug_stall));
   }
   GemmArgs g{};
   g.A = X;
@@ -890,7 +898,8 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
   }
   if (dX != nullptr && !dense) {  // dX = dY W_hat + s V A, W_hat decoded in the GEMM, A [r, K] MN-major
     Timed tm(kFamGemm, s);
-    e = launch_linear_gemm_nf4(w, dY, M, at<uint16_t>(ws, lay.vs), A, r, 0, dX, accumulate, status, true, s);
+    e = launch_linear_gemm_nf4(w, at<float>(ws, lay.scales), dY, M, at<uint16_t>(ws, lay.vs), A, r, 0, dX, accumulate,
+                               status, true, s);
     if (e != cudaSuccess) return gemm_status(e);
   }
   if (dX != nullptr && dense) {  // dense-weight path: W_hat [N, K] and A [r, K] read as MN-major operands

@@ -74,9 +74,16 @@ constexpr int B_TILE = BNH * BK * 2;   // 16 KB
 constexpr int TMEM_COLS = 512;         // two 128 x 256 fp32 accumulators per CTA
 constexpr int kDecodeGroups = 2;
 constexpr int kFirstDecodeWarp = 6;
-constexpr int kThreads = 32 * (kFirstDecodeWarp + 4 * kDecodeGroups);
+constexpr int kCodeWarp = kFirstDecodeWarp + 4 * kDecodeGroups;  // producer of the code ring
+constexpr int kThreads = 32 * (kCodeWarp + 1);
 constexpr int kDecodedArrivals = 2 * 4;    // the four decode warps of each CTA that handle a stage
-constexpr int SMEM_BYTES = 1024 + STAGES * (A_TILE + B_TILE) + 512;
+// Code ring (per CTA): a stage's packed codes (4 KB) and decoded block scales
+// (fp32 boxes of 4 blocks per weight row: 2 KB forward, 1 KB backward).
+constexpr int kCodeStages = 4;             // a multiple of kDecodeGroups: a slot always serves one group
+constexpr int CODE_SLOT = 6144;
+constexpr int kCodeBytes = 4096;
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_TILE + B_TILE) + kCodeStages * CODE_SLOT + 512;
+static_assert(kCodeStages % kDecodeGroups == 0, "a code slot must always serve the same decode group");
 constexpr size_t kL2PanelBudget = size_t(48) << 20;
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -129,26 +136,34 @@ __device__ __forceinline__ void decode_block_to_smem(uint32_t row, uint32_t sw, 
   }
 }
 
-// The packed codes, scale code and second-level scale of one block, in flight.
-struct BlockLoad {
-  uint32_t w[8];
-  float x;   // c2 of the block's chunk, or the fp32 absmax
-  int q;     // int8 / E4M3 scale code (bit pattern)
-};
 
-__device__ __forceinline__ void load_block(BlockLoad& b, const Nf4GemmParams& p, int64_t blk) {
-  if (blk < 0) return;
-  const uint4* src = reinterpret_cast<const uint4*>(p.packed + blk * 32);
-  const uint4 u0 = ld_stream_u4(src), u1 = ld_stream_u4(src + 1);
-  b.w[0] = u0.x; b.w[1] = u0.y; b.w[2] = u0.z; b.w[3] = u0.w;
-  b.w[4] = u1.x; b.w[5] = u1.y; b.w[6] = u1.z; b.w[7] = u1.w;
-  if (p.scale_format == kScalesFp32) {
-    b.x = __ldg(p.absmax + blk);
-    b.q = 0;
-  } else {
-    b.q = __ldg(p.qscale + blk);
-    b.x = __ldg(p.c2 + (blk >> 8));
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr) : "memory");
+}
+
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// Warp-wide bounded wait: lane 0 polls (the other lanes idle at the shuffle,
+// so a waiting warp takes few issue slots), then every lane acquires the
+// completed phase itself.  Returns false (warp-uniformly) on abort / timeout.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          uint64_t lim, bool cluster) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0)
+    ok = cluster ? mbar_wait_cluster(bar, parity, abort_flag, status, lim)
+                 : mbar_wait(bar, parity, abort_flag, status, lim);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok) {
+    if (cluster)
+      (void)mbar_try_wait_cluster(bar, parity);
+    else
+      (void)mbar_try_wait(bar, parity);
   }
+  return ok;
 }
 
 }  // namespace
@@ -156,12 +171,14 @@ __device__ __forceinline__ void load_block(BlockLoad& b, const Nf4GemmParams& p,
 template <bool kBwd>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
-                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ Nf4GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmP,
+                    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ Nf4GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_TILE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_TILE);  // fullA: TMA bytes (even CTA)
+  uint8_t* sC = sB + STAGES * B_TILE;    // code ring
+  uint64_t* full = reinterpret_cast<uint64_t*>(sC + kCodeStages * CODE_SLOT);  // fullA: TMA bytes (even CTA)
   uint64_t* decoded = full + STAGES;      // fullB: decode warps of both CTAs (even CTA)
   uint64_t* empty = decoded + STAGES;
   uint64_t* acc_full = empty + STAGES;    // [2]
@@ -169,7 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint64_t* drained = drain + 1;          // odd CTA: every copy of the pair has landed
   uint64_t* never = drained + 1;          // diagnostic: a barrier nothing arrives at
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
+  uint64_t* cfull = never + 1;            // [kCodeStages] code ring: TMA bytes landed
+  uint64_t* cempty = cfull + kCodeStages; // [kCodeStages] code ring: the group's four warps read the slot
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cempty + kCodeStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_ctarank();
@@ -195,6 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain, 1);
     mbar_init(drained, 1);
     mbar_init(never, 1);
+    for (int c = 0; c < kCodeStages; ++c) {
+      mbar_init(&cfull[c], 1);
+      mbar_init(&cempty[c], 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -307,8 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tl = 0;
     for (int t = pair; t < total_tiles; t += npairs, ++tl) {
       const int buf = tl & 1, use = tl >> 1;
-      const bool ok =
-          __all_sync(0xffffffffu, mbar_wait_cluster(&acc_full[buf], use & 1, abort_flag, status, lim) ? 1 : 0) != 0;
+      const bool ok = warp_wait(&acc_full[buf], use & 1, abort_flag, status, lim, true);
       if (!ok) break;
       tc_fence_after();
       int mb, nb;
@@ -326,138 +348,133 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * static_cast<uint32_t>(buf));
     }
-  } else {
-    // Weight decoders.  Group g takes the pipeline iterations it with
+  } else if (warp < kCodeWarp) {
+    // Weight decoders.  Group g takes the pipeline steps it with
     // it % kDecodeGroups == g; thread `tid` writes one 128-byte row of the
-    // stage's B tile.
+    // stage's B tile from its block's codes and scale in the code ring.  No
+    // decoder thread loads from global memory, so its release-arrives never
+    // wait on loads in flight.
     const int dw = warp - kFirstDecodeWarp;
     const int grp = dw >> 2;
     const int tid = ((dw & 3) << 5) | lane;
     const uint32_t row_off = kBwd ? static_cast<uint32_t>((tid >> 6) * 8192 + (tid & 63) * 128)
                                   : static_cast<uint32_t>(tid * 128);
     const uint32_t sw = static_cast<uint32_t>(tid & 7);
+    // this thread's codes (32 bytes) and scale in a code slot
+    const uint32_t code_off = kBwd ? static_cast<uint32_t>((tid >> 6) * 2048 + (tid & 63) * 32)
+                                   : static_cast<uint32_t>(tid * 32);
+    const uint32_t scale_row = kBwd ? static_cast<uint32_t>(kCodeBytes + (tid & 63) * 16)
+                                    : static_cast<uint32_t>(kCodeBytes + tid * 16);
     float L[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) L[j] = codebook_level(p.codebook, j);
-    const bool fp32_scales = p.scale_format == kScalesFp32;
-    const float mu = fp32_scales ? 0.0f : __ldg(p.mu);
     const int64_t kblocks = p.Kw / kBlock;
     const uint32_t decoded0 = map_to_cta(&decoded[0], 0);
-    const uint32_t sB0 = smem_u32(sB);
-    const int my_tiles = pair < total_tiles ? (total_tiles - 1 - pair) / npairs + 1 : 0;
-    const int total_it = my_tiles * k_iters;
-
-    // The iterations of this group, in order: it = grp, grp + G, ...  Cursor
-    // (tl, i): tile tl of this pair, pipeline step i of that tile; the block
-    // index is recomputed from the tile's coordinates only when tl changes.
-    constexpr int G = kDecodeGroups;
-    struct Cursor {
-      int it, tl, i;
-      int64_t row_base;  // forward: first weight row of this CTA's half; backward: first output block
-    };
-    auto tile_base = [&](int tl) -> int64_t {
-      int mb, nb;
-      pair_tile_coords(pair + tl * npairs, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
-      return kBwd ? (static_cast<int64_t>(nb) * BN + static_cast<int64_t>(rank) * BNH) / kBlock
-                  : static_cast<int64_t>(nb) * BN + static_cast<int64_t>(rank) * BNH;
-    };
-    auto advance = [&](Cursor& c) {
-      c.it += G;
-      c.i += G;
-      if (c.i >= k_iters) {
-        while (c.i >= k_iters) {
-          c.i -= k_iters;
-          ++c.tl;
-        }
-        if (c.it < total_it) c.row_base = tile_base(c.tl);
-      }
-    };
-    // Block index this thread decodes at cursor c: >= 0 a block, -1 a row
-    // past the weight (written as zeros), -2 the rank step (nothing).
-    auto block_of = [&](const Cursor& c) -> int64_t {
-      if (c.i >= num_k) return -2;
-      if constexpr (!kBwd) {
-        const int64_t n = c.row_base + tid;
-        return n < p.Nw ? n * kblocks + c.i : -1;
-      } else {
-        const int64_t n = static_cast<int64_t>(c.i) * BK + (tid & 63);
-        const int64_t kb = c.row_base + (tid >> 6);
-        return (n < p.Nw && kb < kblocks) ? n * kblocks + kb : -1;
-      }
-    };
-
-    // One pipeline step of this group: prefetch the block of `ahead` (two
-    // steps later) into `nxt`, wait for the stage slot, decode `cur` into it,
-    // fence and signal.  The three register sets rotate by unrolling (no
-    // copies), so a load in flight is never waited on before its use.
+    const uint32_t sB0 = smem_u32(sB), sC0 = smem_u32(sC);
+    int it = 0;
     bool ok = true;
-    auto step = [&](const Cursor& c, BlockLoad& cur, int64_t bc, const Cursor& ahead, BlockLoad& nxt,
-                    int64_t& bn) {
-      if (ahead.it < total_it) {
-        bn = block_of(ahead);
-        load_block(nxt, p, bn);
-      }
-      const int s = c.it % STAGES, u = c.it / STAGES;
-      if (c.it >= STAGES &&
-          __all_sync(0xffffffffu, mbar_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim) ? 1 : 0) == 0) {
-        ok = false;
-        return;
-      }
-      // Every stage gets this warp's arrival, the rank step too (its
-      // operands come by TMA), so the barrier's phases follow the slot's uses.
-      if (bc != -2) {
-        const uint32_t row = sB0 + static_cast<uint32_t>(s * B_TILE) + row_off;
-        if (bc >= 0) {
-          const float a = fp32_scales ? cur.x
-                                      : decode_scale_value(scale_code_value(p.scale_format, static_cast<int8_t>(cur.q)),
-                                                           cur.x, mu);
-          decode_block_to_smem(row, sw, cur.w, a, L);
-        } else {
+    for (int t = pair; t < total_tiles && ok; t += npairs) {
+      int mb, nb;
+      pair_tile_coords(t, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
+      const int64_t base = kBwd ? (static_cast<int64_t>(nb) * BN + static_cast<int64_t>(rank) * BNH) / kBlock
+                                : static_cast<int64_t>(nb) * BN + static_cast<int64_t>(rank) * BNH;
+      for (int i = 0; i < k_iters; ++i, ++it) {
+        if (it % kDecodeGroups != grp) continue;
+        const int c = it % kCodeStages, cu = it / kCodeStages;
+        const int s = it % STAGES, u = it / STAGES;
+        if (i < num_k) {
+          // this thread's block: valid row and column, else a zero row
+          bool valid;
+          uint32_t kq;  // the block's column within its 4-block scale box
+          if constexpr (!kBwd) {
+            valid = base + tid < p.Nw;
+            kq = static_cast<uint32_t>(i & 3);
+          } else {
+            const int64_t kb = base + (tid >> 6);
+            valid = static_cast<int64_t>(i) * BK + (tid & 63) < p.Nw && kb < kblocks;
+            kq = static_cast<uint32_t>(kb & 3);
+          }
+          if (!warp_wait(&cfull[c], cu & 1, abort_flag, status, lim, false)) {
+            ok = false;
+            break;
+          }
+          const uint32_t slot = sC0 + static_cast<uint32_t>(c * CODE_SLOT);
+          uint32_t w[8];
+          ld_shared_v4(slot + code_off, w[0], w[1], w[2], w[3]);
+          ld_shared_v4(slot + code_off + 16, w[4], w[5], w[6], w[7]);
+          const float a = ld_shared_f32(slot + scale_row + 4 * kq);
+          if (it >= STAGES && !warp_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim, false)) {
+            ok = false;
+            break;
+          }
+          const uint32_t row = sB0 + static_cast<uint32_t>(s * B_TILE) + row_off;
+          if (valid) {
+            decode_block_to_smem(row, sw, w, a, L);
+          } else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) st_shared_v4(row + (static_cast<uint32_t>(j) << 4), 0u, 0u, 0u, 0u);
+            for (int j = 0; j < 8; ++j) st_shared_v4(row + (static_cast<uint32_t>(j) << 4), 0u, 0u, 0u, 0u);
+          }
+          // One proxy fence orders this thread's code-slot reads before the
+          // slot's next TMA refill and its tile writes before the MMA's reads.
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_cluster(decoded0 + 8u * static_cast<uint32_t>(s));
+            mbar_arrive(&cempty[c]);
+          }
+        } else {
+          // The rank step: its operands come by TMA.  Every stage still gets
+          // this warp's arrivals, so the barriers' phases follow the slots' uses.
+          if (!warp_wait(&cfull[c], cu & 1, abort_flag, status, lim, false) ||
+              (it >= STAGES && !warp_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim, false))) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_cluster(decoded0 + 8u * static_cast<uint32_t>(s));
+            mbar_arrive(&cempty[c]);
+          }
         }
-        fence_async_smem();  // these generic-proxy writes before the tensor core's reads
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(decoded0 + 8u * static_cast<uint32_t>(s));
-    };
-
-    if (grp < total_it) {
-      Cursor c0{grp, 0, grp, 0};
-      while (c0.i >= k_iters) {
-        c0.i -= k_iters;
-        ++c0.tl;
+    }
+  } else {
+    // Code ring producer (lane 0): per pipeline step, this CTA's packed codes
+    // and decoded block scales by TMA into slot it % kCodeStages, as soon as
+    // the decode group that read the slot's previous contents released it.
+    if (lane == 0) {
+      tma_prefetch_desc(&tmP);
+      tma_prefetch_desc(&tmS);
+      int it = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += npairs) {
+        int mb, nb;
+        pair_tile_coords(t, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
+        const int n_half = nb * BN + static_cast<int>(rank) * BNH;  // forward: first weight row; backward: first column
+        for (int i = 0; i < k_iters; ++i, ++it) {
+          const int c = it % kCodeStages, cu = it / kCodeStages;
+          if (it >= kCodeStages && !mbar_wait(&cempty[c], (cu - 1) & 1, abort_flag, status, lim)) {
+            ok = false;
+            break;
+          }
+          uint8_t* slot = sC + c * CODE_SLOT;
+          if (i >= num_k) {
+            mbar_arrive(&cfull[c]);  // the rank step carries no codes
+          } else if constexpr (!kBwd) {
+            mbar_arrive_expect_tx(&cfull[c], kCodeBytes + BNH * 16);
+            tma_load_2d(slot, &tmP, &cfull[c], i * 32, n_half);                          // [128 rows][32 B]
+            tma_load_2d(slot + kCodeBytes, &tmS, &cfull[c], i & ~3, n_half);             // [128 rows][4 scales]
+          } else {
+            const int n0 = i * BK, kb0 = n_half / kBlock;
+            mbar_arrive_expect_tx(&cfull[c], kCodeBytes + BK * 16);
+            tma_load_2d(slot, &tmP, &cfull[c], n_half / 2, n0);                          // [64 rows][32 B]
+            tma_load_2d(slot + 2048, &tmP, &cfull[c], n_half / 2 + 32, n0);              // the next block
+            tma_load_2d(slot + kCodeBytes, &tmS, &cfull[c], kb0 & ~3, n0);               // [64 rows][4 scales]
+          }
+        }
       }
-      c0.row_base = tile_base(c0.tl);
-      Cursor c1 = c0;
-      advance(c1);
-      Cursor c2 = c1;
-      advance(c2);
-      BlockLoad b0, b1, b2;
-      int64_t k0 = block_of(c0), k1 = -2, k2 = -2;
-      load_block(b0, p, k0);
-      if (c1.it < total_it) {
-        k1 = block_of(c1);
-        load_block(b1, p, k1);
-      }
-      // c0 -> b0, c1 -> b1, c2 -> b2 (loaded by the first step)
-      while (true) {
-        step(c0, b0, k0, c2, b2, k2);
-        if (!ok || c1.it >= total_it) break;
-        advance(c0);
-        advance(c0);
-        advance(c0);  // c0 is now three steps ahead: the block after c2
-        step(c1, b1, k1, c0, b0, k0);
-        if (!ok || c2.it >= total_it) break;
-        advance(c1);
-        advance(c1);
-        advance(c1);
-        step(c2, b2, k2, c1, b1, k1);
-        if (!ok || c0.it >= total_it) break;
-        advance(c2);
-        advance(c2);
-        advance(c2);
-      }
+      // Teardown: every copy into the code ring has landed.
+      for (int i = (it > kCodeStages ? it - kCodeStages : 0); i < it; ++i)
+        mbar_wait_teardown(&cfull[i % kCodeStages], (i / kCodeStages) & 1, status);
     }
   }
   tc_fence_before();
@@ -519,8 +536,16 @@ cudaError_t launch_gemm_nf4(const Nf4GemmArgs& a, cudaStream_t stream) {
   // GEMM view: D [M][N] = A [M][K] op(W_hat) + A2 B2
   const int64_t N = bwd ? w.cols : w.rows;
   const int64_t K = bwd ? w.rows : w.cols;
-  CUtensorMap tA, tA2, tB2;
+  CUtensorMap tA, tA2, tB2, tP, tS;
   if (!encode_tensor_map_2d(&tA, a.A, a.M, K, BM, BK)) return cudaErrorInvalidValue;
+  // Code ring sources: the packed codes [N_w][K_w / 2] bytes and the decoded
+  // block scales [N_w][ld] fp32 (a.scales, written by launch_block_scales).
+  const uint32_t code_rows = bwd ? BK : BNH;
+  const int64_t sld = block_scales_ld(w.cols);
+  if (a.scales == nullptr) return cudaErrorInvalidValue;
+  if (!encode_tensor_map_2d_plain(&tP, w.packed, 1, w.rows, w.cols / 2, w.cols / 2, code_rows, 32))
+    return cudaErrorInvalidValue;
+  if (!encode_tensor_map_2d_plain(&tS, a.scales, 4, w.rows, sld, sld, code_rows, 4)) return cudaErrorInvalidValue;
   int r_steps = 0;
   if (a.A2 != nullptr && a.r > 0) {
     r_steps = (a.r + 15) / 16;
@@ -578,8 +603,8 @@ cudaError_t launch_gemm_nf4(const Nf4GemmArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (bwd) return cudaLaunchKernelEx(&cfg, gemm_nf4_kernel<true>, tA, tA2, tB2, p);
-  return cudaLaunchKernelEx(&cfg, gemm_nf4_kernel<false>, tA, tA2, tB2, p);
+  if (bwd) return cudaLaunchKernelEx(&cfg, gemm_nf4_kernel<true>, tA, tA2, tB2, tP, tS, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nf4_kernel<false>, tA, tA2, tB2, tP, tS, p);
 }
 
 }  // namespace qnf4

@@ -78,6 +78,23 @@ bool encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major [rows][cols] tensor of 1-byte (uint8) or 4-byte (fp32) elements,
+// row pitch `ld` elements, box box_rows x box_cols, no swizzle, zero fill
+// outside the tensor.
+bool encode_tensor_map_2d_plain(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
+                                uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr || (elem_bytes != 1 && elem_bytes != 4)) return false;
+  const cuuint64_t gdim[2] = {cols, rows};
+  const cuuint64_t gstride[1] = {ld * static_cast<uint64_t>(elem_bytes)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+            const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tile order: groups of kGroupM consecutive M tiles sweep the N tiles, so the
 // CTAs resident at one time share a few A row panels and a few B row panels
 // (both stay in L2 instead of being re-read from HBM every wave).

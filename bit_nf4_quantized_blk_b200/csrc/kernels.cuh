@@ -93,6 +93,9 @@ struct DequantBatchParams {
 };
 
 cudaError_t launch_dequant_batch(const DequantBatchParams& p, int out_fp32, cudaStream_t stream);
+// Decoded fp32 block scales [rows][block_scales_ld(cols)] (16-byte aligned output).
+int64_t block_scales_ld(int64_t cols);
+cudaError_t launch_block_scales(const WeightView& w, float* out, cudaStream_t stream);
 cudaError_t launch_dequant_transposed(const WeightView& w, uint16_t* out, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
@@ -212,6 +215,7 @@ cudaError_t launch_gemm_tn(const GemmArgs& a, cudaStream_t stream);
 // ---------------------------------------------------------------------------
 struct Nf4GemmArgs {
   WeightView w;
+  const float* scales; // decoded block scales [N_w][block_scales_ld(K_w)] (launch_block_scales)
   const uint16_t* A;   // X (forward) or dY (backward), bf16 row-major
   const uint16_t* A2;  // [M][64] bf16 s*U or s*V, zero padded beyond r; null: no rank step
   const uint16_t* B2;  // see above
@@ -254,5 +258,8 @@ cudaError_t launch_gemm_nf4(const Nf4GemmArgs& a, cudaStream_t stream);
 // Driver entry point used to encode TMA descriptors (resolved once).
 bool encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
                           uint32_t box_cols, bool swizzle128 = true, uint64_t ld = 0);
+// uint8 (elem_bytes 1) or fp32 (4) row-major tensor, pitch ld elements, no swizzle.
+bool encode_tensor_map_2d_plain(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
+                                uint64_t ld, uint32_t box_rows, uint32_t box_cols);
 
 }  // namespace qnf4

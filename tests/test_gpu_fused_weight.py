@@ -111,7 +111,9 @@ def test_fused_path_needs_no_dense_weight_workspace():
         fused = binding.qlora_linear_ws_bytes(M, N, K, r)
     with binding.weight_path(binding.WEIGHT_PATH_DENSE):
         dense = binding.qlora_linear_ws_bytes(M, N, K, r)
-    assert dense - fused >= N * K * 2
+    # the dense arm adds the N x K bf16 copy and drops the fused path's
+    # decoded block scales (N x K / 64 fp32)
+    assert dense - fused >= N * K * 2 - N * (K // 64) * 4
     assert fused < N * K * 2 // 2
     W = workloads.normal_f32((64, 128), 0.02, 5)
     out = gpu_quantize(W)
