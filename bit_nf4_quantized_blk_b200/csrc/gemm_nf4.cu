@@ -41,11 +41,13 @@
 //               tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16
 //   warps 2-5   epilogue of this CTA's 128 accumulator rows
 //   warps 6-13  weight decoders: two groups of four warps take alternate
-//               stages; each thread decodes one block per stage of its group,
-//               keeps the codes of its next two stages in flight in
-//               registers, fences its shared-memory writes for the async
-//               proxy and its warp arrives on the even CTA's decoded-stage
-//               barrier (fullB).
+//               stages; each thread reads its block's codes and scale from
+//               the code ring, decodes the block into the stage's tile,
+//               fences its shared-memory writes for the async proxy, and its
+//               warp arrives on the even CTA's decoded-stage barrier (fullB)
+//               with a CTA-scope arrive (mbar_arrive_remote)
+//   warp 14     code ring producer: per stage, this CTA's packed codes and
+//               decoded block scales by TMA into a 4-slot ring
 // The MMA issuer waits on both barriers of a stage.  Keeping the copies on a
 // barrier of their own lets a teardown wait for exactly the copies in
 // flight: the even producer waits for the last stages' copies of both CTAs
@@ -419,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            mbar_arrive_cluster(decoded0 + 8u * static_cast<uint32_t>(s));
+            mbar_arrive_remote(decoded0 + 8u * static_cast<uint32_t>(s));
             mbar_arrive(&cempty[c]);
           }
         } else {
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           if (lane == 0) {
-            mbar_arrive_cluster(decoded0 + 8u * static_cast<uint32_t>(s));
+            mbar_arrive_remote(decoded0 + 8u * static_cast<uint32_t>(s));
             mbar_arrive(&cempty[c]);
           }
         }
