@@ -33,13 +33,20 @@
 // four codes at a time with byte permutes whose selectors are the packed
 // nibbles themselves (bit 3 of a code picks the upper half of the table).
 //
-// Pair-CTA layout (cluster of 2, 256 x 256 output tile per pair):
-//   warp 0      TMA producer of this CTA's 128 rows of A (X or dY) per stage,
-//               and of the rank step's tiles; the even CTA arms the stage's
-//               copy barrier (fullA) with both CTAs' bytes
+// Pair-CTA layout (cluster of 2, 512 x 256 output tile per pair):
+//   Each decoded weight stage feeds the MMAs of two 256-row halves of A, so
+//   every decoded value serves 512 rows of the activations; decoding then
+//   takes half the share of the SM's issue slots and shared-memory port that
+//   a 256-row tile would.  The two halves' accumulators fill tensor memory
+//   (2 x 256 columns), so the accumulator is single-buffered: the epilogue
+//   drains it while the producers already fill the next tile's stages.
+//   warp 0      TMA producer of this CTA's 2 x 128 rows of A (X or dY) per
+//               stage, and of the rank step's tiles; the even CTA arms the
+//               stage's copy barrier (fullA) with both CTAs' bytes
 //   warp 1      TMEM allocation (both CTAs); in the even CTA, MMA issue:
-//               tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16
-//   warps 2-5   epilogue of this CTA's 128 accumulator rows
+//               tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16,
+//               one accumulator per half
+//   warps 2-5   epilogue of this CTA's 2 x 128 accumulator rows
 //   warps 6-13  weight decoders: two groups of four warps take alternate
 //               stages; each thread reads its block's codes and scale from
 //               the code ring, decodes the block into the stage's tile,
@@ -48,6 +55,9 @@
 //               with a CTA-scope arrive (mbar_arrive_remote)
 //   warp 14     code ring producer: per stage, this CTA's packed codes and
 //               decoded block scales by TMA into a 4-slot ring
+// Tiles are whole (512 rows) except in a last partial wave that would use at
+// most half of the pairs: those tiles are split into their two 256-row
+// halves, which run on twice as many pairs in half the time.
 // The MMA issuer waits on both barriers of a stage.  Keeping the copies on a
 // barrier of their own lets a teardown wait for exactly the copies in
 // flight: the even producer waits for the last stages' copies of both CTAs
@@ -66,14 +76,16 @@ namespace qnf4 {
 
 namespace {
 
-constexpr int BM = 128;          // rows of A per CTA (256 per pair)
+constexpr int BM = 128;          // rows of A per CTA and half (256 per pair and half)
+constexpr int kHalves = 2;       // 256-row halves of A per pair tile
 constexpr int BN = 256;          // output columns per pair tile
 constexpr int BNH = BN / 2;      // B rows (forward) / output columns (backward) per CTA
 constexpr int BK = 64;           // reduction values per stage (one quantization block)
-constexpr int STAGES = 6;
-constexpr int A_TILE = BM * BK * 2;    // 16 KB
-constexpr int B_TILE = BNH * BK * 2;   // 16 KB
-constexpr int TMEM_COLS = 512;         // two 128 x 256 fp32 accumulators per CTA
+constexpr int STAGES = 4;
+constexpr int A_TILE = BM * BK * 2;          // 16 KB per half
+constexpr int A_STAGE = kHalves * A_TILE;    // 32 KB
+constexpr int B_TILE = BNH * BK * 2;         // 16 KB
+constexpr int TMEM_COLS = 512;               // one 128 x 256 fp32 accumulator per half, per CTA
 constexpr int kDecodeGroups = 2;
 constexpr int kFirstDecodeWarp = 6;
 constexpr int kCodeWarp = kFirstDecodeWarp + 4 * kDecodeGroups;  // producer of the code ring
@@ -84,9 +96,49 @@ constexpr int kDecodedArrivals = 2 * 4;    // the four decode warps of each CTA 
 constexpr int kCodeStages = 4;             // a multiple of kDecodeGroups: a slot always serves one group
 constexpr int CODE_SLOT = 6144;
 constexpr int kCodeBytes = 4096;
-constexpr int SMEM_BYTES = 1024 + STAGES * (A_TILE + B_TILE) + kCodeStages * CODE_SLOT + 512;
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_TILE) + kCodeStages * CODE_SLOT + 512;
 static_assert(kCodeStages % kDecodeGroups == 0, "a code slot must always serve the same decode group");
 constexpr size_t kL2PanelBudget = size_t(48) << 20;
+
+// A pair's work item t: pair tile t of the raster whole, or (from full_tiles
+// on) one 256-row half of a tile of the last wave.  mh0 is its first 256-row
+// block of A, nh the number of 256-row blocks (0: past the end of A).
+struct WorkItem {
+  int mh0, nb, nh;
+};
+
+__device__ __forceinline__ WorkItem work_item(int t, const Nf4GemmParams& p, int m_tiles, int n_tiles, int m256) {
+  int tile = t, half = -1;
+  if (t >= p.full_tiles) {
+    tile = p.full_tiles + ((t - p.full_tiles) >> 1);
+    half = (t - p.full_tiles) & 1;
+  }
+  int mb, nb;
+  pair_tile_coords(tile, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
+  WorkItem w;
+  w.nb = nb;
+  if (half < 0) {
+    w.mh0 = kHalves * mb;
+    w.nh = min(kHalves, m256 - w.mh0);
+  } else {
+    w.mh0 = kHalves * mb + half;
+    w.nh = w.mh0 < m256 ? 1 : 0;
+  }
+  return w;
+}
+
+// tcgen05.wait::ld that also hands the loaded registers on, so no use of
+// them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
@@ -178,14 +230,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_TILE;
+  uint8_t* sB = smem + STAGES * A_STAGE;
   uint8_t* sC = sB + STAGES * B_TILE;    // code ring
   uint64_t* full = reinterpret_cast<uint64_t*>(sC + kCodeStages * CODE_SLOT);  // fullA: TMA bytes (even CTA)
   uint64_t* decoded = full + STAGES;      // fullB: decode warps of both CTAs (even CTA)
   uint64_t* empty = decoded + STAGES;
-  uint64_t* acc_full = empty + STAGES;    // [2]
-  uint64_t* acc_empty = acc_full + 2;     // [2], even CTA
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* acc_full = empty + STAGES;    // the accumulators hold a finished tile
+  uint64_t* acc_empty = acc_full + 1;     // even CTA: both CTAs' epilogues drained them
+  uint64_t* drain = acc_empty + 1;
   uint64_t* drained = drain + 1;          // odd CTA: every copy of the pair has landed
   uint64_t* never = drained + 1;          // diagnostic: a barrier nothing arrives at
   uint64_t* cfull = never + 1;            // [kCodeStages] code ring: TMA bytes landed
@@ -196,8 +248,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = p.M, N = p.N, num_k = p.num_k, r_steps = p.r_steps;
-  const int m_tiles = (M + 2 * BM - 1) / (2 * BM), n_tiles = (N + BN - 1) / BN;
-  const int total_tiles = m_tiles * n_tiles;
+  const int m256 = (M + 2 * BM - 1) / (2 * BM);
+  const int m_tiles = (m256 + kHalves - 1) / kHalves, n_tiles = (N + BN - 1) / BN;
+  const int items = p.items;
   const int pair = static_cast<int>(cluster_id_x()), npairs = static_cast<int>(num_clusters_x());
   const int k_iters = num_k + (r_steps > 0 ? 1 : 0);
   int* status = p.status;
@@ -209,10 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&decoded[s], kDecodedArrivals);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 8);  // 4 epilogue warps x 2 CTAs
-    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);  // 4 epilogue warps x 2 CTAs
     mbar_init(drain, 1);
     mbar_init(drained, 1);
     mbar_init(never, 1);
@@ -243,11 +294,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t full0 = map_to_cta(&full[0], 0);
       int it = 0;
       bool ok = true;
-      for (int t = pair; t < total_tiles && ok; t += npairs) {
-        int mb, nb;
-        pair_tile_coords(t, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
-        const int m0 = mb * 2 * BM + static_cast<int>(rank) * BM;
-        const int n0 = nb * BN + static_cast<int>(rank) * BNH;
+      for (int t = pair; t < items && ok; t += npairs) {
+        const WorkItem wi = work_item(t, p, m_tiles, n_tiles, m256);
+        if (wi.nh == 0) continue;
+        const int m0 = wi.mh0 * 2 * BM + static_cast<int>(rank) * BM;  // this CTA's rows of the first half
+        const int n0 = wi.nb * BN + static_cast<int>(rank) * BNH;
         for (int i = 0; i < k_iters; ++i, ++it) {
           const int s = it % STAGES, u = it / STAGES;
           if (it >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim)) {
@@ -255,18 +306,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
+          uint8_t* const a_st = sA + s * A_STAGE;
           if (i < num_k) {
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * A_TILE);
-            tma_load_2d_pair(sA + s * A_TILE, &tmA, fb, i * BK, m0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * wi.nh * A_TILE);
+            for (int h = 0; h < wi.nh; ++h) tma_load_2d_pair(a_st + h * A_TILE, &tmA, fb, i * BK, m0 + h * 2 * BM);
           } else if constexpr (!kBwd) {
             // rank step: A2 = s U [M][64], B2 = LoRA B [N_w][r] (zero filled to 64)
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (A_TILE + B_TILE));
-            tma_load_2d_pair(sA + s * A_TILE, &tmA2, fb, 0, m0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (wi.nh * A_TILE + B_TILE));
+            for (int h = 0; h < wi.nh; ++h) tma_load_2d_pair(a_st + h * A_TILE, &tmA2, fb, 0, m0 + h * 2 * BM);
             tma_load_2d_pair(sB + s * B_TILE, &tmB2, fb, 0, n0);
           } else {
             // rank step: A2 = s V [M][64], B2 = LoRA A [r][K_w] as MN-major boxes
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (A_TILE + (BNH / 64) * r_steps * 16 * 128));
-            tma_load_2d_pair(sA + s * A_TILE, &tmA2, fb, 0, m0);
+            if (rank == 0)
+              mbar_arrive_expect_tx(&full[s], 2 * (wi.nh * A_TILE + (BNH / 64) * r_steps * 16 * 128));
+            for (int h = 0; h < wi.nh; ++h) tma_load_2d_pair(a_st + h * A_TILE, &tmA2, fb, 0, m0 + h * 2 * BM);
             for (int j = 0; j < BNH / 64; ++j)
               tma_load_2d_pair(sB + s * B_TILE + j * 8192, &tmB2, fb, n0 + 64 * j, 0);
           }
@@ -294,11 +347,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // arrives at, so its wait runs out and the whole pair takes the abort
       // path (every other wait then ends on the abort flag or its own limit).
       bool ok = !p.debug_stall || mbar_wait(never, 0, abort_flag, status, lim);
-      for (int t = pair; t < total_tiles && ok; t += npairs, ++tl) {
-        const int buf = tl & 1, use = tl >> 1;
-        if (use > 0 && !mbar_wait_cluster(&acc_empty[buf], (use - 1) & 1, abort_flag, status, lim)) break;
+      for (int t = pair; t < items && ok; t += npairs) {
+        const WorkItem wi = work_item(t, p, m_tiles, n_tiles, m256);
+        if (wi.nh == 0) continue;
+        if (tl > 0 && !mbar_wait_cluster(acc_empty, (tl - 1) & 1, abort_flag, status, lim)) break;
+        ++tl;
         tc_fence_after();
-        const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN);
         for (int i = 0; i < k_iters; ++i, ++it) {
           const int s = it % STAGES, u = it / STAGES;
           if (!mbar_wait_cluster(&full[s], u & 1, abort_flag, status, lim) ||
@@ -308,17 +362,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const int nsteps = i < num_k ? BK / 16 : r_steps;
-          const uint64_t adesc = smem_desc_k128(smem_u32(sA + s * A_TILE));
           const uint64_t bdesc = kBwd ? smem_desc_mn128(smem_u32(sB + s * B_TILE), 8192, 1024)
                                       : smem_desc_k128(smem_u32(sB + s * B_TILE));
           // One K = 16 step: A (K-major) +32 bytes inside the swizzle atom;
           // B +32 bytes (K-major) or +2 atoms of 8 rows = 2048 bytes (MN-major).
           const uint32_t bstep = kBwd ? (2048 >> 4) : 2;
-          for (int kk = 0; kk < nsteps; ++kk)
-            tc_mma_bf16_ss_pair(acc, adesc + 2 * kk, bdesc + bstep * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int h = 0; h < wi.nh; ++h) {
+            const uint32_t acc = tmem + static_cast<uint32_t>(h * BN);
+            const uint64_t adesc = smem_desc_k128(smem_u32(sA + s * A_STAGE + h * A_TILE));
+            for (int kk = 0; kk < nsteps; ++kk)
+              tc_mma_bf16_ss_pair(acc, adesc + 2 * kk, bdesc + bstep * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          }
           tc_commit_pair(&empty[s], 0x3);
         }
-        if (ok) tc_commit_pair(&acc_full[buf], 0x3);
+        if (ok) tc_commit_pair(acc_full, 0x3);
       }
       // Every MMA (which also reads the odd CTA's shared memory) must be
       // complete before the pair's tensor memory and shared memory go.
@@ -328,27 +385,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < kFirstDecodeWarp) {
     // Epilogue warps 2..5 own TMEM lane quadrants (warp % 4).
     const int q = warp & 3;
-    const uint32_t acc_empty0 = map_to_cta(&acc_empty[0], 0);
+    const uint32_t acc_empty0 = map_to_cta(acc_empty, 0);
     int tl = 0;
-    for (int t = pair; t < total_tiles; t += npairs, ++tl) {
-      const int buf = tl & 1, use = tl >> 1;
-      const bool ok = warp_wait(&acc_full[buf], use & 1, abort_flag, status, lim, true);
+    for (int t = pair; t < items; t += npairs) {
+      const WorkItem wi = work_item(t, p, m_tiles, n_tiles, m256);
+      if (wi.nh == 0) continue;
+      const bool ok = warp_wait(acc_full, tl & 1, abort_flag, status, lim, true);
+      ++tl;
       if (!ok) break;
       tc_fence_after();
-      int mb, nb;
-      pair_tile_coords(t, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
-      const int row = mb * 2 * BM + static_cast<int>(rank) * BM + q * 32 + lane;
-      const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(acc + c * 32, v);
-        tmem_wait_ld();
-        store_row32_bf16(v, p.D, row, nb * BN + c * 32, M, N, p.accumulate);
+      const int col0 = wi.nb * BN;
+      for (int h = 0; h < wi.nh; ++h) {
+        const int row = (wi.mh0 + h) * 2 * BM + static_cast<int>(rank) * BM + q * 32 + lane;
+        const uint32_t acc = tmem + static_cast<uint32_t>(h * BN) + (static_cast<uint32_t>(q * 32) << 16);
+        // Two chunks of 32 columns in flight: the next chunk's load overlaps
+        // this chunk's conversion and stores.
+        uint32_t va[32], vb[32];
+        tmem_ld_32x32b_x32(acc, va);
+#pragma unroll
+        for (int c = 0; c < BN / 32; c += 2) {
+          tmem_wait_ld_regs(va);
+          tmem_ld_32x32b_x32(acc + (c + 1) * 32, vb);
+          store_row32_bf16(va, p.D, row, col0 + c * 32, M, N, p.accumulate);
+          tmem_wait_ld_regs(vb);
+          if (c + 2 < BN / 32) tmem_ld_32x32b_x32(acc + (c + 2) * 32, va);
+          store_row32_bf16(vb, p.D, row, col0 + (c + 1) * 32, M, N, p.accumulate);
+        }
       }
-      // Hand the accumulator buffer back to the even CTA's MMA thread.
+      // Hand the accumulators back to the even CTA's MMA thread.
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * static_cast<uint32_t>(buf));
+      if (lane == 0) mbar_arrive_cluster(acc_empty0);
     }
   } else if (warp < kCodeWarp) {
     // Weight decoders.  Group g takes the pipeline steps it with
@@ -375,11 +442,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sB0 = smem_u32(sB), sC0 = smem_u32(sC);
     int it = 0;
     bool ok = true;
-    for (int t = pair; t < total_tiles && ok; t += npairs) {
-      int mb, nb;
-      pair_tile_coords(t, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
-      const int64_t base = kBwd ? (static_cast<int64_t>(nb) * BN + static_cast<int64_t>(rank) * BNH) / kBlock
-                                : static_cast<int64_t>(nb) * BN + static_cast<int64_t>(rank) * BNH;
+    for (int t = pair; t < items && ok; t += npairs) {
+      const WorkItem wi = work_item(t, p, m_tiles, n_tiles, m256);
+      if (wi.nh == 0) continue;
+      const int64_t nh0 = static_cast<int64_t>(wi.nb) * BN + static_cast<int64_t>(rank) * BNH;
+      const int64_t base = kBwd ? nh0 / kBlock : nh0;
       for (int i = 0; i < k_iters; ++i, ++it) {
         if (it % kDecodeGroups != grp) continue;
         const int c = it % kCodeStages, cu = it / kCodeStages;
@@ -448,10 +515,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmS);
       int it = 0;
       bool ok = true;
-      for (int t = pair; t < total_tiles && ok; t += npairs) {
-        int mb, nb;
-        pair_tile_coords(t, m_tiles, n_tiles, p.group, p.along_n, mb, nb);
-        const int n_half = nb * BN + static_cast<int>(rank) * BNH;  // forward: first weight row; backward: first column
+      for (int t = pair; t < items && ok; t += npairs) {
+        const WorkItem wi = work_item(t, p, m_tiles, n_tiles, m256);
+        if (wi.nh == 0) continue;
+        const int n_half = wi.nb * BN + static_cast<int>(rank) * BNH;  // forward: first weight row; backward: first column
         for (int i = 0; i < k_iters; ++i, ++it) {
           const int c = it % kCodeStages, cu = it / kCodeStages;
           if (it >= kCodeStages && !mbar_wait(&cempty[c], (cu - 1) & 1, abort_flag, status, lim)) {
@@ -583,12 +650,22 @@ cudaError_t launch_gemm_nf4(const Nf4GemmArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns ? a.wait_limit_ns : kWaitLimitNs;
   p.debug_stall = a.debug_stall;
-  const int64_t m_tiles = (a.M + 2 * BM - 1) / (2 * BM), n_tiles = (N + BN - 1) / BN;
+  const int64_t m256 = (a.M + 2 * BM - 1) / (2 * BM);
+  const int64_t m_tiles = (m256 + kHalves - 1) / kHalves, n_tiles = (N + BN - 1) / BN;
   const int64_t tiles = m_tiles * n_tiles;
-  const int pairs = static_cast<int>(tiles < clusters ? tiles : clusters);
-  // HBM bytes of one 256-wide panel: A (bf16 activations) 2 B per value;
+  // Whole tiles fill complete waves of the pairs; a last partial wave that
+  // would occupy at most half of them is split into half tiles, so it takes
+  // half a wave's time.
+  const int64_t rem = tiles % clusters;
+  const int64_t split = (rem > 0 && 2 * rem <= clusters) ? rem : 0;
+  const int64_t items = tiles + split;
+  if (items > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  p.full_tiles = static_cast<int>(tiles - split);
+  p.items = static_cast<int>(items);
+  const int pairs = static_cast<int>(items < clusters ? items : clusters);
+  // HBM bytes of one tile-wide panel: A (bf16 activations) 2 B per value;
   // the weight 0.5 B of codes + 1/64 B of scale codes per value.
-  const double a_panel = 256.0 * static_cast<double>(K) * 2.0;
+  const double a_panel = static_cast<double>(kHalves * 2 * BM) * static_cast<double>(K) * 2.0;
   const double b_panel = 256.0 * static_cast<double>(K) * (0.5 + 1.0 / 64.0);
   const RasterChoice rc = choose_raster(m_tiles, n_tiles, a_panel, b_panel, static_cast<double>(kL2PanelBudget));
   p.group = rc.group;
