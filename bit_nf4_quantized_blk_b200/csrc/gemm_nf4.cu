@@ -46,7 +46,8 @@
 //   warp 1      TMEM allocation (both CTAs); in the even CTA, MMA issue:
 //               tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16,
 //               one accumulator per half
-//   warps 2-5   epilogue of this CTA's 2 x 128 accumulator rows
+//   warps 2-5   epilogue of this CTA's 2 x 128 accumulator rows (each lane
+//               one row; 32-byte stores, so a lane writes whole sectors)
 //   warps 6-13  weight decoders: two groups of four warps take alternate
 //               stages; each thread reads its block's codes and scale from
 //               the code ring, decodes the block into the stage's tile,
@@ -190,6 +191,27 @@ __device__ __forceinline__ void decode_block_to_smem(uint32_t row, uint32_t sw, 
   }
 }
 
+
+// Store 32 fp32 accumulator columns of one output row as bf16 with two
+// 32-byte stores (D rows 32-byte aligned: N % 16 == 0, 32-byte aligned base).
+// A segment that reaches past column N takes the element-wise path.
+__device__ __forceinline__ void store_row32_bf16_wide(const uint32_t (&v)[32], uint16_t* __restrict__ D, int row,
+                                                      int col, int M, int N) {
+  if (row >= M || col >= N) return;
+  if (col + 32 > N) {
+    store_row32_bf16(v, D, row, col, M, N, 0);
+    return;
+  }
+  uint32_t lo[8], hi[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    lo[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+    hi[e] = pack_bf16x2(__uint_as_float(v[16 + 2 * e]), __uint_as_float(v[16 + 2 * e + 1]));
+  }
+  uint16_t* dst = D + static_cast<int64_t>(row) * N + col;
+  st_stream_v8(dst, lo);
+  st_stream_v8(dst + 16, hi);
+}
 
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr) : "memory");
@@ -406,10 +428,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BN / 32; c += 2) {
           tmem_wait_ld_regs(va);
           tmem_ld_32x32b_x32(acc + (c + 1) * 32, vb);
-          store_row32_bf16(va, p.D, row, col0 + c * 32, M, N, p.accumulate);
+          if (p.wide_store)
+            store_row32_bf16_wide(va, p.D, row, col0 + c * 32, M, N);
+          else
+            store_row32_bf16(va, p.D, row, col0 + c * 32, M, N, p.accumulate);
           tmem_wait_ld_regs(vb);
           if (c + 2 < BN / 32) tmem_ld_32x32b_x32(acc + (c + 2) * 32, va);
-          store_row32_bf16(vb, p.D, row, col0 + (c + 1) * 32, M, N, p.accumulate);
+          if (p.wide_store)
+            store_row32_bf16_wide(vb, p.D, row, col0 + (c + 1) * 32, M, N);
+          else
+            store_row32_bf16(vb, p.D, row, col0 + (c + 1) * 32, M, N, p.accumulate);
         }
       }
       // Hand the accumulators back to the even CTA's MMA thread.
@@ -650,6 +678,7 @@ cudaError_t launch_gemm_nf4(const Nf4GemmArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns ? a.wait_limit_ns : kWaitLimitNs;
   p.debug_stall = a.debug_stall;
+  p.wide_store = !a.accumulate && N % 16 == 0 && (reinterpret_cast<uintptr_t>(a.D) & 31) == 0;
   const int64_t m256 = (a.M + 2 * BM - 1) / (2 * BM);
   const int64_t m_tiles = (m256 + kHalves - 1) / kHalves, n_tiles = (N + BN - 1) / BN;
   const int64_t tiles = m_tiles * n_tiles;

@@ -247,6 +247,7 @@ struct Nf4GemmParams {
   int accumulate;
   int* status;
   int group, along_n;  // tile raster
+  int wide_store;      // output rows 32-byte aligned and no accumulation: 32-byte stores
   int full_tiles;      // pair tiles taken whole; the ones after them are split into two halves
   int items;           // work items: full_tiles whole tiles, then the halves
   uint64_t wait_limit_ns;
