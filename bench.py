@@ -355,13 +355,22 @@ def timed(fn, steps, warmup, world, window=None):
 def timed_reps(fn, reps, warmup, before=None):
     """Per-call device times (ms) of `reps` calls after `warmup` untimed ones,
     every call bracketed by its own pair of events on the current stream;
-    `before` (untimed) runs ahead of each call.  All calls are enqueued before
-    the host waits, so host launch latency stays outside the intervals."""
+    `before` (untimed) runs ahead of each call.  A device-side sleep queued
+    first keeps the GPU busy while the host enqueues every timed call, so the
+    calls run back to back and no interval holds time the device spent
+    waiting for the host to launch the call's kernels."""
     for _ in range(warmup):
         if before is not None:
             before(0)
         fn()
     torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    if before is not None:
+        before(0)
+    fn()
+    host_s = time.perf_counter() - t0  # host time to enqueue one call
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(min(2.0, 2.0 * reps * host_s + 1e-3) * 2.0e9))  # cycles at about 2 GHz
     evs = []
     for i in range(reps):
         if before is not None:

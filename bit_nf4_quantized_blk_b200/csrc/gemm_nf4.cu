@@ -48,14 +48,19 @@
 //               one accumulator per half
 //   warps 2-5   epilogue of this CTA's 2 x 128 accumulator rows (each lane
 //               one row; 32-byte stores, so a lane writes whole sectors)
-//   warps 6-13  weight decoders: two groups of four warps take alternate
+//   warps 6-8, 10-12, 14, 15
+//               weight decoders: two groups of four warps take alternate
 //               stages; each thread reads its block's codes and scale from
 //               the code ring, decodes the block into the stage's tile,
 //               fences its shared-memory writes for the async proxy, and its
 //               warp arrives on the even CTA's decoded-stage barrier (fullB)
 //               with a CTA-scope arrive (mbar_arrive_remote)
-//   warp 14     code ring producer: per stage, this CTA's packed codes and
+//   warp 9      code ring producer: per stage, this CTA's packed codes and
 //               decoded block scales by TMA into a 4-slot ring
+//   warp 13     idle
+// No decoder shares the MMA warp's scheduler (warp % 4 == 1): decoders there
+// take issue slots from the MMA issue and slow the tensor pipe by 10-15%;
+// only the light code-ring producer and one epilogue warp sit beside it.
 // Tiles are whole (512 rows) except in a last partial wave that would use at
 // most half of the pairs: those tiles are split into their two 256-row
 // halves, which run on twice as many pairs in half the time.
@@ -89,8 +94,13 @@ constexpr int B_TILE = BNH * BK * 2;         // 16 KB
 constexpr int TMEM_COLS = 512;               // one 128 x 256 fp32 accumulator per half, per CTA
 constexpr int kDecodeGroups = 2;
 constexpr int kFirstDecodeWarp = 6;
-constexpr int kCodeWarp = kFirstDecodeWarp + 4 * kDecodeGroups;  // producer of the code ring
-constexpr int kThreads = 32 * (kCodeWarp + 1);
+constexpr int kCodeWarp = 9;     // producer of the code ring
+constexpr int kThreads = 32 * 16;
+// Decoder index 0..7 of a warp (-1: not a decoder): warps 6..15 except those
+// on the MMA warp's scheduler (9, 13).
+__device__ __forceinline__ int decoder_index(int warp) {
+  return (warp < kFirstDecodeWarp || (warp & 3) == 1) ? -1 : (warp - kFirstDecodeWarp) - ((warp - 5) >> 2);
+}
 constexpr int kDecodedArrivals = 2 * 4;    // the four decode warps of each CTA that handle a stage
 // Code ring (per CTA): a stage's packed codes (4 KB) and decoded block scales
 // (fp32 boxes of 4 blocks per weight row: 2 KB forward, 1 KB backward).
@@ -445,91 +455,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0);
     }
-  } else if (warp < kCodeWarp) {
+  } else if (warp != kCodeWarp) {
     // Weight decoders.  Group g takes the pipeline steps it with
     // it % kDecodeGroups == g; thread `tid` writes one 128-byte row of the
     // stage's B tile from its block's codes and scale in the code ring.  No
     // decoder thread loads from global memory, so its release-arrives never
     // wait on loads in flight.
-    const int dw = warp - kFirstDecodeWarp;
-    const int grp = dw >> 2;
-    const int tid = ((dw & 3) << 5) | lane;
-    const uint32_t row_off = kBwd ? static_cast<uint32_t>((tid >> 6) * 8192 + (tid & 63) * 128)
-                                  : static_cast<uint32_t>(tid * 128);
-    const uint32_t sw = static_cast<uint32_t>(tid & 7);
-    // this thread's codes (32 bytes) and scale in a code slot
-    const uint32_t code_off = kBwd ? static_cast<uint32_t>((tid >> 6) * 2048 + (tid & 63) * 32)
-                                   : static_cast<uint32_t>(tid * 32);
-    const uint32_t scale_row = kBwd ? static_cast<uint32_t>(kCodeBytes + (tid & 63) * 16)
-                                    : static_cast<uint32_t>(kCodeBytes + tid * 16);
-    float L[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) L[j] = codebook_level(p.codebook, j);
-    const int64_t kblocks = p.Kw / kBlock;
-    const uint32_t decoded0 = map_to_cta(&decoded[0], 0);
-    const uint32_t sB0 = smem_u32(sB), sC0 = smem_u32(sC);
-    int it = 0;
-    bool ok = true;
-    for (int t = pair; t < items && ok; t += npairs) {
-      const WorkItem wi = work_item(t, p, m_tiles, n_tiles, m256);
-      if (wi.nh == 0) continue;
-      const int64_t nh0 = static_cast<int64_t>(wi.nb) * BN + static_cast<int64_t>(rank) * BNH;
-      const int64_t base = kBwd ? nh0 / kBlock : nh0;
-      for (int i = 0; i < k_iters; ++i, ++it) {
-        if (it % kDecodeGroups != grp) continue;
-        const int c = it % kCodeStages, cu = it / kCodeStages;
-        const int s = it % STAGES, u = it / STAGES;
-        if (i < num_k) {
-          // this thread's block: valid row and column, else a zero row
-          bool valid;
-          uint32_t kq;  // the block's column within its 4-block scale box
-          if constexpr (!kBwd) {
-            valid = base + tid < p.Nw;
-            kq = static_cast<uint32_t>(i & 3);
+    const int dw = decoder_index(warp);
+    if (dw >= 0) {  // (warp 13 idles)
+      const int grp = dw >> 2;
+      const int tid = ((dw & 3) << 5) | lane;
+      const uint32_t row_off = kBwd ? static_cast<uint32_t>((tid >> 6) * 8192 + (tid & 63) * 128)
+                                    : static_cast<uint32_t>(tid * 128);
+      const uint32_t sw = static_cast<uint32_t>(tid & 7);
+      // this thread's codes (32 bytes) and scale in a code slot
+      const uint32_t code_off = kBwd ? static_cast<uint32_t>((tid >> 6) * 2048 + (tid & 63) * 32)
+                                     : static_cast<uint32_t>(tid * 32);
+      const uint32_t scale_row = kBwd ? static_cast<uint32_t>(kCodeBytes + (tid & 63) * 16)
+                                      : static_cast<uint32_t>(kCodeBytes + tid * 16);
+      float L[16];
+  #pragma unroll
+      for (int j = 0; j < 16; ++j) L[j] = codebook_level(p.codebook, j);
+      const int64_t kblocks = p.Kw / kBlock;
+      const uint32_t decoded0 = map_to_cta(&decoded[0], 0);
+      const uint32_t sB0 = smem_u32(sB), sC0 = smem_u32(sC);
+      int it = 0;
+      bool ok = true;
+      for (int t = pair; t < items && ok; t += npairs) {
+        const WorkItem wi = work_item(t, p, m_tiles, n_tiles, m256);
+        if (wi.nh == 0) continue;
+        const int64_t nh0 = static_cast<int64_t>(wi.nb) * BN + static_cast<int64_t>(rank) * BNH;
+        const int64_t base = kBwd ? nh0 / kBlock : nh0;
+        for (int i = 0; i < k_iters; ++i, ++it) {
+          if (it % kDecodeGroups != grp) continue;
+          const int c = it % kCodeStages, cu = it / kCodeStages;
+          const int s = it % STAGES, u = it / STAGES;
+          if (i < num_k) {
+            // this thread's block: valid row and column, else a zero row
+            bool valid;
+            uint32_t kq;  // the block's column within its 4-block scale box
+            if constexpr (!kBwd) {
+              valid = base + tid < p.Nw;
+              kq = static_cast<uint32_t>(i & 3);
+            } else {
+              const int64_t kb = base + (tid >> 6);
+              valid = static_cast<int64_t>(i) * BK + (tid & 63) < p.Nw && kb < kblocks;
+              kq = static_cast<uint32_t>(kb & 3);
+            }
+            if (!warp_wait(&cfull[c], cu & 1, abort_flag, status, lim, false)) {
+              ok = false;
+              break;
+            }
+            const uint32_t slot = sC0 + static_cast<uint32_t>(c * CODE_SLOT);
+            uint32_t w[8];
+            ld_shared_v4(slot + code_off, w[0], w[1], w[2], w[3]);
+            ld_shared_v4(slot + code_off + 16, w[4], w[5], w[6], w[7]);
+            const float a = ld_shared_f32(slot + scale_row + 4 * kq);
+            if (it >= STAGES && !warp_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim, false)) {
+              ok = false;
+              break;
+            }
+            const uint32_t row = sB0 + static_cast<uint32_t>(s * B_TILE) + row_off;
+            if (valid) {
+              decode_block_to_smem(row, sw, w, a, L);
+            } else {
+  #pragma unroll
+              for (int j = 0; j < 8; ++j) st_shared_v4(row + (static_cast<uint32_t>(j) << 4), 0u, 0u, 0u, 0u);
+            }
+            // One proxy fence orders this thread's code-slot reads before the
+            // slot's next TMA refill and its tile writes before the MMA's reads.
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive_remote(decoded0 + 8u * static_cast<uint32_t>(s));
+              mbar_arrive(&cempty[c]);
+            }
           } else {
-            const int64_t kb = base + (tid >> 6);
-            valid = static_cast<int64_t>(i) * BK + (tid & 63) < p.Nw && kb < kblocks;
-            kq = static_cast<uint32_t>(kb & 3);
-          }
-          if (!warp_wait(&cfull[c], cu & 1, abort_flag, status, lim, false)) {
-            ok = false;
-            break;
-          }
-          const uint32_t slot = sC0 + static_cast<uint32_t>(c * CODE_SLOT);
-          uint32_t w[8];
-          ld_shared_v4(slot + code_off, w[0], w[1], w[2], w[3]);
-          ld_shared_v4(slot + code_off + 16, w[4], w[5], w[6], w[7]);
-          const float a = ld_shared_f32(slot + scale_row + 4 * kq);
-          if (it >= STAGES && !warp_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim, false)) {
-            ok = false;
-            break;
-          }
-          const uint32_t row = sB0 + static_cast<uint32_t>(s * B_TILE) + row_off;
-          if (valid) {
-            decode_block_to_smem(row, sw, w, a, L);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) st_shared_v4(row + (static_cast<uint32_t>(j) << 4), 0u, 0u, 0u, 0u);
-          }
-          // One proxy fence orders this thread's code-slot reads before the
-          // slot's next TMA refill and its tile writes before the MMA's reads.
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive_remote(decoded0 + 8u * static_cast<uint32_t>(s));
-            mbar_arrive(&cempty[c]);
-          }
-        } else {
-          // The rank step: its operands come by TMA.  Every stage still gets
-          // this warp's arrivals, so the barriers' phases follow the slots' uses.
-          if (!warp_wait(&cfull[c], cu & 1, abort_flag, status, lim, false) ||
-              (it >= STAGES && !warp_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim, false))) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
-            mbar_arrive_remote(decoded0 + 8u * static_cast<uint32_t>(s));
-            mbar_arrive(&cempty[c]);
+            // The rank step: its operands come by TMA.  Every stage still gets
+            // this warp's arrivals, so the barriers' phases follow the slots' uses.
+            if (!warp_wait(&cfull[c], cu & 1, abort_flag, status, lim, false) ||
+                (it >= STAGES && !warp_wait(&empty[s], (u - 1) & 1, abort_flag, status, lim, false))) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) {
+              mbar_arrive_remote(decoded0 + 8u * static_cast<uint32_t>(s));
+              mbar_arrive(&cempty[c]);
+            }
           }
         }
       }
