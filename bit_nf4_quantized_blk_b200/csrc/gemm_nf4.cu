@@ -42,7 +42,7 @@
 //   drains it while the producers already fill the next tile's stages.
 //   warp 0      TMA producer of this CTA's 2 x 128 rows of A (X or dY) per
 //               stage, and of the rank step's tiles; the even CTA arms the
-//               stage's copy barrier (fullA) with both CTAs' bytes
+//               stage's barrier (full) with both CTAs' bytes
 //   warp 1      TMEM allocation (both CTAs); in the even CTA, MMA issue:
 //               tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16,
 //               one accumulator per half
@@ -53,8 +53,8 @@
 //               stages; each thread reads its block's codes and scale from
 //               the code ring, decodes the block into the stage's tile,
 //               fences its shared-memory writes for the async proxy, and its
-//               warp arrives on the even CTA's decoded-stage barrier (fullB)
-//               with a CTA-scope arrive (mbar_arrive_remote)
+//               warp arrives on the even CTA's stage barrier (full) with a
+//               CTA-scope arrive (mbar_arrive_remote)
 //   warp 9      code ring producer: per stage, this CTA's packed codes and
 //               decoded block scales by TMA into a 4-slot ring
 //   warp 13     idle
@@ -64,11 +64,14 @@
 // Tiles are whole (512 rows) except in a last partial wave that would use at
 // most half of the pairs: those tiles are split into their two 256-row
 // halves, which run on twice as many pairs in half the time.
-// The MMA issuer waits on both barriers of a stage.  Keeping the copies on a
-// barrier of their own lets a teardown wait for exactly the copies in
-// flight: the even producer waits for the last stages' copies of both CTAs
-// and then signals the odd CTA (`drained`), which waits for that before its
-// shared memory can go.
+// A stage is complete when its copies have landed and the eight decode warps
+// of the pair have arrived: one barrier, so the MMA issuer checks one phase
+// per stage (each check costs about 100 cycles even when the phase is
+// complete; a non-blocking test of the next stage placed between two halves'
+// MMAs delays the second half's issue and costs more than it saves).  At
+// teardown the even producer waits for the
+// last stages' phases (so for the copies of both CTAs) and then signals the
+// odd CTA (`drained`), which waits for that before its shared memory can go.
 // The rank-r LoRA term is one more pipeline step of ceil(r/16) MMAs into the
 // same accumulator, its operands loaded by TMA.  No TMA load uses cluster
 // multicast; the MMA's tcgen05.commit is delivered to both CTAs of the pair
@@ -264,9 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE;
   uint8_t* sC = sB + STAGES * B_TILE;    // code ring
-  uint64_t* full = reinterpret_cast<uint64_t*>(sC + kCodeStages * CODE_SLOT);  // fullA: TMA bytes (even CTA)
-  uint64_t* decoded = full + STAGES;      // fullB: decode warps of both CTAs (even CTA)
-  uint64_t* empty = decoded + STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sC + kCodeStages * CODE_SLOT);  // even CTA: copies + decode warps
+  uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;    // the accumulators hold a finished tile
   uint64_t* acc_empty = acc_full + 1;     // even CTA: both CTAs' epilogues drained them
   uint64_t* drain = acc_empty + 1;
@@ -290,8 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&decoded[s], kDecodedArrivals);
+      mbar_init(&full[s], 1 + kDecodedArrivals);  // the producer's expect-tx arrive and the decode warps
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -387,8 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int i = 0; i < k_iters; ++i, ++it) {
           const int s = it % STAGES, u = it / STAGES;
-          if (!mbar_wait_cluster(&full[s], u & 1, abort_flag, status, lim) ||
-              !mbar_wait_cluster(&decoded[s], u & 1, abort_flag, status, lim)) {
+          if (!mbar_wait_cluster(&full[s], u & 1, abort_flag, status, lim)) {
             ok = false;
             break;
           }
@@ -477,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   #pragma unroll
       for (int j = 0; j < 16; ++j) L[j] = codebook_level(p.codebook, j);
       const int64_t kblocks = p.Kw / kBlock;
-      const uint32_t decoded0 = map_to_cta(&decoded[0], 0);
+      const uint32_t decoded0 = map_to_cta(&full[0], 0);
       const uint32_t sB0 = smem_u32(sB), sC0 = smem_u32(sC);
       int it = 0;
       bool ok = true;
