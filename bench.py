@@ -816,7 +816,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}",
                    **({"streams": "projections alternate over 2 streams"} if args.streams == 2 else {})},
         "roofline": {"bound": "tensor",
-                     "kernel": "gemm_nf4_kernel (tcgen05 pair-CTA 256x256 tile, 4-bit weight decoded into shared memory)",
+                     "kernel": "gemm_nf4_kernel (tcgen05 pair-CTA 512x256 tile, 4-bit weight decoded into shared memory)",
                      "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tflops / peak,
                      "peak_source": f"{peak_src} bf16_tflops (burst; the timed region is "
                                     f"{args.steps * ms / 1e3:.2f} s at the sampled clock)",

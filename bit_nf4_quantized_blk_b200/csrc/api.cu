@@ -784,7 +784,7 @@ qlora_status linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
   const uint16_t* B2 = b_direct ? B : at<uint16_t>(ws, lay.bpad);
   const int64_t ldb2 = b_direct ? r : kRankPad;
   if (!dense) {
-    Timed tm(kFamGemm, s);
+    Timed tm(kFamGemm, s, 2);  // block-scale pre-pass + GEMM
     return gemm_status(launch_linear_gemm_nf4(w, at<float>(ws, lay.scales), X, M, at<uint16_t>(ws, lay.us), B2, r,
                                               ldb2, Y, 0, status, false, s, diag.wait_limit_ns, diag.debug_stall));
   }
@@ -897,7 +897,7 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
     }
   }
   if (dX != nullptr && !dense) {  // dX = dY W_hat + s V A, W_hat decoded in the GEMM, A [r, K] MN-major
-    Timed tm(kFamGemm, s);
+    Timed tm(kFamGemm, s, 2);  // block-scale pre-pass + GEMM
     e = launch_linear_gemm_nf4(w, at<float>(ws, lay.scales), dY, M, at<uint16_t>(ws, lay.vs), A, r, 0, dX, accumulate,
                                status, true, s);
     if (e != cudaSuccess) return gemm_status(e);
