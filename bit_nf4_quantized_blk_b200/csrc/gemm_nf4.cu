@@ -66,10 +66,10 @@
 // halves, which run on twice as many pairs in half the time.
 // A stage is complete when its copies have landed and the eight decode warps
 // of the pair have arrived: one barrier, so the MMA issuer checks one phase
-// per stage (each check costs about 100 cycles even when the phase is
-// complete; a non-blocking test of the next stage placed between two halves'
-// MMAs delays the second half's issue and costs more than it saves).  At
-// teardown the even producer waits for the
+// per stage.  The issuer is a single thread whose scalar work between two
+// stages' MMAs delays the tensor pipe, so its loop is kept lean: the slot
+// descriptors are the slot-0 descriptors plus constant offsets, and a full
+// stage's eight MMAs are unrolled.  At teardown the even producer waits for the
 // last stages' phases (so for the copies of both CTAs) and then signals the
 // odd CTA (`drained`), which waits for that before its shared memory can go.
 // The rank-r LoRA term is one more pipeline step of ceil(r/16) MMAs into the
@@ -375,6 +375,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = idesc_bf16_f32(2 * BM, BN, kBwd);
+      // Stage descriptors: the start-address field (bits 0..13, address >> 4)
+      // of slot s is the slot-0 descriptor's plus the slot's offset >> 4
+      // (shared addresses stay below 256 KB, so the field cannot overflow).
+      const uint64_t a_desc0 = smem_desc_k128(smem_u32(sA));
+      const uint64_t b_desc0 = kBwd ? smem_desc_mn128(smem_u32(sB), 8192, 1024) : smem_desc_k128(smem_u32(sB));
+      constexpr uint32_t kAStage16 = A_STAGE >> 4, kATile16 = A_TILE >> 4, kBTile16 = B_TILE >> 4;
+      // One K = 16 step: A (K-major) +32 bytes inside the swizzle atom;
+      // B +32 bytes (K-major) or +2 atoms of 8 rows = 2048 bytes (MN-major).
+      constexpr uint32_t kBStep = kBwd ? (2048 >> 4) : 2;
       int it = 0, tl = 0;
       // Diagnostic launch: the issuer first waits on a barrier nothing
       // arrives at, so its wait runs out and the whole pair takes the abort
@@ -386,24 +395,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tl > 0 && !mbar_wait_cluster(acc_empty, (tl - 1) & 1, abort_flag, status, lim)) break;
         ++tl;
         tc_fence_after();
+        const bool two = wi.nh == 2;
         for (int i = 0; i < k_iters; ++i, ++it) {
-          const int s = it % STAGES, u = it / STAGES;
+          const uint32_t s = static_cast<uint32_t>(it) % STAGES, u = static_cast<uint32_t>(it) / STAGES;
           if (!mbar_wait_cluster(&full[s], u & 1, abort_flag, status, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nsteps = i < num_k ? BK / 16 : r_steps;
-          const uint64_t bdesc = kBwd ? smem_desc_mn128(smem_u32(sB + s * B_TILE), 8192, 1024)
-                                      : smem_desc_k128(smem_u32(sB + s * B_TILE));
-          // One K = 16 step: A (K-major) +32 bytes inside the swizzle atom;
-          // B +32 bytes (K-major) or +2 atoms of 8 rows = 2048 bytes (MN-major).
-          const uint32_t bstep = kBwd ? (2048 >> 4) : 2;
-          for (int h = 0; h < wi.nh; ++h) {
-            const uint32_t acc = tmem + static_cast<uint32_t>(h * BN);
-            const uint64_t adesc = smem_desc_k128(smem_u32(sA + s * A_STAGE + h * A_TILE));
-            for (int kk = 0; kk < nsteps; ++kk)
-              tc_mma_bf16_ss_pair(acc, adesc + 2 * kk, bdesc + bstep * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t ad = a_desc0 + s * kAStage16, bd = b_desc0 + s * kBTile16;
+          if (i > 0 && i < num_k) {  // a full stage after the first: four K steps per half
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) tc_mma_bf16_ss_pair(tmem, ad + 2 * kk, bd + kBStep * kk, idesc, 1u);
+            if (two) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                tc_mma_bf16_ss_pair(tmem + BN, ad + kATile16 + 2 * kk, bd + kBStep * kk, idesc, 1u);
+            }
+          } else {  // the tile's first stage (accumulators start over) or the rank step
+            const int nsteps = i < num_k ? BK / 16 : r_steps;
+            for (int h = 0; h < wi.nh; ++h)
+              for (int kk = 0; kk < nsteps; ++kk)
+                tc_mma_bf16_ss_pair(tmem + static_cast<uint32_t>(h * BN), ad + h * kATile16 + 2 * kk,
+                                    bd + kBStep * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[s], 0x3);
         }
