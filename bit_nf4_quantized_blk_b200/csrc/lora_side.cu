@@ -33,7 +33,7 @@ constexpr int kTileCols = 64;   // columns (c) per tile
 // four CTAs share an SM, four TMA-issuing threads per SM instead of two with an
 // 8-deep ring; that moved the side kernels of a 7B layer step from 1.17 to
 // 1.07 ms (the same bytes in flight, more issuers).
-constexpr int kStages = 4;      // TMA ring depth
+constexpr int kStages = 3;      // TMA ring depth (several CTAs per SM keep more tiles in flight)
 constexpr int kCtasPerSm = 4;   // grid sizing target (148 SMs)
 constexpr int kInTile = kTileRows * 128;  // one [64][64] bf16 tile, 128B-swizzled
 constexpr int kThreads = 160;   // warp 0: TMA producer; warps 1-4: MMA consumers
@@ -481,7 +481,7 @@ cudaError_t launch_colsum(const uint16_t* In, int64_t M, int64_t C, const uint16
 // Partials are [blocks][rows][r16] fp32; vdb_finalize_kernel sums them in
 // block order.
 template <int NT, int TC>
-__global__ void __launch_bounds__(kThreads) vdb_kernel(const __grid_constant__ CUtensorMap tmG,
+__global__ void __launch_bounds__(kThreads, 5) vdb_kernel(const __grid_constant__ CUtensorMap tmG,
                                                        const __grid_constant__ CUtensorMap tmB,
                                                        const __grid_constant__ CUtensorMap tmHi,
                                                        const __grid_constant__ CUtensorMap tmLo, int64_t M, int64_t N,
@@ -673,10 +673,12 @@ __global__ void vdb_finalize_kernel(const float* __restrict__ vpart, int ncb, co
 
 namespace {
 
-// Column tiles per CTA of vdb_kernel (its dB accumulators live in registers,
-// eight column tiles at rank <= 16).
-constexpr int vdb_tc(int nt) { return nt <= 2 ? 8 : nt <= 4 ? 4 : 2; }
-constexpr int kVdbCtasTarget = 2 * 148;
+// Column tiles per CTA of vdb_kernel (its dB accumulators live in registers):
+// four at rank <= 16 keep it at 72 registers, so five CTAs share an SM
+// (eight tiles needed 128 registers, which left room for three).
+constexpr int vdb_tc(int nt) { return nt <= 4 ? 4 : 2; }
+constexpr int kVdbCtasPerSm = 5;
+constexpr int kVdbCtasTarget = kVdbCtasPerSm * 148;
 
 struct VdbGrid {
   int ncb, ntb, tmc;

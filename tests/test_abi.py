@@ -74,7 +74,7 @@ def test_linear_ws_bytes(lib):
     # the fused path holds no dense copy of the weight; the dense-weight
     # ablation path adds one of N x K bf16 for the tensor-core calls (M > 16)
     fused = binding.qlora_linear_ws_bytes(8192, 14336, 4096, 16)
-    assert 0 < fused < 14336 * 4096
+    assert 0 < fused < 14336 * 4096 * 2  # smaller than a bf16 copy of the weight alone
     with binding.weight_path(binding.WEIGHT_PATH_DENSE):
         # the dense arm holds the N x K bf16 copy (it needs no decoded-scale array, N x K / 64 fp32)
         assert binding.qlora_linear_ws_bytes(8192, 14336, 4096, 16) >= fused + 14336 * 4096 * 2 - 14336 * 64 * 4
