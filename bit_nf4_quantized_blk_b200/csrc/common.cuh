@@ -159,6 +159,48 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// try_wait that may suspend the thread for up to `hint_ns` (it resumes as soon
+// as the phase completes): a waiting warp then takes no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, bool cluster, uint32_t hint_ns) {
+  uint32_t ok;
+  if (cluster)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+  return ok != 0;
+}
+
+// mbar_wait / mbar_wait_cluster for a thread whose wait is long and whose
+// scheduler is shared with latency-critical work: each try may suspend it.
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity, bool cluster,
+                                                  volatile int* abort_flag, int* status,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  constexpr uint32_t kHintNs = 2000;
+  if (mbar_try_wait_suspend(bar, parity, cluster, kHintNs)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait_suspend(bar, parity, cluster, kHintNs)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      raise_status(status, QLORA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Same, ignoring the abort flag (teardown waits for work already in flight).
 // Always the full limit: copies and MMAs already issued land within it.
 __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity, int* status) {

@@ -239,12 +239,14 @@ __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
 // Warp-wide bounded wait: lane 0 polls (the other lanes idle at the shuffle,
 // so a waiting warp takes few issue slots), then every lane acquires the
 // completed phase itself.  Returns false (warp-uniformly) on abort / timeout.
+// `suspend`: lane 0's tries may suspend it (a long wait beside the MMA warp).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
-                                          uint64_t lim, bool cluster) {
+                                          uint64_t lim, bool cluster, bool suspend = false) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0)
-    ok = cluster ? mbar_wait_cluster(bar, parity, abort_flag, status, lim)
-                 : mbar_wait(bar, parity, abort_flag, status, lim);
+    ok = suspend   ? mbar_wait_suspend(bar, parity, cluster, abort_flag, status, lim)
+         : cluster ? mbar_wait_cluster(bar, parity, abort_flag, status, lim)
+                   : mbar_wait(bar, parity, abort_flag, status, lim);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   if (ok) {
     if (cluster)
@@ -436,7 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = pair; t < items; t += npairs) {
       const WorkItem wi = work_item(t, p, m_tiles, n_tiles, m256);
       if (wi.nh == 0) continue;
-      const bool ok = warp_wait(acc_full, tl & 1, abort_flag, status, lim, true);
+      // The tile's whole main loop passes meanwhile; warp 5 shares the MMA
+      // warp's scheduler, so the waiting lane sleeps between tries.
+      const bool ok = warp_wait(acc_full, tl & 1, abort_flag, status, lim, true, true);
       ++tl;
       if (!ok) break;
       tc_fence_after();
@@ -575,7 +579,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_half = wi.nb * BN + static_cast<int>(rank) * BNH;  // forward: first weight row; backward: first column
         for (int i = 0; i < k_iters; ++i, ++it) {
           const int c = it % kCodeStages, cu = it / kCodeStages;
-          if (it >= kCodeStages && !mbar_wait(&cempty[c], (cu - 1) & 1, abort_flag, status, lim)) {
+          // (this warp shares the MMA warp's scheduler: it sleeps between tries)
+          if (it >= kCodeStages && !mbar_wait_suspend(&cempty[c], (cu - 1) & 1, false, abort_flag, status, lim)) {
             ok = false;
             break;
           }
