@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqlora_nf4.so")
 
-SOURCES = ["api.cu", "quantize.cu", "dequant.cu", "gemv.cu", "lora_side.cu", "gemm_tc.cu", "gemm_nf4.cu", "merge.cu"]
+SOURCES = ["api.cu", "quantize.cu", "dequant.cu", "gemv.cu", "lora_side.cu", "gemm_tc.cu", "gemm_nf4.cu", "merge.cu", "vdb_tc.cu"]
 
 NVCC_FLAGS = [
     "-O3",

@@ -345,7 +345,7 @@ int64_t max_group_chunks(const qlora_nf4_weight* outs, int32_t count) {
 
 // Linear workspace layout.
 struct LinearWs {
-  size_t wbf, scales, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, vdbpart, gu, gy, total;
+  size_t wbf, scales, us, uhi, ulo, vs, vhi, vlo, bpad, part, skpart, vdbpart, bt, uht, ult, gu, gy, total;
 };
 
 LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, bool dense) {
@@ -373,7 +373,12 @@ LinearWs linear_ws_layout(int64_t M, int64_t N, int64_t K, bool dense) {
   l.part = take(p1 > p2 ? p1 : p2);
   const size_t s1 = skinny_partial_bytes(M, N), s2 = skinny_partial_bytes(M, K);
   l.skpart = take(s1 > s2 ? s1 : s2);
-  l.vdbpart = take(M > kGemvMaxM ? vdb_partial_bytes(M, N) : 0);
+  // The tensor-core V / dB pass: its partials and the transposed B and U split.
+  const bool vdb = M > kGemvMaxM;
+  l.vdbpart = take(vdb ? vdb_tc_partial_bytes(M, N) : 0);
+  l.bt = take(vdb ? static_cast<size_t>(16) * static_cast<size_t>(N) * 2 : 0);
+  l.uht = take(vdb ? static_cast<size_t>(16) * static_cast<size_t>(vdb_tc_ldm(M)) * 2 : 0);
+  l.ult = take(vdb ? static_cast<size_t>(16) * static_cast<size_t>(vdb_tc_ldm(M)) * 2 : 0);
   // Decode path (M <= 16): U partials and, for K > 4096, per-chunk fp32 outputs.
   const bool decode = M <= kGemvMaxM;
   l.gu = take(decode ? static_cast<size_t>(gemv_upart_count(K)) * kGemvMaxM * kRankPad * 4 : 0);
@@ -870,10 +875,11 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
     // V = dY B (s*V for the dX rank step, hi/lo for dA) and dB = s dY^T U in one pass over dY.
     e = u_hilo();
     if (e != cudaSuccess) return from_cuda(e);
-    Timed tm(kFamSide, s, 2);
-    e = launch_vdb(dY, M, N, Bk, ldbk, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), r, scale,
-                   at<float>(ws, lay.vdbpart), at<uint16_t>(ws, lay.vs), at<uint16_t>(ws, lay.vhi),
-                   at<uint16_t>(ws, lay.vlo), dB, status, s);
+    Timed tm(kFamSide, s, 3);  // the rank transposes, the pass, the reduction
+    e = launch_vdb_tc(dY, M, N, Bk, ldbk, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), r, scale,
+                      at<float>(ws, lay.vdbpart), at<uint16_t>(ws, lay.bt), at<uint16_t>(ws, lay.uht),
+                      at<uint16_t>(ws, lay.ult), at<uint16_t>(ws, lay.vs), at<uint16_t>(ws, lay.vhi),
+                      at<uint16_t>(ws, lay.vlo), dB, status, s);
     if (e != cudaSuccess) return from_cuda(e);
   } else {
     // V = dY B (bf16 s*V for the dX rank step; hi/lo split for dA).

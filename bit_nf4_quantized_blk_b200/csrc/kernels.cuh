@@ -173,17 +173,30 @@ size_t colsum_partial_bytes(int64_t M, int64_t C);
 cudaError_t launch_colsum(const uint16_t* In, int64_t M, int64_t C, const uint16_t* hi, const uint16_t* lo, int r,
                           float scale, float* part, float* dst, bool dst_rc, int* status, cudaStream_t stream);
 
-// Both rank-r products of the backward from one pass over G = dY [M][N]:
-// V = G B written as vs = s*V (bf16 [M][64]) and its hi / lo split (vhi,
-// vlo, [M][64]); dB = scale * G^T (uhi + ulo) into dB [N][r] (may be null).
-// B is [N][ldb] bf16 with r valid columns (ldb * 2 bytes a multiple of 16).
-// `part` is scratch of vdb_partial_bytes(M, N).  Ranks 1..kVdbMaxRank (wider
-// ranks use launch_skinny + launch_colsum).
+// Both rank-r products of the backward from one pass over G = dY [M][N]
+// (vdb_tc.cu, ranks 1..kVdbMaxRank; wider ranks use launch_skinny +
+// launch_colsum): V = G B written as vs = s*V (bf16 [M][64]) and its hi / lo
+// split (vhi, vlo, [M][64]); dB = scale * G^T (uhi + ulo) into dB [N][r] (may
+// be null).  B is [N][ldb] bf16 with r valid columns.
 constexpr int kVdbMaxRank = 16;
-size_t vdb_partial_bytes(int64_t M, int64_t N);
-cudaError_t launch_vdb(const uint16_t* G, int64_t M, int64_t N, const uint16_t* B, int64_t ldb, const uint16_t* uhi,
-                       const uint16_t* ulo, int r, float scale, float* part, uint16_t* vs, uint16_t* vhi,
-                       uint16_t* vlo, float* dB, int* status, cudaStream_t stream);
+// The pass writes partials [ncb][M][16] and [ntb][N][16] fp32 (`part`, vdb_tc_partial_bytes
+// bytes); bt [16][N], uht and ult [16][vdb_tc_ldm(M)] are bf16 scratch for
+// B^T and the transposed U split (uhi / ulo [M][64] as written by
+// launch_split_hilo or launch_skinny).
+struct VdbTcGrid {
+  int ct, tt, ncb, ntb;  // column / token tiles per CTA; column / token blocks
+};
+VdbTcGrid vdb_tc_grid(int64_t M, int64_t N);
+size_t vdb_tc_partial_bytes(int64_t M, int64_t N);
+inline int64_t vdb_tc_ldm(int64_t M) { return (M + 7) / 8 * 8; }  // 16-byte rows for TMA
+cudaError_t launch_vdb_tc(const uint16_t* G, int64_t M, int64_t N, const uint16_t* B, int64_t ldb,
+                          const uint16_t* uhi, const uint16_t* ulo, int r, float scale, float* part, uint16_t* bt,
+                          uint16_t* uht, uint16_t* ult, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,
+                          int* status, cudaStream_t stream);
+// The fixed-order reduction of vdb partials [ncb][M][16] and [ntb][N][16].
+cudaError_t launch_vdb_finalize(const float* vpart, int ncb, const float* dbpart, int ntb, int64_t M, int64_t N,
+                                int r, float scale, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,
+                                cudaStream_t stream);
 
 // Copy a bf16 [rows][r] matrix into [rows][64] zero padded, optionally from
 // the transposed source [r][rows].

@@ -15,10 +15,10 @@
 //  colsum_kernel   part[z][c][j] = sum_{m in split z} In[m][c] * S[m][j]
 //                  (dA with In = X, S = V), then colsum_reduce_kernel adds
 //                  the splits in a fixed order and applies s.
-//  vdb_kernel      the backward's two products of G in one pass over G:
-//                  V = G B and the dB partials G^T U from the same tiles,
-//                  then vdb_finalize_kernel forms s*V, the hi/lo split of V
-//                  and dB = s * (sum of the partials).
+//  vdb_finalize_kernel  after the backward's one pass over G (vdb_tc.cu:
+//                  V = G B and the dB partials G^T U on the tensor cores),
+//                  forms s*V, the hi/lo split of V and dB = s * (sum of the
+//                  partials).
 // Deterministic: every sum runs in a fixed order; no atomics.
 #include "common.cuh"
 #include "kernels.cuh"
@@ -465,175 +465,8 @@ cudaError_t launch_colsum(const uint16_t* In, int64_t M, int64_t C, const uint16
 }
 
 // ---------------------------------------------------------------------------
-// vdb: V = G B and dB = s G^T U from one pass over G = dY [M][N]
+// vdb reduction: the partials of the tensor-core V / dB pass (vdb_tc.cu)
 // ---------------------------------------------------------------------------
-// Grid (column blocks, token blocks).  CTA (zc, zm) covers up to TC column
-// tiles and `tmc` token tiles of G (64 x 64 each).  Warp 0 streams, per tile,
-// the G tile (128-byte swizzle), the 64 x r16 tile of B [N][ldb] for its
-// columns and the 64 x r16 tiles of the hi / lo split of U for its tokens
-// through a kStages-deep TMA ring.  Warps 1-4 use every G tile twice:
-//   V:  warp w owns tokens 16w..16w+15: A = the G tile, B = the B tile;
-//       accumulated over the CTA's column tiles of one token tile, then
-//       stored as the partial vpart[zc][m][j];
-//   dB: warp w owns columns 16w..16w+15: A = G^T (transposed 8x8 loads),
-//       B = U hi and lo; one accumulator per column tile of the CTA, held
-//       across its token tiles, then stored as dbpart[zm][c][j].
-// Partials are [blocks][rows][r16] fp32; vdb_finalize_kernel sums them in
-// block order.
-template <int NT, int TC>
-__global__ void __launch_bounds__(kThreads, 5) vdb_kernel(const __grid_constant__ CUtensorMap tmG,
-                                                       const __grid_constant__ CUtensorMap tmB,
-                                                       const __grid_constant__ CUtensorMap tmHi,
-                                                       const __grid_constant__ CUtensorMap tmLo, int64_t M, int64_t N,
-                                                       int tmc, float* __restrict__ vpart, float* __restrict__ dbpart,
-                                                       int* status) {
-  constexpr int kR16 = NT * 8;
-  constexpr int kSmall = 128 * kR16;  // [64][r16] bf16
-  constexpr int kStage = kInTile + 3 * kSmall;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  PipeBarriers* bars = reinterpret_cast<PipeBarriers*>(smem + kStages * kStage);
-  volatile int* abort_flag = &bars->abort_flag;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int zc = blockIdx.x, zm = blockIdx.y;
-  const int ctiles = static_cast<int>((N + kTileCols - 1) / kTileCols);
-  const int mtiles = static_cast<int>((M + kTileRows - 1) / kTileRows);
-  const int tc0 = zc * TC, tm0 = zm * tmc;
-  const int ntc = min(TC, ctiles - tc0), ntm = min(tmc, mtiles - tm0);
-  const int nsteps = ntc * ntm;  // token-tile major: step i = tm * ntc + tc
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->empty[s], 4);
-    }
-    bars->abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        const int s = i % kStages, u = i / kStages;
-        if (i >= kStages && !mbar_wait(&bars->empty[s], (u - 1) & 1, abort_flag, status)) break;
-        uint8_t* st = smem + s * kStage;
-        const int tm = i / ntc, tc = i - tm * ntc;
-        const int c = (tc0 + tc) * kTileCols, m = (tm0 + tm) * kTileRows;
-        mbar_arrive_expect_tx(&bars->full[s], kStage);
-        tma_load_2d(st, &tmG, &bars->full[s], c, m);
-        tma_load_2d(st + kInTile, &tmB, &bars->full[s], 0, c);               // B rows c..c+63
-        tma_load_2d(st + kInTile + kSmall, &tmHi, &bars->full[s], 0, m);     // U hi rows m..m+63
-        tma_load_2d(st + kInTile + 2 * kSmall, &tmLo, &bars->full[s], 0, m); // U lo rows m..m+63
-        issued = i + 1;
-      }
-      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-        mbar_wait_teardown(&bars->full[i % kStages], (i / kStages) & 1, status);
-    }
-    return;
-  }
-
-  const int cw = warp - 1;
-  const int mat = lane >> 3, rr = lane & 7;
-  const int g = lane >> 2, t4 = lane & 3;
-  float accV[NT][4];
-  float accB[TC][NT][4];
-#pragma unroll
-  for (int t = 0; t < TC; ++t)
-#pragma unroll
-    for (int i = 0; i < NT; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) accB[t][i][j] = 0.0f;
-
-  int it = 0;
-  bool ok = true;
-  for (int tm = 0; tm < ntm && ok; ++tm) {
-#pragma unroll
-    for (int i = 0; i < NT; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) accV[i][j] = 0.0f;
-#pragma unroll
-    for (int t = 0; t < TC; ++t) {
-      if (t < ntc && ok) {
-        const int s = it % kStages, u = it / kStages;
-        if (!mbar_wait(&bars->full[s], u & 1, abort_flag, status)) {
-          ok = false;
-        } else {
-          const uint32_t g_base = smem_u32(smem + s * kStage);
-          const uint32_t b_base = g_base + kInTile;
-          const uint32_t hi_base = b_base + kSmall;
-          const uint32_t lo_base = hi_base + kSmall;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            // V: rows = tokens 16cw.., k = columns 16kk..
-            uint32_t afr[4];
-            ldmatrix_x4(afr, g_base + swz(cw * 16 + (lane & 15), kk * 2 + (lane >> 4)));
-            const int c = kk * 16 + (mat & 1) * 8 + rr;
-#pragma unroll
-            for (int nt = 0; nt < NT; nt += 2) {
-              uint32_t bfr[4];
-              ldmatrix_x4_trans(bfr, b_base + c * (2 * kR16) + (nt + (mat >> 1)) * 16);
-              const uint32_t b0[2] = {bfr[0], bfr[1]};
-              const uint32_t b1[2] = {bfr[2], bfr[3]};
-              mma_bf16_16816(accV[nt], afr, b0);
-              mma_bf16_16816(accV[nt + 1], afr, b1);
-            }
-            // dB: rows = columns 16cw.., k = tokens 16kk..
-            uint32_t gfr[4];
-            ldmatrix_x4_trans(gfr, g_base + swz(kk * 16 + (mat >> 1) * 8 + rr, cw * 2 + (mat & 1)));
-            const int m = kk * 16 + (mat & 1) * 8 + rr;
-#pragma unroll
-            for (int nt = 0; nt < NT; nt += 2) {
-              const uint32_t off = m * (2 * kR16) + (nt + (mat >> 1)) * 16;
-              uint32_t bh[4], bl[4];
-              ldmatrix_x4_trans(bh, hi_base + off);
-              ldmatrix_x4_trans(bl, lo_base + off);
-              const uint32_t h0[2] = {bh[0], bh[1]}, l0[2] = {bl[0], bl[1]};
-              const uint32_t h1[2] = {bh[2], bh[3]}, l1[2] = {bl[2], bl[3]};
-              mma_bf16_16816(accB[t][nt], gfr, h0);
-              mma_bf16_16816(accB[t][nt], gfr, l0);
-              mma_bf16_16816(accB[t][nt + 1], gfr, h1);
-              mma_bf16_16816(accB[t][nt + 1], gfr, l1);
-            }
-          }
-          fence_proxy_async_shared();  // this warp's ldmatrix reads of stage s before its TMA refill
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->empty[s]);
-          ++it;
-        }
-      }
-    }
-    if (!ok) break;
-    // V partial of this token tile over the CTA's columns
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int64_t m = static_cast<int64_t>(tm0 + tm) * kTileRows + cw * 16 + g + half * 8;
-      if (m >= M) continue;
-      float* dst = vpart + (static_cast<int64_t>(zc) * M + m) * kR16;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        *reinterpret_cast<float2*>(dst + nt * 8 + 2 * t4) = make_float2(accV[nt][half * 2], accV[nt][half * 2 + 1]);
-    }
-  }
-  if (!ok) return;
-  // dB partials of the CTA's column tiles over its tokens
-#pragma unroll
-  for (int t = 0; t < TC; ++t) {
-    if (t >= ntc) continue;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int64_t c = static_cast<int64_t>(tc0 + t) * kTileCols + cw * 16 + g + half * 8;
-      if (c >= N) continue;
-      float* dst = dbpart + (static_cast<int64_t>(zm) * N + c) * kR16;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        *reinterpret_cast<float2*>(dst + nt * 8 + 2 * t4) =
-            make_float2(accB[t][nt][half * 2], accB[t][nt][half * 2 + 1]);
-    }
-  }
-}
-
 // V (fp32) = sum over column blocks of vpart, written as s*V (bf16, [M][64]
 // zero padded) and its hi / lo split; dB[c][j] = scale * sum over token
 // blocks of dbpart.  Threads [0, M*32) take pairs of V, the rest dB entries.
@@ -671,78 +504,12 @@ __global__ void vdb_finalize_kernel(const float* __restrict__ vpart, int ncb, co
   dB[c * r + j] = scale * s;
 }
 
-namespace {
-
-// Column tiles per CTA of vdb_kernel (its dB accumulators live in registers):
-// four at rank <= 16 keep it at 72 registers, so five CTAs share an SM
-// (eight tiles needed 128 registers, which left room for three).
-constexpr int vdb_tc(int nt) { return nt <= 4 ? 4 : 2; }
-constexpr int kVdbCtasPerSm = 5;
-constexpr int kVdbCtasTarget = kVdbCtasPerSm * 148;
-
-struct VdbGrid {
-  int ncb, ntb, tmc;
-};
-
-VdbGrid vdb_grid(int64_t M, int64_t N, int r) {
-  const int nt = ((r + 15) / 16) * 2;
-  const int64_t ctiles = (N + kTileCols - 1) / kTileCols, mtiles = (M + kTileRows - 1) / kTileRows;
-  VdbGrid g;
-  g.ncb = static_cast<int>((ctiles + vdb_tc(nt) - 1) / vdb_tc(nt));
-  int64_t ntb = (kVdbCtasTarget + g.ncb - 1) / g.ncb;
-  if (ntb < 1) ntb = 1;
-  if (ntb > mtiles) ntb = mtiles;
-  g.tmc = static_cast<int>((mtiles + ntb - 1) / ntb);
-  g.ntb = static_cast<int>((mtiles + g.tmc - 1) / g.tmc);
-  return g;
-}
-
-}  // namespace
-
-size_t vdb_partial_bytes(int64_t M, int64_t N) {
-  const VdbGrid g = vdb_grid(M, N, kVdbMaxRank);
-  return (static_cast<size_t>(g.ncb) * static_cast<size_t>(M) + static_cast<size_t>(g.ntb) * static_cast<size_t>(N)) *
-         static_cast<size_t>(kVdbMaxRank) * sizeof(float);
-}
-
-template <int NT>
-cudaError_t launch_vdb_nt(const CUtensorMap& tg, const CUtensorMap& tb, const CUtensorMap& thi, const CUtensorMap& tlo,
-                          int64_t M, int64_t N, const VdbGrid& grid, float* vpart, float* dbpart, int* status,
-                          cudaStream_t stream) {
-  constexpr int TC = vdb_tc(NT);
-  constexpr int kStage = kInTile + 3 * 128 * NT * 8;
-  constexpr int smem = 1024 + kStages * kStage + static_cast<int>(sizeof(PipeBarriers));
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  static DeviceOnce configured;
-  e = configured.run(dev, [] {
-    return cudaFuncSetAttribute(vdb_kernel<NT, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (e != cudaSuccess) return e;
-  vdb_kernel<NT, TC><<<dim3(static_cast<unsigned>(grid.ncb), static_cast<unsigned>(grid.ntb)), kThreads, smem,
-                       stream>>>(tg, tb, thi, tlo, M, N, grid.tmc, vpart, dbpart, status);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_vdb(const uint16_t* G, int64_t M, int64_t N, const uint16_t* B, int64_t ldb, const uint16_t* uhi,
-                       const uint16_t* ulo, int r, float scale, float* part, uint16_t* vs, uint16_t* vhi,
-                       uint16_t* vlo, float* dB, int* status, cudaStream_t stream) {
-  if (r < 1 || r > kVdbMaxRank) return cudaErrorInvalidValue;
-  const int nt = ((r + 15) / 16) * 2;
-  const VdbGrid grid = vdb_grid(M, N, r);
-  CUtensorMap tg, tb, thi, tlo;
-  if (!encode_tensor_map_2d(&tg, G, M, N, kTileRows, kTileCols)) return cudaErrorInvalidValue;
-  if (!encode_tensor_map_2d(&tb, B, N, r, kTileCols, nt * 8, false, ldb)) return cudaErrorInvalidValue;
-  if (!encode_tensor_map_2d(&thi, uhi, M, kRankPad, kTileRows, nt * 8, false)) return cudaErrorInvalidValue;
-  if (!encode_tensor_map_2d(&tlo, ulo, M, kRankPad, kTileRows, nt * 8, false)) return cudaErrorInvalidValue;
-  float* vpart = part;
-  float* dbpart = part + static_cast<int64_t>(grid.ncb) * M * (nt * 8);
-  cudaError_t e = launch_vdb_nt<2>(tg, tb, thi, tlo, M, N, grid, vpart, dbpart, status, stream);
-  if (e != cudaSuccess) return e;
+cudaError_t launch_vdb_finalize(const float* vpart, int ncb, const float* dbpart, int ntb, int64_t M, int64_t N,
+                                int r, float scale, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,
+                                cudaStream_t stream) {
   const int64_t total = M * (kRankPad / 2) + (dB != nullptr ? N * r : 0);
-  vdb_finalize_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
-      vpart, grid.ncb, dbpart, grid.ntb, M, N, r, nt * 8, scale, vs, vhi, vlo, dB);
+  vdb_finalize_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(vpart, ncb, dbpart, ntb, M, N,
+                                                                                       r, 16, scale, vs, vhi, vlo, dB);
   return cudaGetLastError();
 }
 
