@@ -8,11 +8,11 @@
 // is HBM-bound: it streams the codes once and never writes a dequantized
 // copy.  Up to three kernels:
 //
-//   xa_part_kernel   U partials, each CTA reduces X A^T over 1024 of K with
-//                    warp MMAs ([P][16][64] fp32); it releases the next
-//                    kernel at once (programmatic dependent launch).  Not
-//                    launched for 9..16 tokens and K <= 4096: the GEMV then
-//                    computes U itself from the X fragments it holds.
+//   xa_part_kernel   only when K > 4096: U partials, each CTA reduces
+//                    X A^T over 1024 of K with warp MMAs ([P][16][64] fp32);
+//                    it releases the GEMV at once (programmatic dependent
+//                    launch).  For K <= 4096 the GEMV computes U itself from
+//                    the X fragments it holds (one launch per call).
 //   gemv_kernel      persistent, one CTA per SM, which owns a contiguous
 //                    range of 16-row tiles.  Each of its 16 warps owns one
 //                    quarter-kilo slice of K (4 blocks of 64; X held in
@@ -445,18 +445,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
     // partials ([tile][token tile][lane][4]).
     __syncthreads();
     if (first_reduce) {
-      // U from the preceding kernel (programmatic launch): its partials must
-      // be complete before they are read here (K <= 4096) or before this
-      // grid ends (K > 4096: the finalize kernel reads them).  When this
-      // kernel computed U itself no kernel precedes by programmatic launch
-      // and the wait returns at once.
+      // K > 4096: the U partials of the preceding kernel (programmatic
+      // launch) must be complete before this grid ends (the finalize kernel
+      // reads them).  For K <= 4096 this kernel computed U itself, no kernel
+      // precedes by programmatic launch and the wait returns at once.
       pdl_wait_prior();
-      if (single && !kM16) {
-        // The B rows were this thread's oldest copy group, complete since its
-        // first item's wait; the barrier above published every thread's.
-        gather_u(p, s_u, tid, kGvThreads);
-        __syncthreads();
-      }
       first_reduce = false;
     }
     if (tid < np * NT * 128) {
@@ -543,7 +536,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
           load16(p.X, K, tok, (blkw + b) * kBlock + 16 * t, blkw + b < nbk && tok < p.M, xf[nt][b]);
         }
       x_chunk = cc.c;
-      if (kM16 && single) compute_u();
+      if (single) compute_u();
     }
     run_pass(np);
     i0 += np;
@@ -584,7 +577,7 @@ __global__ void __launch_bounds__(256) gemv_finalize_kernel(const __grid_constan
 int gemv_upart_count(int64_t K) { return static_cast<int>((K / kBlock + kXaWarps - 1) / kXaWarps); }
 int gemv_chunks(int64_t K) { return static_cast<int>((K / kBlock + kGvUnitBlocks - 1) / kGvUnitBlocks); }
 
-int gemv_launches(int64_t K, int M) { return gemv_chunks(K) > 1 ? 3 : (M > 8 ? 1 : 2); }
+int gemv_launches(int64_t K, int /*M*/) { return gemv_chunks(K) > 1 ? 3 : 1; }
 
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   int dev = 0, sms = 0;
@@ -604,11 +597,12 @@ cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream) {
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
 
-  // M > 8 and K <= 4096: the GEMV computes U itself (its first reduction
-  // comes after two tiles, too early to hide a separate kernel); otherwise U
-  // partials come from the first kernel, which releases the GEMV at once
-  // (programmatic launch) and finishes while the GEMV streams its tiles.
-  const bool fused_u = gemv_chunks(p.K) == 1 && p.M > 8;
+  // K <= 4096: the GEMV computes U itself from the X fragments it holds (a
+  // separate U kernel before it cost about 4 us per call when calls follow
+  // one another); otherwise U partials come from the first kernel, which
+  // releases the GEMV at once (programmatic launch) and finishes while the
+  // GEMV streams its tiles.
+  const bool fused_u = gemv_chunks(p.K) == 1;
   if (!fused_u) {
     xa_part_kernel<<<p.n_upart, kXaWarps * 32, kXaWarps * kGemvMaxM * kRankPad * 4, stream>>>(p.X, p.A, p.M, p.K,
                                                                                             p.r, p.upart);
