@@ -16,13 +16,18 @@
 // over j, so it runs on the tensor cores: each warp owns one 64-column
 // quantization-block stripe, keeps the stripe's A operand (r x 64, bf16) in
 // registers for every row tile it visits, and per 16-row tile issues
-// 8 * ceil(r / 16) m16n8k16 MMAs with fp32 accumulation.  The decode of the
-// codes (NF4 level by a lane shuffle, fp32 block scale) and
-// out = fma(s, BA, Qhat(W)) run in the accumulator layout; a per-warp shared
-// tile turns the two-column fragments into 16-byte row-contiguous stores.
-// Loads of the next tile (codes, scale codes, B rows) are issued before the
-// current tile's arithmetic.  Pairs of B columns are loaded as one word
-// where B allows it (4-byte aligned, even r).
+// 8 * ceil(r / 16) m16n8k16 MMAs with fp32 accumulation.  The columns are
+// dealt to the MMAs so that lane t of a quad ends up with the 16 contiguous
+// columns 16t .. 16t+15 of its rows: column slot 2t + e of 8-column group i
+// is weight column 16t + 2i + e.  A lane therefore loads exactly the 8 code
+// bytes it decodes (one 8-byte load per row) and stores its outputs straight
+// from registers, 32 bytes of a row per store (a whole sector per lane, whole
+// lines per warp), with no shared-memory staging.  The
+// decode (NF4 level by a lane shuffle, fp32 block scale) and
+// out = fma(s, BA, Qhat(W)) run in the accumulator layout.  Loads of the next
+// tile (codes, scale codes, B rows) are issued before the current tile's
+// arithmetic.  Pairs of B columns are loaded as one word where B allows it
+// (4-byte aligned, even r).
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -36,7 +41,7 @@ constexpr int kMergeThreads = 32 * kMergeWarps;
 // Inputs of one 16-row tile for one lane: rows g and g + 8 of the tile.
 template <int kSteps>
 struct MergeTileIn {
-  uint4 code[2][2];        // the row's 64 codes (32 bytes) in the stripe
+  uint2 code[2];           // codes of the row's columns 16t .. 16t+15 in the stripe (8 bytes)
   int q[2];                // scale codes
   float c2[2];             // second-level scales
   uint32_t bf[kSteps][4];  // MMA A operand: B rows of the tile, bf16 pairs
@@ -65,10 +70,9 @@ __device__ __forceinline__ void merge_load_tile(MergeTileIn<kSteps>& in, const W
     const int64_t n = n0 + g + 8 * h;
     const bool ok = n < N;
     const int64_t nn = ok ? n : 0;
-    const uint4* src = reinterpret_cast<const uint4*>(w.packed) + nn * (K / 32) + 2 * stripe;
+    const uint2* src = reinterpret_cast<const uint2*>(w.packed) + nn * (K / 16) + 4 * stripe + t;
     const int64_t blk = nn * kb + stripe;
-    in.code[h][0] = ok ? __ldg(src) : make_uint4(0, 0, 0, 0);
-    in.code[h][1] = ok ? __ldg(src + 1) : make_uint4(0, 0, 0, 0);
+    in.code[h] = ok ? __ldg(src) : make_uint2(0, 0);
     if (w.scale_format == kScalesFp32) {  // t = 1, c2 = the absmax (see scale_table_entry)
       in.q[h] = 127;
       in.c2[h] = ok ? __ldg(w.absmax + blk) : 0.0f;
@@ -98,12 +102,7 @@ __device__ __forceinline__ void mma_16816_zero(float (&d)[4], const uint32_t (&a
 template <int kSteps, bool kFp32, bool kPair32>
 __global__ void __launch_bounds__(kMergeThreads, kSteps == 1 ? 4 : (kSteps == 2 ? 3 : 2))
     merge_kernel(WeightView w, const uint16_t* __restrict__ A, const uint16_t* __restrict__ B, int r, float scale,
-                 void* __restrict__ out) {
-  // Output staging: 16 rows per warp, padded so that the fragment stores hit
-  // 32 distinct banks (bf16: 36-word pitch; fp32: 72-word pitch, 8-byte stores
-  // in half-warp phases).
-  constexpr int kPitch = kFp32 ? 288 : 144;
-  __shared__ __align__(16) uint8_t s_out[kMergeWarps][16 * kPitch];
+                 void* __restrict__ out, bool wide32) {
   __shared__ float s_qdiv[256];  // scale-code values t(q), q = -128 .. 127
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -117,7 +116,8 @@ __global__ void __launch_bounds__(kMergeThreads, kSteps == 1 ? 4 : (kSteps == 2 
   const float level = codebook_level(w.codebook, lane & 15);
   const float mu = weight_mu(w);
 
-  // MMA B operand: the stripe's A columns, fragment (k = j, n = column).
+  // MMA B operand: the stripe's A columns, fragment (k = j, n = column slot
+  // g of group i), slot g holding column 16 (g / 2) + 2i + g % 2.
   uint32_t af[kSteps][8][2];
 #pragma unroll
   for (int s = 0; s < kSteps; ++s)
@@ -126,27 +126,23 @@ __global__ void __launch_bounds__(kMergeThreads, kSteps == 1 ? 4 : (kSteps == 2 
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int j = 16 * s + 2 * t + 8 * h;
-        const uint16_t* col = A + c0 + 8 * i + g;
+        const uint16_t* col = A + c0 + 16 * (g >> 1) + 2 * i + (g & 1);
         const uint32_t lo = j < r ? col[static_cast<int64_t>(j) * K] : 0u;
         const uint32_t hi = j + 1 < r ? col[static_cast<int64_t>(j + 1) * K] : 0u;
         af[s][i][h] = lo | (hi << 16);
       }
 
-  uint8_t* stage = s_out[warp];
   const int64_t n_tiles = (N + 15) / 16;
 
-  // One 16-row tile: MMA per 8-column group, decode, fma, stage, store.
+  // One 16-row tile: per 8-column group i an MMA, then for rows g and g + 8
+  // the lane's columns 16t + 2i, 16t + 2i + 1 (byte i of its 8 code bytes,
+  // low nibble first): decode, fma, and every 16 bytes of output a store.
   auto process = [&](const MergeTileIn<kSteps>& in, int64_t n0) {
     float sc[2];
-    uint32_t words[2][8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      sc[h] = __fadd_rn(__fmul_rn(s_qdiv[in.q[h] + 128], in.c2[h]), mu);
-      words[h][0] = in.code[h][0].x, words[h][1] = in.code[h][0].y;
-      words[h][2] = in.code[h][0].z, words[h][3] = in.code[h][0].w;
-      words[h][4] = in.code[h][1].x, words[h][5] = in.code[h][1].y;
-      words[h][6] = in.code[h][1].z, words[h][7] = in.code[h][1].w;
-    }
+    for (int h = 0; h < 2; ++h) sc[h] = __fadd_rn(__fmul_rn(s_qdiv[in.q[h] + 128], in.c2[h]), mu);
+    constexpr int kGroupsPerStore = kFp32 ? 4 : 8;  // 32 bytes per store and row
+    uint32_t o[2][8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       float d[4];
@@ -155,38 +151,40 @@ __global__ void __launch_bounds__(kMergeThreads, kSteps == 1 ? 4 : (kSteps == 2 
       for (int s = 1; s < kSteps; ++s) mma_16816(d, in.bf[s], af[s][i]);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        // Columns 8i + 2t and 8i + 2t + 1 are byte t of word i (low nibble
-        // first).  The shuffle reads the source lane from the low five bits;
-        // lanes hold L[lane % 16], so the high bits need no mask.
-        const uint32_t x = words[h][i] >> (8 * t);
+        // The shuffle reads the source lane from the low five bits; lanes
+        // hold L[lane % 16], so the high bits need no mask.
+        const uint32_t x = (i < 4 ? in.code[h].x : in.code[h].y) >> (8 * (i & 3));
         const float l0 = __shfl_sync(0xffffffffu, level, static_cast<int>(x));
         const float l1 = __shfl_sync(0xffffffffu, level, static_cast<int>(x >> 4));
         const float m0 = fmaf(scale, d[2 * h], __fmul_rn(l0, sc[h]));
         const float m1 = fmaf(scale, d[2 * h + 1], __fmul_rn(l1, sc[h]));
-        const int row = g + 8 * h;
         if constexpr (kFp32) {
-          *reinterpret_cast<float2*>(stage + row * kPitch + 32 * i + 8 * t) = make_float2(m0, m1);
+          o[h][2 * (i & 3)] = __float_as_uint(m0);
+          o[h][2 * (i & 3) + 1] = __float_as_uint(m1);
         } else {
-          *reinterpret_cast<uint32_t*>(stage + row * kPitch + 16 * i + 4 * t) = pack_bf16x2(m0, m1);
+          o[h][i] = pack_bf16x2(m0, m1);
+        }
+      }
+      if (i % kGroupsPerStore == kGroupsPerStore - 1) {
+        // 32 bytes of the row: a full sector per lane and eight whole lines
+        // per warp (two 16-byte stores when the output is only 16-byte
+        // aligned).
+        const int piece = i / kGroupsPerStore;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t n = n0 + g + 8 * h;
+          if (n < N) {
+            uint8_t* dst = static_cast<uint8_t*>(out) + (n * K + c0 + 16 * t) * (kFp32 ? 4 : 2) + 32 * piece;
+            if (wide32) {
+              st_stream_v8(dst, o[h]);
+            } else {
+              *reinterpret_cast<uint4*>(dst) = make_uint4(o[h][0], o[h][1], o[h][2], o[h][3]);
+              *reinterpret_cast<uint4*>(dst + 16) = make_uint4(o[h][4], o[h][5], o[h][6], o[h][7]);
+            }
+          }
         }
       }
     }
-    __syncwarp();
-    constexpr int kChunksPerRow = kFp32 ? 16 : 8;  // 16-byte pieces of a 64-column row
-#pragma unroll
-    for (int k = 0; k < kChunksPerRow / 2; ++k) {
-      const int q = lane + 32 * k;
-      const int row = q / kChunksPerRow, ch = q % kChunksPerRow;
-      const uint4 v = *reinterpret_cast<const uint4*>(stage + row * kPitch + 16 * ch);
-      const int64_t n = n0 + row;
-      if (n < N) {
-        if constexpr (kFp32)
-          *reinterpret_cast<uint4*>(static_cast<float*>(out) + n * K + c0 + 4 * ch) = v;
-        else
-          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + n * K + c0 + 8 * ch) = v;
-      }
-    }
-    __syncwarp();
   };
 
   // 16-row tiles of this warp: blockIdx.y, +gridDim.y, ... (the CTAs of one
@@ -237,7 +235,8 @@ cudaError_t launch_merge_kernel(const WeightView& w, const uint16_t* A, const ui
   if (gy > 65535) gy = 65535;
   if (gy < 1) gy = 1;
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-  merge_kernel<kSteps, kFp32, kPair32><<<grid, kMergeThreads, 0, stream>>>(w, A, B, r, scale, out);
+  const bool wide32 = (reinterpret_cast<uintptr_t>(out) & 31) == 0;
+  merge_kernel<kSteps, kFp32, kPair32><<<grid, kMergeThreads, 0, stream>>>(w, A, B, r, scale, out, wide32);
   return cudaGetLastError();
 }
 
