@@ -5,7 +5,7 @@
 device at most), runs the library call ``reps`` times and exits; a profiler
 pointed at it with a kernel filter and a launch count captures the kernel of
 interest.  The cases use the 7B gate projection (14336 x 4096) at 8192
-tokens, the decode shape (16 tokens) for the GEMV, and the bf16 merged
+tokens, the decode shape (16 tokens, or ``--decode-tokens``) for the GEMV, and the bf16 merged
 weight (r = 16) for the merge.  ``--path dense`` runs the tensor-core calls on
 the dense-weight ablation path instead of the default fused one.
 """
@@ -30,12 +30,13 @@ def main():
     ap.add_argument("--case", choices=CASES, required=True)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--tokens", type=int, default=8192)
+    ap.add_argument("--decode-tokens", type=int, default=16, help="tokens of the gemv case (1..16)")
     ap.add_argument("--path", choices=("fused", "dense"), default="fused")
     args = ap.parse_args()
     torch.cuda.set_device(0)
     binding.qlora_linear_set_weight_path(
         binding.WEIGHT_PATH_DENSE if args.path == "dense" else binding.WEIGHT_PATH_FUSED)
-    M = 16 if args.case in ("gemv", "merge") else args.tokens
+    M = args.decode_tokens if args.case == "gemv" else (16 if args.case == "merge" else args.tokens)
     case = workloads.linear_case(workloads.GATE7B, M, 16, 32.0, 4, 0, 4, device="cuda", with_dy=args.case not in ("gemv", "merge"))
     out = binding.NF4Weight.empty(case.proj.n, case.proj.k)
     qws = torch.empty(binding.qlora_nf4_sizes(case.proj.n, case.proj.k)["ws_bytes"], dtype=torch.uint8, device="cuda")
