@@ -28,6 +28,7 @@ STATUS_NAMES = {
     5: "QLORA_ERR_CUDA",
     6: "QLORA_ERR_TIMEOUT",
     7: "QLORA_ERR_UNSUPPORTED",
+    8: "QLORA_ERR_CHECK",
 }
 
 EXPORTED = [
@@ -49,6 +50,7 @@ EXPORTED = [
     "qlora_linear_weight_path",
     "qlora_linear_fwd",
     "qlora_linear_fwd_stall_diagnostic",
+    "qlora_selftest_mbarrier_ring",
     "qlora_linear_bwd",
     "qlora_timing_enable",
     "qlora_timing_read",
@@ -119,6 +121,7 @@ def lib() -> ctypes.CDLL:
         "qlora_linear_weight_path": (i32, []),
         "qlora_linear_fwd": (i32, [W, P, i64, P, P, i32, f32, P, P, P, sz, P]),
         "qlora_linear_fwd_stall_diagnostic": (i32, [W, P, i64, P, P, i32, f32, P, P, sz, i32, P]),
+        "qlora_selftest_mbarrier_ring": (i32, [i32, i32, i32, i32, P, P]),
         "qlora_linear_bwd": (i32, [W, P, P, i64, P, P, i32, f32, P, P, i32, P, P, P, sz, P]),
         "qlora_timing_enable": (i32, [i32]),
         "qlora_timing_read": (i32, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]),
@@ -435,6 +438,16 @@ def qlora_linear_fwd_stall_diagnostic(w: NF4Weight, X, A, B, r: int, scale: floa
     _check("qlora_linear_fwd_stall_diagnostic",
            lib().qlora_linear_fwd_stall_diagnostic(ctypes.byref(st), xp, M, ap, bp, r, float(scale), yp, wsp, wsb,
                                                    int(wait_limit_us), _stream(stream)))
+
+
+def qlora_selftest_mbarrier_ring(stages: int, consumers: int, iters: int, wait_limit_us: int, result,
+                                 stream=None) -> None:
+    """Diagnostic: the barrier-ring self-test (see the header); `result` is a
+    device int32 tensor of 3 elements, overwritten."""
+    rp = _dev(result, "result", (torch.int32,), 3)
+    _check("qlora_selftest_mbarrier_ring",
+           lib().qlora_selftest_mbarrier_ring(int(stages), int(consumers), int(iters), int(wait_limit_us), rp,
+                                              _stream(stream)))
 
 
 def qlora_linear_bwd(w: NF4Weight, X, dY, A, B, r: int, scale: float, dX, accumulate: int, dA, dB, ws,

@@ -491,6 +491,7 @@ extern "C" const char* qlora_status_string(qlora_status status) {
     case QLORA_ERR_CUDA: return "CUDA error";
     case QLORA_ERR_TIMEOUT: return "device-side wait timed out";
     case QLORA_ERR_UNSUPPORTED: return "unsupported device or size";
+    case QLORA_ERR_CHECK: return "a debug-build index or alignment check failed";
   }
   return "unknown status";
 }
@@ -825,6 +826,18 @@ extern "C" qlora_status qlora_linear_fwd_stall_diagnostic(const qlora_nf4_weight
   if (M <= kGemvMaxM || wait_limit_us < 1 || wait_limit_us > 1000000) return QLORA_ERR_INVALID_ARG;
   return linear_fwd(w, X, M, A, B, r, scale, Y, nullptr, ws, ws_bytes, stream,
                     GemmDiagnostics{static_cast<uint64_t>(wait_limit_us) * 1000ull, 1});
+}
+
+extern "C" qlora_status qlora_selftest_mbarrier_ring(int32_t stages, int32_t consumers, int32_t iters,
+                                                     int32_t wait_limit_us, int32_t* d_result, void* stream) {
+  if (stages < 1 || stages > 8 || consumers < 0 || consumers > 4 || iters < 1 || iters > (1 << 24) ||
+      wait_limit_us < 1 || wait_limit_us > 1000000 || d_result == nullptr)
+    return QLORA_ERR_INVALID_ARG;
+  if (!aligned(d_result, 4)) return QLORA_ERR_ALIGNMENT;
+  const qlora_status st = check_device();
+  if (st != QLORA_OK) return st;
+  return from_cuda(launch_mbarrier_ring_selftest(stages, consumers, iters, static_cast<uint64_t>(wait_limit_us) * 1000ull,
+                                                 d_result, static_cast<cudaStream_t>(stream)));
 }
 
 extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,

@@ -52,6 +52,24 @@ __device__ __forceinline__ void raise_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// Debug-build checks.  A library built with -DQLORA_CHECKS
+// (libqlora_nf4_checks.so, `build(checks=True)`) tests index and alignment
+// conditions before the accesses they guard: a failed test records
+// QLORA_ERR_CHECK in the call's status word (when it has one) and the access
+// is skipped, with no trap; a skipped tensor copy then ends its consumer's
+// bounded wait.  In the default build every test is the constant true and
+// compiles away.
+#ifdef QLORA_CHECKS
+constexpr bool kChecks = true;
+#else
+constexpr bool kChecks = false;
+#endif
+
+__device__ __forceinline__ bool qlora_checked(int* status, bool ok) {
+  if (kChecks && !ok) raise_status(status, QLORA_ERR_CHECK);
+  return !kChecks || ok;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   // cvt.rn.bf16x2.f32 d, a, b packs a into the upper and b into the lower half.
   uint32_t r;
@@ -223,9 +241,13 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 }
 
 // 2-D tiled load global -> shared; completion is signalled on `bar` as bytes.
-// Coordinates are in elements: c0 along the contiguous dimension (must be a
-// multiple of 16 bytes / element size), c1 along rows.
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+// Coordinates are in elements of kElemBytes bytes: c0 along the contiguous
+// dimension (c0 * kElemBytes must be a multiple of 16; a checks build tests
+// it and skips a copy that breaks it), c1 along rows.
+template <int kElemBytes = 2>
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int* check_status = nullptr) {
+  if (!qlora_checked(check_status, (c0 * kElemBytes) % 16 == 0)) return;
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
           smem_u32(smem_dst)),
@@ -236,8 +258,10 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 // 2-D tiled load into this CTA's shared memory whose completion (transaction
 // bytes) is signalled on an mbarrier of either CTA of the pair, given by its
 // shared::cluster address.  No multicast.
+template <int kElemBytes = 2>
 __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster_addr,
-                                                 int c0, int c1) {
+                                                 int c0, int c1, int* check_status = nullptr) {
+  if (!qlora_checked(check_status, (c0 * kElemBytes) % 16 == 0)) return;
   asm volatile(
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
       "[%2];" ::"r"(smem_u32(smem_dst)),

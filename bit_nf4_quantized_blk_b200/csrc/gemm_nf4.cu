@@ -589,14 +589,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&cfull[c]);  // the rank step carries no codes
           } else if constexpr (!kBwd) {
             mbar_arrive_expect_tx(&cfull[c], kCodeBytes + BNH * 16);
-            tma_load_2d(slot, &tmP, &cfull[c], i * 32, n_half);                          // [128 rows][32 B]
-            tma_load_2d(slot + kCodeBytes, &tmS, &cfull[c], i & ~3, n_half);             // [128 rows][4 scales]
+            tma_load_2d<1>(slot, &tmP, &cfull[c], i * 32, n_half, status);                          // [128 rows][32 B]
+            tma_load_2d<4>(slot + kCodeBytes, &tmS, &cfull[c], i & ~3, n_half, status);             // [128 rows][4 scales]
           } else {
             const int n0 = i * BK, kb0 = n_half / kBlock;
             mbar_arrive_expect_tx(&cfull[c], kCodeBytes + BK * 16);
-            tma_load_2d(slot, &tmP, &cfull[c], n_half / 2, n0);                          // [64 rows][32 B]
-            tma_load_2d(slot + 2048, &tmP, &cfull[c], n_half / 2 + 32, n0);              // the next block
-            tma_load_2d(slot + kCodeBytes, &tmS, &cfull[c], kb0 & ~3, n0);               // [64 rows][4 scales]
+            tma_load_2d<1>(slot, &tmP, &cfull[c], n_half / 2, n0, status);                          // [64 rows][32 B]
+            tma_load_2d<1>(slot + 2048, &tmP, &cfull[c], n_half / 2 + 32, n0, status);              // the next block
+            tma_load_2d<4>(slot + kCodeBytes, &tmS, &cfull[c], kb0 & ~3, n0, status);               // [64 rows][4 scales]
           }
         }
       }

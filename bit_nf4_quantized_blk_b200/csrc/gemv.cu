@@ -267,7 +267,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
   auto issue_next = [&]() {
     const bool live = issued < items;
     const uint32_t dst = ring_lane + (issued & (kGvDepth - 1)) * kGvSliceBytes;
-    if (live && t0 + i_tile != ragged_tile && i_chunk < full_chunks) {
+    // A checks build also tests that the four unpredicated copies stay inside
+    // the packed weight (else it takes the predicated path).
+    if (live && t0 + i_tile != ragged_tile && i_chunk < full_chunks &&
+        qlora_checked(p.status, isrc >= p.packed && isrc + 3 * rows4_bytes + 16 <= p.packed + N * (K / 2))) {
 #pragma unroll
       for (int h = 0; h < 4; ++h) cp_async_16_full(dst + h * 4 * kGvSlicePitch, isrc + h * rows4_bytes);
     } else {

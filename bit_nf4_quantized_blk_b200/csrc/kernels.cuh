@@ -278,4 +278,13 @@ bool encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uin
 bool encode_tensor_map_2d_plain(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
                                 uint64_t ld, uint32_t box_rows, uint32_t box_cols);
 
+// ---------------------------------------------------------------------------
+// Barrier ring self-test (selftest.cu)
+// ---------------------------------------------------------------------------
+
+// result (device int[3]) is cleared, then receives the wrong / read counts and
+// the timeout status of the ring kernel.
+cudaError_t launch_mbarrier_ring_selftest(int stages, int consumers, int iters, uint64_t limit_ns, int* result,
+                                          cudaStream_t stream);
+
 }  // namespace qnf4

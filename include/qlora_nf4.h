@@ -68,7 +68,9 @@ typedef enum qlora_status {
   QLORA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required   */
   QLORA_ERR_CUDA = 5,         /* a CUDA runtime/launch error                  */
   QLORA_ERR_TIMEOUT = 6,      /* a device-side wait ran past its time limit   */
-  QLORA_ERR_UNSUPPORTED = 7   /* no sm_100 device, or a size beyond limits    */
+  QLORA_ERR_UNSUPPORTED = 7,  /* no sm_100 device, or a size beyond limits    */
+  QLORA_ERR_CHECK = 8         /* a debug-build (QLORA_CHECKS) index or
+                                 alignment test failed; the access was skipped */
 } qlora_status;
 
 /*
@@ -347,6 +349,27 @@ qlora_status qlora_linear_fwd_stall_diagnostic(const qlora_nf4_weight *w, const 
                                                const uint16_t *A, const uint16_t *B, int32_t r, float scale,
                                                uint16_t *Y, void *ws, size_t ws_bytes, int32_t wait_limit_us,
                                                void *stream);
+
+/*
+ * Self-test of the shared-memory barrier ring that the pipelined kernels use
+ * (the pages have no counterpart: it checks this library's synchronisation,
+ * not a step of the method).  One CTA: a producer thread writes the values
+ * 1 .. iters into a ring of `stages` shared slots; one thread in each of
+ * `consumers` warps reads every value in order.  A slot is published by an
+ * mbarrier of one arrival and handed back by one of `consumers` arrivals.
+ * Every wait takes the phase parity of its pass over the ring, as the GEMM
+ * and side-product rings do, and gives up after wait_limit_us.
+ *   stages     : 1 .. 8.   consumers : 0 .. 4 (0: nothing hands a slot back,
+ *                so the producer's wait on its second pass runs out).
+ *   iters      : 1 .. 2^24.   wait_limit_us : 1 .. 1,000,000.
+ *   d_result   : device int32[3], 4-byte aligned, overwritten: [0] values a
+ *                consumer read wrong, [1] values read (iters * consumers when
+ *                every wait succeeded), [2] QLORA_ERR_TIMEOUT if a wait ran
+ *                out, else 0.
+ * Returns QLORA_OK once enqueued (INVALID_ARG for an argument out of range).
+ */
+qlora_status qlora_selftest_mbarrier_ring(int32_t stages, int32_t consumers, int32_t iters, int32_t wait_limit_us,
+                                          int32_t *d_result, void *stream);
 
 /*
  * LoRA linear backward for upstream gradient dY of Y.

@@ -49,10 +49,34 @@ def test_every_declared_symbol_is_exported(lib):
     assert sorted(names) == sorted(binding.EXPORTED)
 
 
+def test_checks_library_exports_the_same_symbols():
+    """The debug library (QLORA_CHECKS: index and alignment tests compiled in)
+    is built beside the default one and has the same C ABI."""
+    from bit_nf4_quantized_blk_b200 import build
+
+    path = build.build(checks=True)
+    assert path.endswith("libqlora_nf4_checks.so") and os.path.exists(path)
+    L = ctypes.CDLL(path)
+    for n in _declared_functions():
+        assert hasattr(L, n), n
+
+
 def test_status_strings(lib):
     assert binding.qlora_status_string(0) == "ok"
     assert "workspace" in binding.qlora_status_string(4)
+    assert "check" in binding.qlora_status_string(8)
+    assert binding.STATUS_NAMES[8] == "QLORA_ERR_CHECK"
     assert binding.qlora_status_string(99) == "unknown status"
+
+
+def test_ring_selftest_arguments_checked_on_the_host(lib):
+    """Out-of-range self-test arguments are refused before any launch."""
+    f = lib.qlora_selftest_mbarrier_ring
+    buf = ctypes.c_void_p(256)  # never dereferenced: every call below is refused first
+    for args in ((0, 1, 16, 1000), (9, 1, 16, 1000), (2, 5, 16, 1000), (2, -1, 16, 1000), (2, 1, 0, 1000),
+                 (2, 1, (1 << 24) + 1, 1000), (2, 1, 16, 0), (2, 1, 16, 1000001)):
+        assert f(*args, buf, None) == 1, args
+    assert f(2, 1, 16, 1000, None, None) == 1
 
 
 def test_sizes(lib):
