@@ -738,12 +738,12 @@ def run_reference(args, rank, world):
     }))
 
 
-GEMM_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "gemm_tn_layer_step_traffic.md")
+GEMM_TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "gemm_nf4_layer_step_traffic.md")
 GEMM_SOURCES = ("csrc/gemm_nf4.cu", "csrc/gemm_common.cuh", "csrc/common.cuh")  # the GEMM and its device helpers
 
 
 def gemm_traffic_per_launch():
-    """DRAM bytes per gemm_tn launch from the committed ncu summary, or None
+    """DRAM bytes per gemm_nf4 launch from the committed ncu summary, or None
     when the kernel's sources changed since that capture."""
     import hashlib
     try:
