@@ -886,10 +886,14 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
   };
   if (dB != nullptr && r <= kVdbMaxRank && M > kGemvMaxM) {
     // V = dY B (s*V for the dX rank step, hi/lo for dA) and dB = s dY^T U in one pass over dY.
-    e = u_hilo();
-    if (e != cudaSuccess) return from_cuda(e);
+    // A saved fp32 U goes straight to the rank transposes, which split it
+    // themselves; otherwise U is recomputed as its hi/lo split first.
+    if (U == nullptr) {
+      e = u_hilo();
+      if (e != cudaSuccess) return from_cuda(e);
+    }
     Timed tm(kFamSide, s, 3);  // the rank transposes, the pass, the reduction
-    e = launch_vdb_tc(dY, M, N, Bk, ldbk, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), r, scale,
+    e = launch_vdb_tc(dY, M, N, Bk, ldbk, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), U, r, scale,
                       at<float>(ws, lay.vdbpart), at<uint16_t>(ws, lay.bt), at<uint16_t>(ws, lay.uht),
                       at<uint16_t>(ws, lay.ult), at<uint16_t>(ws, lay.vs), at<uint16_t>(ws, lay.vhi),
                       at<uint16_t>(ws, lay.vlo), dB, status, s);

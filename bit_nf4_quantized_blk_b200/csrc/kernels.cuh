@@ -181,8 +181,10 @@ cudaError_t launch_colsum(const uint16_t* In, int64_t M, int64_t C, const uint16
 constexpr int kVdbMaxRank = 16;
 // The pass writes partials [ncb][M][16] and [ntb][N][16] fp32 (`part`, vdb_tc_partial_bytes
 // bytes); bt [16][N], uht and ult [16][vdb_tc_ldm(M)] are bf16 scratch for
-// B^T and the transposed U split (uhi / ulo [M][64] as written by
-// launch_split_hilo or launch_skinny).
+// B^T and the transposed U split.  U comes either as the hi / lo split
+// (uhi / ulo [M][64], as launch_skinny writes it; u32 null) or as the saved
+// fp32 U [M][r] (u32; uhi / ulo unused), which the transposes split
+// themselves.
 struct VdbTcGrid {
   int ct, tt, ncb, ntb;  // column / token tiles per CTA; column / token blocks
 };
@@ -190,9 +192,9 @@ VdbTcGrid vdb_tc_grid(int64_t M, int64_t N);
 size_t vdb_tc_partial_bytes(int64_t M, int64_t N);
 inline int64_t vdb_tc_ldm(int64_t M) { return (M + 7) / 8 * 8; }  // 16-byte rows for TMA
 cudaError_t launch_vdb_tc(const uint16_t* G, int64_t M, int64_t N, const uint16_t* B, int64_t ldb,
-                          const uint16_t* uhi, const uint16_t* ulo, int r, float scale, float* part, uint16_t* bt,
-                          uint16_t* uht, uint16_t* ult, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,
-                          int* status, cudaStream_t stream);
+                          const uint16_t* uhi, const uint16_t* ulo, const float* u32, int r, float scale, float* part,
+                          uint16_t* bt, uint16_t* uht, uint16_t* ult, uint16_t* vs, uint16_t* vhi, uint16_t* vlo,
+                          float* dB, int* status, cudaStream_t stream);
 // The fixed-order reduction of vdb partials [ncb][M][16] and [ntb][N][16].
 cudaError_t launch_vdb_finalize(const float* vpart, int ncb, const float* dbpart, int ntb, int64_t M, int64_t N,
                                 int r, float scale, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,

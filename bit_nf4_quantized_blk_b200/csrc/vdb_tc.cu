@@ -242,14 +242,27 @@ __global__ void __launch_bounds__(kVtThreads, kVtPerSm)
 // threads take consecutive rows of one j, so the stores are contiguous.
 __global__ void rank16_transpose3_kernel(const uint16_t* __restrict__ B, int64_t ldb, int64_t N,
                                          const uint16_t* __restrict__ uhi, const uint16_t* __restrict__ ulo,
-                                         int64_t M, int64_t ldm, int r, uint16_t* __restrict__ bt,
-                                         uint16_t* __restrict__ uht, uint16_t* __restrict__ ult) {
+                                         const float* __restrict__ u32, int64_t M, int64_t ldm, int r,
+                                         uint16_t* __restrict__ bt, uint16_t* __restrict__ uht,
+                                         uint16_t* __restrict__ ult) {
   int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const uint16_t* src;
   uint16_t* dst;
   int64_t ld, rows, ldd;
   if (i < 16 * N) {
     src = B, dst = bt, ld = ldb, rows = N, ldd = N;
+  } else if (u32 != nullptr) {
+    // The saved fp32 U [M][r]: each thread forms both halves of one element,
+    // hi = bf16(u) and lo = bf16(u - hi).
+    i -= 16 * N;
+    if (i >= 16 * M) return;
+    const int j = static_cast<int>(i / M);
+    const int64_t row = i % M;
+    const float v = j < r ? u32[row * r + j] : 0.0f;
+    const uint32_t h = pack_bf16x2(v, 0.0f) & 0xFFFFu;
+    uht[j * ldm + row] = static_cast<uint16_t>(h);
+    ult[j * ldm + row] = static_cast<uint16_t>(pack_bf16x2(v - bf16_bits_to_float(h), 0.0f) & 0xFFFFu);
+    return;
   } else {
     i -= 16 * N;
     if (i >= 32 * M) return;
@@ -290,7 +303,8 @@ size_t vdb_tc_partial_bytes(int64_t M, int64_t N) {
 }
 
 cudaError_t launch_vdb_tc(const uint16_t* G, int64_t M, int64_t N, const uint16_t* B, int64_t ldb,
-                          const uint16_t* uhi, const uint16_t* ulo, int r, float scale, float* part, uint16_t* bt,
+                          const uint16_t* uhi, const uint16_t* ulo, const float* u32, int r, float scale, float* part,
+                          uint16_t* bt,
                           uint16_t* uht, uint16_t* ult, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,
                           int* status, cudaStream_t stream) {
   if (r < 1 || r > 16) return cudaErrorInvalidValue;
@@ -305,9 +319,9 @@ cudaError_t launch_vdb_tc(const uint16_t* G, int64_t M, int64_t N, const uint16_
   // B^T [16][N] and the hi / lo split of U^T [16][ldm]: the MMAs' K-major
   // B operands.
   const int64_t ldm = vdb_tc_ldm(M);
-  const int64_t items = 16 * N + 32 * M;
-  rank16_transpose3_kernel<<<static_cast<unsigned>((items + 255) / 256), 256, 0, stream>>>(B, ldb, N, uhi, ulo, M, ldm,
-                                                                                          r, bt, uht, ult);
+  const int64_t items = 16 * N + (u32 != nullptr ? 16 : 32) * M;
+  rank16_transpose3_kernel<<<static_cast<unsigned>((items + 255) / 256), 256, 0, stream>>>(B, ldb, N, uhi, ulo, u32, M,
+                                                                                          ldm, r, bt, uht, ult);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tg, tbt, tuh, tul;
