@@ -449,12 +449,17 @@ qlora_status check_linear_args(const qlora_nf4_weight* w, int64_t M, int32_t r, 
 // The 4-bit weight decoded inside the tensor-core GEMM.
 // The 4-bit weight decoded inside the tensor-core GEMM; its decoded block
 // scales (`scales`, workspace) are written first by a small pre-pass.
+// `scales_written`: the caller's preceding reduction kernel already wrote the
+// block scales (a BlockScalesJob on its spare threads); otherwise a pre-pass
+// launch writes them here.
 cudaError_t launch_linear_gemm_nf4(const qlora_nf4_weight* w, float* scales, const uint16_t* A, int64_t M,
                                    const uint16_t* A2, const uint16_t* B2, int r, int64_t ldb2, uint16_t* D,
-                                   int accumulate, int* status, bool backward, cudaStream_t s,
+                                   int accumulate, int* status, bool backward, cudaStream_t s, bool scales_written,
                                    uint64_t wait_limit_ns = 0, int debug_stall = 0) {
-  cudaError_t e = launch_block_scales(view_of(w), scales, s);
-  if (e != cudaSuccess) return e;
+  if (!scales_written) {
+    const cudaError_t e = launch_block_scales(view_of(w), scales, s);
+    if (e != cudaSuccess) return e;
+  }
   Nf4GemmArgs g{};
   g.w = view_of(w);
   g.scales = scales;
@@ -778,6 +783,8 @@ qlora_status linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
   so.o32_ld = r;
   so.os = at<uint16_t>(ws, lay.us);
   so.scale = scale;
+  // The fused GEMM's block scales ride in the U reduction's launch.
+  if (!dense) so.bs = block_scales_job(view_of(w), at<float>(ws, lay.scales));
   // The caller's B [N, r] feeds the rank step directly when its rows are
   // 16-byte multiples; otherwise a zero-padded copy [N, 64] does.
   const bool b_direct = (r % 8) == 0 && aligned(B, 16);
@@ -790,9 +797,10 @@ qlora_status linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
   const uint16_t* B2 = b_direct ? B : at<uint16_t>(ws, lay.bpad);
   const int64_t ldb2 = b_direct ? r : kRankPad;
   if (!dense) {
-    Timed tm(kFamGemm, s, 2);  // block-scale pre-pass + GEMM
+    Timed tm(kFamGemm, s, 1);  // the block scales came with the U reduction
     return gemm_status(launch_linear_gemm_nf4(w, at<float>(ws, lay.scales), X, M, at<uint16_t>(ws, lay.us), B2, r,
-                                              ldb2, Y, 0, status, false, s, diag.wait_limit_ns, diag.debug_stall));
+                                              ldb2, Y, 0, status, false, s, true, diag.wait_limit_ns,
+                                              diag.debug_stall));
   }
   GemmArgs g{};
   g.A = X;
@@ -884,6 +892,7 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
     Timed tm(kFamSide, s, 2);
     return launch_skinny(X, M, K, A, true, r, 0, at<float>(ws, lay.skpart), uo, status, s);
   };
+  BlockScalesJob bs{};  // the dX GEMM's block scales, when a kernel before it carries them
   if (dB != nullptr && r <= kVdbMaxRank && M > kGemvMaxM) {
     // V = dY B (s*V for the dX rank step, hi/lo for dA) and dB = s dY^T U in one pass over dY.
     // A saved fp32 U goes straight to the rank transposes, which split it
@@ -892,11 +901,13 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
       e = u_hilo();
       if (e != cudaSuccess) return from_cuda(e);
     }
+    // The dX GEMM's block scales ride in the pass's reduction launch.
+    if (dX != nullptr && !dense) bs = block_scales_job(view_of(w), at<float>(ws, lay.scales));
     Timed tm(kFamSide, s, 3);  // the rank transposes, the pass, the reduction
     e = launch_vdb_tc(dY, M, N, Bk, ldbk, at<uint16_t>(ws, lay.uhi), at<uint16_t>(ws, lay.ulo), U, r, scale,
                       at<float>(ws, lay.vdbpart), at<uint16_t>(ws, lay.bt), at<uint16_t>(ws, lay.uht),
                       at<uint16_t>(ws, lay.ult), at<uint16_t>(ws, lay.vs), at<uint16_t>(ws, lay.vhi),
-                      at<uint16_t>(ws, lay.vlo), dB, status, s);
+                      at<uint16_t>(ws, lay.vlo), dB, bs, status, s);
     if (e != cudaSuccess) return from_cuda(e);
   } else {
     // V = dY B (bf16 s*V for the dX rank step; hi/lo split for dA).
@@ -920,9 +931,10 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16
     }
   }
   if (dX != nullptr && !dense) {  // dX = dY W_hat + s V A, W_hat decoded in the GEMM, A [r, K] MN-major
-    Timed tm(kFamGemm, s, 2);  // block-scale pre-pass + GEMM
+    const bool scales_written = bs.out != nullptr;
+    Timed tm(kFamGemm, s, scales_written ? 1 : 2);  // (block-scale pre-pass +) GEMM
     e = launch_linear_gemm_nf4(w, at<float>(ws, lay.scales), dY, M, at<uint16_t>(ws, lay.vs), A, r, 0, dX, accumulate,
-                               status, true, s);
+                               status, true, s, scales_written);
     if (e != cudaSuccess) return gemm_status(e);
   }
   if (dX != nullptr && dense) {  // dense-weight path: W_hat [N, K] and A [r, K] read as MN-major operands

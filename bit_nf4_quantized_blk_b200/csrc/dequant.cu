@@ -180,26 +180,29 @@ __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, u
 // Decoded block scales of a weight as an fp32 [rows][ld] array (ld >= cols /
 // 64; the pad columns are 0), read by the 4-bit GEMM's tile producer: the same
 // a = fp32(fp32(t * c2) + mu), or the stored fp32 absmax, that every decoder
-// of this library applies.  Four blocks per thread (one 16-byte store).
-__global__ void __launch_bounds__(256) block_scales_kernel(WeightView w, float* __restrict__ out, int64_t ld) {
+// of this library applies.  Four blocks per thread (one 16-byte store;
+// block_scales_group).  The linear calls usually run this job on spare
+// threads of the U or V reduction that precedes the GEMM; this kernel runs
+// it alone.
+__global__ void __launch_bounds__(256) block_scales_kernel(BlockScalesJob j) {
   const int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // 4-column group
-  const int64_t groups = ld / 4;
-  if (q >= w.rows * groups) return;
-  const int64_t n = q / groups, kb0 = (q - n * groups) * 4;
-  const int64_t kblocks = w.cols / kBlock;
-  const float mu = weight_mu(w);
-  float v[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) v[j] = kb0 + j < kblocks ? weight_block_scale(w, n * kblocks + kb0 + j, mu) : 0.0f;
-  *reinterpret_cast<float4*>(out + n * ld + kb0) = make_float4(v[0], v[1], v[2], v[3]);
+  if (q < j.groups) block_scales_group(j, q);
 }
 
 int64_t block_scales_ld(int64_t cols) { return (cols / kBlock + 3) / 4 * 4; }
 
+BlockScalesJob block_scales_job(const WeightView& w, float* out) {
+  BlockScalesJob j;
+  j.w = w;
+  j.out = out;
+  j.ld = block_scales_ld(w.cols);
+  j.groups = w.rows * (j.ld / 4);
+  return j;
+}
+
 cudaError_t launch_block_scales(const WeightView& w, float* out, cudaStream_t stream) {
-  const int64_t ld = block_scales_ld(w.cols);
-  const int64_t threads = w.rows * (ld / 4);
-  block_scales_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(w, out, ld);
+  const BlockScalesJob j = block_scales_job(w, out);
+  block_scales_kernel<<<static_cast<unsigned>((j.groups + 255) / 256), 256, 0, stream>>>(j);
   return cudaGetLastError();
 }
 

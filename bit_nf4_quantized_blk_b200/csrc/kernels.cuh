@@ -64,6 +64,28 @@ __device__ __forceinline__ float weight_mu(const WeightView& w) {
   return w.scale_format == kScalesFp32 ? 0.0f : *w.mu;
 }
 
+// The 4-bit GEMM's decoded block scales, fp32 [rows][ld] (pad columns 0),
+// as a job of `groups` four-block groups that runs on spare threads of
+// another small kernel's launch (or alone, launch_block_scales).  out null:
+// no job.
+struct BlockScalesJob {
+  WeightView w;
+  float* out;
+  int64_t ld, groups;
+};
+
+// Group q: blocks 4 (q % (ld / 4)) .. + 3 of row q / (ld / 4), one 16-byte store.
+__device__ __forceinline__ void block_scales_group(const BlockScalesJob& j, int64_t q) {
+  const int64_t per_row = j.ld / 4;
+  const int64_t n = q / per_row, kb0 = (q - n * per_row) * 4;
+  const int64_t kblocks = j.w.cols / kBlock;
+  const float mu = weight_mu(j.w);
+  float v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = kb0 + i < kblocks ? weight_block_scale(j.w, n * kblocks + kb0 + i, mu) : 0.0f;
+  *reinterpret_cast<float4*>(j.out + n * j.ld + kb0) = make_float4(v[0], v[1], v[2], v[3]);
+}
+
 // Entry i of a 256-entry table of scale-code values t(q), q = i - 128 the
 // int8 view of the stored code: fp32(q / 127) for int8 codes, the E4M3 value
 // for FP8 codes.  With fp32 scales the table is the int8 one and the kernels
@@ -95,6 +117,7 @@ struct DequantBatchParams {
 cudaError_t launch_dequant_batch(const DequantBatchParams& p, int out_fp32, cudaStream_t stream);
 // Decoded fp32 block scales [rows][block_scales_ld(cols)] (16-byte aligned output).
 int64_t block_scales_ld(int64_t cols);
+BlockScalesJob block_scales_job(const WeightView& w, float* out);
 cudaError_t launch_block_scales(const WeightView& w, float* out, cudaStream_t stream);
 cudaError_t launch_dequant_transposed(const WeightView& w, uint16_t* out, cudaStream_t stream);
 
@@ -157,6 +180,7 @@ struct SkinnyOut {
   uint16_t* ohi;
   uint16_t* olo;
   float scale;
+  BlockScalesJob bs;  // run on further threads of the reduction's launch (out null: none)
 };
 int skinny_splits(int64_t M, int64_t C);
 size_t skinny_partial_bytes(int64_t M, int64_t C);
@@ -191,14 +215,16 @@ struct VdbTcGrid {
 VdbTcGrid vdb_tc_grid(int64_t M, int64_t N);
 size_t vdb_tc_partial_bytes(int64_t M, int64_t N);
 inline int64_t vdb_tc_ldm(int64_t M) { return (M + 7) / 8 * 8; }  // 16-byte rows for TMA
+// `bs`: a block-scales job run in the reduction's launch (out null: none).
 cudaError_t launch_vdb_tc(const uint16_t* G, int64_t M, int64_t N, const uint16_t* B, int64_t ldb,
                           const uint16_t* uhi, const uint16_t* ulo, const float* u32, int r, float scale, float* part,
                           uint16_t* bt, uint16_t* uht, uint16_t* ult, uint16_t* vs, uint16_t* vhi, uint16_t* vlo,
-                          float* dB, int* status, cudaStream_t stream);
-// The fixed-order reduction of vdb partials [ncb][M][16] and [ntb][N][16].
+                          float* dB, const BlockScalesJob& bs, int* status, cudaStream_t stream);
+// The fixed-order reduction of vdb partials [ncb][M][16] and [ntb][N][16],
+// plus the block-scales job `bs` on further threads.
 cudaError_t launch_vdb_finalize(const float* vpart, int ncb, const float* dbpart, int ntb, int64_t M, int64_t N,
                                 int r, float scale, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,
-                                cudaStream_t stream);
+                                const BlockScalesJob& bs, cudaStream_t stream);
 
 // Copy a bf16 [rows][r] matrix into [rows][64] zero padded, optionally from
 // the transposed source [r][rows].

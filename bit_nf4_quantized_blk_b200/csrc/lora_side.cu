@@ -179,9 +179,14 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const __grid_constant_
 }
 
 // out(m, j) = sum_z part[z][m][j] (fixed order); j >= r gives 0.
+// Threads past the M * 32 pairs run out.bs (the GEMM's block scales) when set.
 __global__ void skinny_finalize_kernel(const float* __restrict__ part, int64_t M, int r, int splits, SkinnyOut out) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // over M * 32 pairs
-  if (i >= M * (kRankPad / 2)) return;
+  if (i >= M * (kRankPad / 2)) {
+    const int64_t q = i - M * (kRankPad / 2);
+    if (out.bs.out != nullptr && q < out.bs.groups) block_scales_group(out.bs, q);
+    return;
+  }
   const int64_t m = i / (kRankPad / 2);
   const int j = static_cast<int>(i % (kRankPad / 2)) * 2;
   float v0 = 0.0f, v1 = 0.0f;
@@ -278,7 +283,7 @@ cudaError_t launch_skinny(const uint16_t* In, int64_t M, int64_t C, const uint16
                   : launch_skinny_nt<false, 8>(tin, tw, M, C, splits, part, status, stream);
   }
   if (e != cudaSuccess) return e;
-  const int64_t total = M * (kRankPad / 2);
+  const int64_t total = M * (kRankPad / 2) + (out.bs.out != nullptr ? out.bs.groups : 0);
   skinny_finalize_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(part, M, r, splits, out);
   return cudaGetLastError();
 }
@@ -473,7 +478,7 @@ cudaError_t launch_colsum(const uint16_t* In, int64_t M, int64_t C, const uint16
 __global__ void vdb_finalize_kernel(const float* __restrict__ vpart, int ncb, const float* __restrict__ dbpart,
                                     int ntb, int64_t M, int64_t N, int r, int r16, float scale,
                                     uint16_t* __restrict__ vs, uint16_t* __restrict__ vhi, uint16_t* __restrict__ vlo,
-                                    float* __restrict__ dB) {
+                                    float* __restrict__ dB, BlockScalesJob bs) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nv = M * (kRankPad / 2);
   if (i < nv) {
@@ -496,7 +501,11 @@ __global__ void vdb_finalize_kernel(const float* __restrict__ vpart, int ncb, co
     return;
   }
   const int64_t k = i - nv;
-  if (dB == nullptr || k >= N * r) return;
+  const int64_t ndb = dB != nullptr ? N * r : 0;
+  if (k >= ndb) {  // the GEMM's block scales, when set
+    if (bs.out != nullptr && k - ndb < bs.groups) block_scales_group(bs, k - ndb);
+    return;
+  }
   const int64_t c = k / r;
   const int j = static_cast<int>(k % r);
   float s = 0.0f;
@@ -506,10 +515,12 @@ __global__ void vdb_finalize_kernel(const float* __restrict__ vpart, int ncb, co
 
 cudaError_t launch_vdb_finalize(const float* vpart, int ncb, const float* dbpart, int ntb, int64_t M, int64_t N,
                                 int r, float scale, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,
-                                cudaStream_t stream) {
-  const int64_t total = M * (kRankPad / 2) + (dB != nullptr ? N * r : 0);
+                                const BlockScalesJob& bs, cudaStream_t stream) {
+  const int64_t total =
+      M * (kRankPad / 2) + (dB != nullptr ? N * r : 0) + (bs.out != nullptr ? bs.groups : 0);
   vdb_finalize_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(vpart, ncb, dbpart, ntb, M, N,
-                                                                                       r, 16, scale, vs, vhi, vlo, dB);
+                                                                                       r, 16, scale, vs, vhi, vlo, dB,
+                                                                                       bs);
   return cudaGetLastError();
 }
 

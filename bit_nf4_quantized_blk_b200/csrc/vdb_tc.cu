@@ -304,9 +304,8 @@ size_t vdb_tc_partial_bytes(int64_t M, int64_t N) {
 
 cudaError_t launch_vdb_tc(const uint16_t* G, int64_t M, int64_t N, const uint16_t* B, int64_t ldb,
                           const uint16_t* uhi, const uint16_t* ulo, const float* u32, int r, float scale, float* part,
-                          uint16_t* bt,
-                          uint16_t* uht, uint16_t* ult, uint16_t* vs, uint16_t* vhi, uint16_t* vlo, float* dB,
-                          int* status, cudaStream_t stream) {
+                          uint16_t* bt, uint16_t* uht, uint16_t* ult, uint16_t* vs, uint16_t* vhi, uint16_t* vlo,
+                          float* dB, const BlockScalesJob& bs, int* status, cudaStream_t stream) {
   if (r < 1 || r > 16) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -336,7 +335,7 @@ cudaError_t launch_vdb_tc(const uint16_t* G, int64_t M, int64_t N, const uint16_
       tg, tbt, tuh, tul, M, N, g.ct, g.tt, vpart, dbpart, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_vdb_finalize(vpart, g.ncb, dbpart, g.ntb, M, N, r, scale, vs, vhi, vlo, dB, stream);
+  return launch_vdb_finalize(vpart, g.ncb, dbpart, g.ntb, M, N, r, scale, vs, vhi, vlo, dB, bs, stream);
 }
 
 }  // namespace qnf4
