@@ -579,7 +579,8 @@ extern "C" qlora_status qlora_nf4_quantize_batched_ex(const void* const* W, int3
     e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * kMaxQuantBatch, s);
     if (e != cudaSuccess) return from_cuda(e);
     {
-      Timed tm(kFamQuant, s, 2);
+      // The codes kernel, then (double-quantized formats) the chunk sums and the DQ codes.
+      Timed tm(kFamQuant, s, p.scale_format == kScalesFp32 ? 1 : 3);
       e = launch_quantize_batch(p, s);
     }
     if (e != cudaSuccess) return from_cuda(e);
