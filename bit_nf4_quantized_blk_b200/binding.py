@@ -51,6 +51,7 @@ EXPORTED = [
     "qlora_linear_fwd",
     "qlora_linear_fwd_stall_diagnostic",
     "qlora_selftest_mbarrier_ring",
+    "qlora_selftest_checks",
     "qlora_linear_bwd",
     "qlora_timing_enable",
     "qlora_timing_read",
@@ -122,6 +123,7 @@ def lib() -> ctypes.CDLL:
         "qlora_linear_fwd": (i32, [W, P, i64, P, P, i32, f32, P, P, P, sz, P]),
         "qlora_linear_fwd_stall_diagnostic": (i32, [W, P, i64, P, P, i32, f32, P, P, sz, i32, P]),
         "qlora_selftest_mbarrier_ring": (i32, [i32, i32, i32, i32, P, P]),
+        "qlora_selftest_checks": (i32, [P, P]),
         "qlora_linear_bwd": (i32, [W, P, P, i64, P, P, i32, f32, P, P, i32, P, P, P, sz, P]),
         "qlora_timing_enable": (i32, [i32]),
         "qlora_timing_read": (i32, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]),
@@ -448,6 +450,13 @@ def qlora_selftest_mbarrier_ring(stages: int, consumers: int, iters: int, wait_l
     _check("qlora_selftest_mbarrier_ring",
            lib().qlora_selftest_mbarrier_ring(int(stages), int(consumers), int(iters), int(wait_limit_us), rp,
                                               _stream(stream)))
+
+
+def qlora_selftest_checks(result, stream=None) -> None:
+    """Diagnostic: `result` (device int32, 1 element) becomes QLORA_ERR_CHECK
+    (8) when the loaded library was built with the debug checks, else 0."""
+    rp = _dev(result, "result", (torch.int32,), 1)
+    _check("qlora_selftest_checks", lib().qlora_selftest_checks(rp, _stream(stream)))
 
 
 def qlora_linear_bwd(w: NF4Weight, X, dY, A, B, r: int, scale: float, dX, accumulate: int, dA, dB, ws,

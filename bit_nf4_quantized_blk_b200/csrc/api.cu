@@ -849,6 +849,14 @@ extern "C" qlora_status qlora_selftest_mbarrier_ring(int32_t stages, int32_t con
                                                  d_result, static_cast<cudaStream_t>(stream)));
 }
 
+extern "C" qlora_status qlora_selftest_checks(int32_t* d_result, void* stream) {
+  if (d_result == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(d_result, 4)) return QLORA_ERR_ALIGNMENT;
+  const qlora_status st = check_device();
+  if (st != QLORA_OK) return st;
+  return from_cuda(launch_checks_selftest(d_result, static_cast<cudaStream_t>(stream)));
+}
+
 extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,
                                          const uint16_t* A, const uint16_t* B, int32_t r, float scale, const float* U,
                                          uint16_t* dX, int32_t accumulate, float* dA, float* dB, void* ws,

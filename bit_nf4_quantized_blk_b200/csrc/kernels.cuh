@@ -314,5 +314,7 @@ bool encode_tensor_map_2d_plain(CUtensorMap* map, const void* base, int elem_byt
 // the timeout status of the ring kernel.
 cudaError_t launch_mbarrier_ring_selftest(int stages, int consumers, int iters, uint64_t limit_ns, int* result,
                                           cudaStream_t stream);
+// *result = QLORA_ERR_CHECK when the device code was built with QLORA_CHECKS, else 0.
+cudaError_t launch_checks_selftest(int* result, cudaStream_t stream);
 
 }  // namespace qnf4

@@ -58,7 +58,19 @@ __global__ void __launch_bounds__(160) mbarrier_ring_kernel(int stages, int iter
   atomicAdd(result + 1, read);
 }
 
+// One thread runs a test that always fails: a library built with
+// QLORA_CHECKS records QLORA_ERR_CHECK in *result, the default build (where
+// the test compiles away) leaves the 0 written before.
+__global__ void checks_probe_kernel(int* result) { qlora_checked(result, false); }
+
 }  // namespace
+
+cudaError_t launch_checks_selftest(int* result, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(result, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  checks_probe_kernel<<<1, 1, 0, stream>>>(result);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_mbarrier_ring_selftest(int stages, int consumers, int iters, uint64_t limit_ns, int* result,
                                           cudaStream_t stream) {

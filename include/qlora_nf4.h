@@ -372,6 +372,19 @@ qlora_status qlora_selftest_mbarrier_ring(int32_t stages, int32_t consumers, int
                                           int32_t *d_result, void *stream);
 
 /*
+ * Whether the debug checks are live in this library's device code (the pages
+ * have no counterpart).  A library built with QLORA_CHECKS
+ * (libqlora_nf4_checks.so) tests index and alignment conditions before the
+ * accesses they guard and records QLORA_ERR_CHECK in the call's status word
+ * when one fails, skipping the access.  This call runs one such test that
+ * always fails, on no memory but the result word.
+ *   d_result : device int32, 4-byte aligned, overwritten: QLORA_ERR_CHECK in
+ *              the checks library, 0 in the default one.
+ * Returns QLORA_OK once enqueued.
+ */
+qlora_status qlora_selftest_checks(int32_t *d_result, void *stream);
+
+/*
  * LoRA linear backward for upstream gradient dY of Y.
  *   X, dY      : bf16 [M, K] and [M, N].
  *   U          : fp32 [M, r] = X A^T as saved by qlora_linear_fwd, or NULL to

@@ -32,6 +32,9 @@ def _quantize(W, codebook, fmt):
 
 def run(out_path: str) -> None:
     res = {}
+    probe = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    binding.qlora_selftest_checks(probe)
+    res["checks_probe"] = probe.cpu()
     formats = [(cb, sf) for cb in (binding.CODEBOOK_NF4, binding.CODEBOOK_FP4)
                for sf in (binding.SCALES_DQ_INT8, binding.SCALES_DQ_FP8, binding.SCALES_FP32)]
     for cb, sf in formats:

@@ -77,6 +77,7 @@ def test_ring_selftest_arguments_checked_on_the_host(lib):
                  (2, 1, (1 << 24) + 1, 1000), (2, 1, 16, 0), (2, 1, 16, 1000001)):
         assert f(*args, buf, None) == 1, args
     assert f(2, 1, 16, 1000, None, None) == 1
+    assert lib.qlora_selftest_checks(None, None) == 1
 
 
 def test_sizes(lib):

@@ -40,6 +40,9 @@ def test_checks_build_matches_default_build(tmp_path):
     ref = _run(default_lib, str(tmp_path / "default.pt"))
     chk = _run(checks_lib, str(tmp_path / "checks.pt"))
     assert sorted(ref) == sorted(chk)
+    # The checks are live in the debug library's device code, compiled away in the default one.
+    assert int(ref.pop("checks_probe")) == 0
+    assert int(chk.pop("checks_probe")) == 8  # QLORA_ERR_CHECK
     for key in ref:
         if key.endswith("/status"):
             assert int(chk[key]) == 0, f"{key}: status {int(chk[key])} under the checks build"
