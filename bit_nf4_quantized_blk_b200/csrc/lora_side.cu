@@ -19,6 +19,9 @@
 //                  V = G B and the dB partials G^T U on the tensor cores),
 //                  forms s*V, the hi/lo split of V and dB = s * (sum of the
 //                  partials).
+// The two reductions that precede a 4-bit GEMM (skinny_finalize_kernel for U
+// in the forward, vdb_finalize_kernel in the backward) also run the GEMM's
+// block-scale job (BlockScalesJob) on further threads of their launch.
 // Deterministic: every sum runs in a fixed order; no atomics.
 #include "common.cuh"
 #include "kernels.cuh"
